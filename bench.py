@@ -1,0 +1,375 @@
+"""Benchmark of the MoE SwiGLU forward layer (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is one pass of the whole layer (route, dispatch, expert GEMMs, shared
+expert, combine) over one batch of synthetic tokens of the workload, inputs
+resident in HBM.  `value` = tokens processed by all ranks / max-over-ranks
+device time.  Under torchrun each rank runs its own batch with replicated
+weights (data parallel, no collective on the data path): weak scaling.
+
+`--impl reference` times the float64 CPU oracle on a bounded sample of the
+same workload (rank 0 only; other ranks exit at once).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE fwd tokens/s (T=4096,D=4096,E=8,top-2,bf16); % of tensor/HBM roofline"
+DEFAULT_WORKLOAD = "mixtral_bf16"
+
+
+def describe(p) -> str:
+    s = f"{p.name}: T={p.T} D={p.D} F={p.F} E={p.E} top-{p.k} act={p.act} experts={p.wdtype} gate={p.gate}"
+    if p.capacity_factor:
+        s += f" cf={p.capacity_factor}"
+    if p.clamp:
+        s += f" clamp={p.clamp}"
+    if p.Fs:
+        s += f" shared_F={p.Fs}"
+    return s
+
+
+def layer_flops(p, rows: int) -> float:
+    """Algorithmic FLOPs of one layer pass: router 2TDE, experts 6 rows D F, shared 6 T D Fs."""
+    return 2.0 * p.T * p.D * p.E + 6.0 * rows * p.D * p.F + 6.0 * p.T * p.D * p.Fs
+
+
+def layer_bytes(p) -> float:
+    """Algorithmic bytes: every weight once, x in, out back."""
+    a = 4 if p.act == "f32" else 2
+    we = {"f32": 4.0, "bf16": 2.0, "nvfp4": 0.5 + 1.0 / 16}[p.wdtype]
+    return (3.0 * p.E * p.F * p.D * we + p.E * p.D * a + 3.0 * p.Fs * p.D * a + 2.0 * p.T * p.D * a)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
+
+
+def gemm_sources_sha() -> str:
+    h = hashlib.sha256()
+    for n in ("gemm_tc.cu", "gemm_simt.cu", "tc_ptx.cuh", "api.cu"):
+        p = os.path.join(ROOT, "mixture_experts_layer_sqrt_b200", "csrc", n)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_key: str):
+    """DRAM bytes per launch recorded from an ncu capture, if the kernel sources are unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = gemm_sources_sha()
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 3 and parts[0] == kernel_key and parts[1] == want:
+            return float(parts[2])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(p, arrays, n_tokens: int, seed: int):
+    """The float64 oracle on a bounded sample: routing and dispatch of every
+    token (capacity needs them), the expert FFN and combine for n_tokens."""
+    import oracle.moe_oracle as O
+    L = O.StoredLayer(arrays, p.act, p.wdtype)
+    t0 = time.perf_counter()
+    logits = O.router_logits(L.x(), L.w_router())
+    idx, w, _ = O.route(logits, p.k, p.gate, arrays.get("bias"), arrays.get("bias_vl"), arrays.get("image_mask"))
+    C = O.expert_capacity(p.T, p.k, p.E, p.capacity_factor)
+    toks = np.random.default_rng(seed).choice(p.T, size=n_tokens, replace=False)
+    O.moe_forward(L.x(), logits, idx, w, L.expert, p.E, C, p.clamp, "preact", L.shared(), tokens=toks)
+    return time.perf_counter() - t0
+
+
+# --------------------------------------------------------------------- ours
+
+def run_ours(args, p, rank, world, local_rank):
+    import torch
+    from mixture_experts_layer_sqrt_b200 import binding as B, synth, workload as WL
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    arrays = synth.generate(p)
+    if rank > 0:  # each rank its own tokens, same weights
+        arrays["x"] = synth.generate(p.with_(seed=p.seed + 1000 * rank), experts=False)["x"]
+    cfg = WL.config_of(p)
+    wt = WL.device_weights(p, arrays, dev)
+    w = B.make_weights(wt)
+    x = WL.to_torch(arrays["x"], dev)
+    mask = WL.to_torch(arrays.get("image_mask"), dev)
+    T, k, D = p.T, p.k, p.D
+    act = torch.float32 if p.act == "f32" else torch.bfloat16
+    # preallocated stage buffers
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    tw = torch.empty((T, k), dtype=torch.float32, device=dev)
+    disp = dict(expert_counts=torch.empty(p.E, dtype=torch.int32, device=dev),
+                expert_offsets=torch.empty(p.E + 1, dtype=torch.int32, device=dev),
+                slot_row=torch.empty((T, k), dtype=torch.int32, device=dev),
+                row_token=torch.empty(T * k, dtype=torch.int32, device=dev),
+                row_weight=torch.empty(T * k, dtype=torch.float32, device=dev),
+                x_perm=torch.empty((T * k, D), dtype=act, device=dev))
+    h = torch.empty((max(T * k * p.F, T * p.Fs),), dtype=act, device=dev)
+    y = torch.empty((T * k, D), dtype=act, device=dev)
+    shy = torch.empty((T, D), dtype=act, device=dev) if p.Fs else None
+    out = torch.empty((T, D), dtype=act, device=dev)
+    ws_d = B.workspace(B.dispatch_workspace_size(cfg, T), dev)
+    ws_e = B.workspace(B.expert_workspace_size(cfg), dev)
+    scfg = B.make_config(E=1, k=1, D=D, F=max(p.Fs, 1), clamp=p.clamp, act=p.act, expert=p.act) if p.Fs else None
+    ws_s = B.workspace(B.expert_workspace_size(scfg), dev) if p.Fs else None
+    stream = torch.cuda.current_stream(dev)
+    hF = h[:T * k * p.F].view(T * k, p.F)
+
+    def step(ev=None):
+        B.route_topk(cfg, x, w, mask, idx, tw)
+        B.dispatch(cfg, x, idx, tw, disp, ws_d)
+        if ev is not None:
+            ev[0].record(stream)
+        B.expert_gate_up(cfg, disp["x_perm"], disp["expert_offsets"], wt["w_gate"], wt["w_up"],
+                         wt.get("s_gate"), wt.get("s_up"), hF, ws_e)
+        if ev is not None:
+            ev[1].record(stream)
+        B.expert_down(cfg, hF, disp["expert_offsets"], wt["w_down"], wt.get("s_down"), disp["row_weight"], y, ws_e)
+        if p.Fs:
+            hs = h[:T * p.Fs].view(T, p.Fs)
+            B.expert_gate_up(scfg, x, None, wt["sh_gate"], wt["sh_up"], None, None, hs, ws_s)
+            B.expert_down(scfg, hs, None, wt["sh_down"], None, None, shy, ws_s)
+        B.combine(cfg, y, disp["slot_row"], T, shy, out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    B.check_device_status(ws_e)
+    rows = int(disp["expert_offsets"][-1].item())
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler("GPU-" + str(props.uuid)) if rank == 0 else None
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = B.launch_count()
+    step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    g_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    step_ev[0].record(stream)
+    for i in range(args.steps):
+        step(g_ev[i])
+        step_ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    n_launch = B.launch_count() - n0
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    total_ms = step_ev[0].elapsed_time(step_ev[-1])
+    per_step = [step_ev[i].elapsed_time(step_ev[i + 1]) for i in range(args.steps)]
+    gemm_ms = sum(a.elapsed_time(b) for a, b in g_ev) / args.steps
+    B.check_device_status(ws_e)
+    t_max = total_ms
+    if dist:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt.item())
+    ms = t_max / args.steps
+    value = world * T / (ms / 1e3)
+
+    # end to end through the public API: pinned host x in, host out back
+    layer = B.MoELayer(cfg, wt, T, dev)
+    x_h = WL.to_torch(arrays["x"], "cpu", pin=True)
+    m_h = WL.to_torch(arrays.get("image_mask"), "cpu", pin=True)
+    out_h = torch.empty((T, D), dtype=act).pin_memory()
+    x_d = torch.empty_like(x_h, device=dev)
+    m_d = torch.empty_like(m_h, device=dev) if m_h is not None else None
+    out_d = torch.empty((T, D), dtype=act, device=dev)
+    for _ in range(max(1, args.warmup)):
+        layer.forward_host(x_h, out_h, m_h, x_d, out_d, m_d)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        layer.forward_host(x_h, out_h, m_h, x_d, out_d, m_d)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    B.check_device_status(layer.ws)
+    e2e = {"value": world * T / (e2e_ms / args.steps / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(x_h.numel() * x_h.element_size() + (m_h.numel() if m_h is not None else 0)),
+           "d2h_bytes_per_step": int(out_h.numel() * out_h.element_size())}
+
+    if rank != 0:
+        return None
+    peaks = load_peaks()
+    flops = layer_flops(p, rows)
+    gemm1_flops = 4.0 * rows * p.D * p.F
+    peak_t = peaks["bf16_sustained"]
+    achieved = gemm1_flops / (gemm_ms / 1e3) / 1e12
+    ideal_ms = max(flops / (peaks["bf16_sustained"] * 1e12), layer_bytes(p) / (peaks["hbm"] * 1e9)) * 1e3
+    res = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32" if p.act == "f32" else "bf16", "data": "synthetic",
+        "config": {"workload": describe(p), "tokens_per_gpu": T, "rows_after_capacity": rows,
+                   "parallelism": f"dp{world} (independent token batches, replicated weights)",
+                   "l2": "inputs larger than L2: expert weights %.2f GB streamed every step" % (layer_bytes(p) / 1e9)},
+        "latency_ms": {"p50": float(np.percentile(per_step, 50)), "p95": float(np.percentile(per_step, 95)),
+                       "p99": float(np.percentile(per_step, 99))},
+        "layer_roofline": {"ideal_ms": ideal_ms, "frac": ideal_ms / ms, "flops": flops, "bytes": layer_bytes(p),
+                           "peak": f"bf16 sustained {peak_t} TFLOP/s, HBM {peaks['hbm']} GB/s ({peaks['src']})"},
+        "roofline": {"kernel": "grouped gate/up GEMM + SwiGLU epilogue", "bound": "tensor",
+                     "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s", "frac": achieved / peak_t,
+                     "peak_kind": f"bf16_tflops_sustained of {peaks['src']}",
+                     "flops_per_launch": gemm1_flops, "ms_per_launch": gemm_ms,
+                     "traffic": profiled_traffic("gate_up_" + p.name)},
+        "e2e": e2e,
+        "gpu_launches": int(n_launch),
+        "clocks": clocks,
+    }
+    return res
+
+
+def cpu_baseline_leg(p, n_tokens=8):
+    from mixture_experts_layer_sqrt_b200 import synth
+    arrays = synth.generate(p)
+    el = oracle_sample(p, arrays, n_tokens, seed=1)
+    return {"value": n_tokens / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"float64 numpy oracle: route + dispatch of all {p.T} tokens, expert FFN + combine "
+                      f"for {n_tokens} sampled tokens, {el:.1f} s"}
+
+
+def run_reference(args, p):
+    from mixture_experts_layer_sqrt_b200 import synth
+    arrays = synth.generate(p)
+    n_tok = 4
+    for i in range(args.warmup):
+        oracle_sample(p, arrays, n_tok, seed=100 + i)
+    times = [oracle_sample(p, arrays, n_tok, seed=i) for i in range(args.steps)]
+    ms = 1e3 * sum(times) / len(times)
+    value = n_tok / (ms / 1e3)
+    sample = (f"float64 numpy oracle per step: route + dispatch of all {p.T} tokens, expert FFN + combine "
+              f"for {n_tok} sampled tokens")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(p), "tokens_per_step": n_tok},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    from mixture_experts_layer_sqrt_b200 import synth
+    p = synth.PROBLEMS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, p)), flush=True)
+        return
+
+    from mixture_experts_layer_sqrt_b200 import build
+    build.build()
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, p, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline_leg(p)
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,230 @@
+/*
+ * moe.h -- C ABI of libmoe_b200.so: forward pass of a Mixture-of-Experts
+ * SwiGLU FFN layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer (sources are web pages on the subject, cited by title and section):
+ *
+ *   logits  r = W_r x                     "FFN、SwiGLU 与 MoE" sec. 3; ops-transformer
+ *                                          MoE walkthrough, MoEForward step 1 / 优化一
+ *   gate    softmax + top-k renormalised  "FFN、SwiGLU 与 MoE" sec. 3 (example module)
+ *           or sqrt(softplus(s)) raw,     "5A · MoE fine-grained" sec. 1 (DeepSeek-V4.1-Flash
+ *           selection on s + bias/bias_vl  course): selection separated from weighting
+ *   dispatch group tokens by expert,      ops-transformer walkthrough, MoEForward step 3,
+ *           capacity drops in token order  坑一 (expert capacity)
+ *   experts y = W_down[SiLU(W_gate x) * (W_up x)], optional +-clamp, optional shared
+ *           expert                         "FFN、SwiGLU 与 MoE" sec. 2; "5A" sec. 1, 3
+ *   combine out[t] = sum_j w_j y_j (+ shared)
+ *                                          ops-transformer MoEForward step 4 (WeightedSum);
+ *                                          Echo MoE quick reference, "Combine"
+ *
+ * Conventions for every entry point:
+ *  - Pointers named in the argument lists are DEVICE pointers owned by the
+ *    caller, unless documented as host.  The library allocates and frees no
+ *    memory; scratch comes from the caller's workspace `ws`.
+ *  - Tensors are dense row-major (last index fastest), 16-byte aligned.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  Argument errors are detected on the host and returned
+ *    synchronously, before anything is enqueued.  Device-side errors (a
+ *    bounded wait inside a kernel that gave up) are recorded in the status
+ *    word at the start of `ws`; read them with moe_check_device_status().
+ *  - Nothing is kept between calls: no global state besides a launch counter.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,    /* null pointer, bad size, k > E, misaligned pointer */
+  MOE_ERR_UNSUPPORTED = 2,    /* valid but not implemented (dtype combination, E too large) */
+  MOE_ERR_WORKSPACE = 3,      /* ws_bytes smaller than the matching *_workspace_size() */
+  MOE_ERR_CUDA = 4,           /* a CUDA runtime call failed (launch error, no device) */
+  MOE_ERR_DEVICE_TIMEOUT = 5  /* a kernel's bounded wait expired; results are invalid */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_NVFP4 = 2 } moe_dtype;
+
+typedef enum {
+  /* p = softmax(r) over all experts, top-k of p, divided by the selected sum
+   * ("FFN、SwiGLU 与 MoE" sec. 3).  An optional per-expert bias is a router
+   * LOGIT bias: r_e + bias[e] enters both the selection and the weights. */
+  MOE_GATE_SOFTMAX_TOPK_RENORM = 0,
+  /* selection: top-k of s_e + bias_vl[e] at image positions, s_e + bias[e]
+   * elsewhere; multiplier: sqrt(softplus(s_e)) of the raw score, not
+   * normalised ("5A · MoE fine-grained" sec. 1, 3). */
+  MOE_GATE_SQRT_SOFTPLUS_RAW = 1
+} moe_gate;
+
+typedef enum {
+  MOE_CLAMP_PREACT = 0, /* clip g = W_gate x and u = W_up x to [-L, L], then SiLU(g) * u */
+  MOE_CLAMP_OUTPUT = 1  /* clip h = SiLU(g) * u to [-L, L] */
+} moe_clamp_mode;
+
+/* Layer configuration.  The first five fields are the ops-transformer
+ * walkthrough's MoEConfig ("MoE的核心思路" section). */
+typedef struct {
+  int num_experts;             /* E, 1..1024 */
+  int top_k;                   /* k, 1..min(E, 16) */
+  int expert_capacity;         /* C: max kept assignments per expert; 0 = unlimited */
+  int hidden_dim;              /* D */
+  int intermediate_dim;        /* F (routed experts) */
+  int shared_intermediate_dim; /* F_s of the always-on shared expert; 0 = none */
+  moe_gate gate;
+  float swiglu_clamp;          /* L; 0 = no clamp */
+  moe_clamp_mode clamp_mode;
+  moe_dtype act_dtype;         /* x, router weights, shared-expert weights, every
+                                  intermediate and out: MOE_F32 or MOE_BF16 */
+  moe_dtype expert_dtype;      /* routed expert weights: MOE_F32 (only with F32
+                                  activations), MOE_BF16 or MOE_NVFP4 (BF16 activations) */
+} MoEConfig;
+
+/* Weights.  Matrices are in nn.Linear layout (out_features x in_features), so
+ * the reduction dimension is the last one ("K-major").  NVFP4 matrices are
+ * stored as two e2m1 codes per byte (even K index in the low nibble) plus one
+ * e4m3 scale byte per 16 consecutive K elements: value = e2m1 * e4m3. */
+typedef struct {
+  const void *w_router;        /* [E, D] act dtype (no router bias) */
+  const void *w_gate;          /* [E, F, D]   (NVFP4: uint8 [E, F, D/2]) */
+  const void *w_up;            /* [E, F, D]   (NVFP4: uint8 [E, F, D/2]) */
+  const void *w_down;          /* [E, D, F]   (NVFP4: uint8 [E, D, F/2]) */
+  const void *s_gate;          /* NVFP4 only: e4m3 [E, F, D/16] */
+  const void *s_up;            /* NVFP4 only: e4m3 [E, F, D/16] */
+  const void *s_down;          /* NVFP4 only: e4m3 [E, D, F/16] */
+  const void *sh_gate;         /* [F_s, D] act dtype (shared expert) */
+  const void *sh_up;           /* [F_s, D] */
+  const void *sh_down;         /* [D, F_s] */
+  const float *bias;           /* [E] or NULL: softmax mode logit bias / sqrt mode selection bias */
+  const float *bias_vl;        /* [E] or NULL: sqrt mode selection bias at image positions */
+} MoEWeights;
+
+/* ------------------------------------------------------------------ misc */
+
+/* Human-readable name of a status code (static string). */
+const char *moe_status_string(moe_status s);
+
+/* Library version string (static). */
+const char *moe_version(void);
+
+/* C = ceil(T * k * cf / E) with cf = cf_num / cf_den, in exact integer
+ * arithmetic (ops-transformer walkthrough, 坑一: capacity = S*top_k/E*1.2,
+ * here rounded up).  Returns 0 (unlimited) when cf_num <= 0, -1 on bad input. */
+int moe_expert_capacity(int T, int top_k, int num_experts, int cf_num, int cf_den);
+
+/* Kernels launched by this library in this process so far (diagnostic). */
+uint64_t moe_launch_count(void);
+
+/* Synchronises `stream`, then reads and clears the device status word at the
+ * start of `ws` (any workspace passed to the calls above).  Returns MOE_OK or
+ * MOE_ERR_DEVICE_TIMEOUT; MOE_ERR_CUDA if the stream reports an error. */
+moe_status moe_check_device_status(void *ws, moe_stream_t stream);
+
+/* ------------------------------------------------------------ stage 1: route */
+
+/* Router GEMM + gate + top-k for T tokens (a1-a2).
+ *   x          [T, D] act dtype
+ *   w->w_router, w->bias, w->bias_vl as in MoEWeights (other fields unused)
+ *   image_mask [T] uint8 (nonzero = image position) or NULL; sqrt gate only
+ *   topk_idx   [T, k] int32 out: selected experts, descending selection key,
+ *              equal keys ordered by lower expert index
+ *   topk_w     [T, k] float out: the multipliers (renormalised softmax, or raw
+ *              sqrt(softplus(s)))
+ * Logits are accumulated in fp32 (ops-transformer walkthrough, 坑三). */
+moe_status moe_route_topk(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
+                          const uint8_t *image_mask, int32_t *topk_idx, float *topk_w,
+                          moe_stream_t stream);
+
+/* --------------------------------------------------------- stage 2: dispatch */
+
+/* Bytes of workspace moe_dispatch needs for T tokens. */
+size_t moe_dispatch_workspace_size(const MoEConfig *cfg, int T);
+
+/* Histogram, scan, capacity and permute (a3-a5).  Assignment (t, j) with
+ * expert e = topk_idx[t, j] gets position p = number of assignments of e
+ * from tokens t' < t; it is kept iff C == 0 or p < C, and then lands in
+ * row expert_offsets[e] + p of x_perm.
+ *   expert_counts  [E] int32 out: assignments per expert before capacity
+ *   expert_offsets [E+1] int32 out: prefix sums of the kept counts; R =
+ *                  expert_offsets[E] rows are used (R <= T*k)
+ *   slot_row       [T, k] int32 out: row of (t, j), or -1 if dropped
+ *   row_token      [T*k] int32 out: token of each row (first R valid)
+ *   row_weight     [T*k] float out: topk_w of each row (first R valid)
+ *   x_perm         [T*k, D] act dtype out: x_perm[r] = x[row_token[r]], r < R
+ *   ws             >= moe_dispatch_workspace_size(cfg, T) bytes
+ * Deterministic: no global atomics; counts and rows are identical run to run. */
+moe_status moe_dispatch(const MoEConfig *cfg, int T, const int32_t *topk_idx, const float *topk_w,
+                        const void *x, int32_t *expert_counts, int32_t *expert_offsets,
+                        int32_t *slot_row, int32_t *row_token, float *row_weight, void *x_perm,
+                        void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------- stage 3: experts */
+
+/* Bytes of workspace moe_grouped_swiglu needs for up to `rows` rows. */
+size_t moe_grouped_swiglu_workspace_size(const MoEConfig *cfg, int rows);
+/* Bytes of workspace moe_expert_gate_up / moe_expert_down need (status word). */
+size_t moe_expert_workspace_size(const MoEConfig *cfg);
+
+/* Grouped gate/up GEMM with the SwiGLU epilogue (a6).  For every expert e and
+ * row r in [expert_offsets[e], expert_offsets[e+1]):
+ *   h[r, :] = SiLU(clip(x_perm[r] W_gate[e]^T)) * clip(x_perm[r] W_up[e]^T)
+ * (clip per cfg->swiglu_clamp / clamp_mode), fp32 accumulation, stored in the
+ * act dtype.  expert_offsets == NULL means one group of `rows` rows using
+ * expert 0's weights.  `rows` bounds every offset (R <= rows).
+ *   w_gate/w_up [E, F, D] in cfg->expert_dtype; s_gate/s_up NVFP4 scales or NULL
+ *   h           [rows, F] out */
+moe_status moe_expert_gate_up(const MoEConfig *cfg, int rows, const void *x_perm,
+                              const int32_t *expert_offsets, const void *w_gate, const void *w_up,
+                              const void *s_gate, const void *s_up, void *h, void *ws,
+                              size_t ws_bytes, moe_stream_t stream);
+
+/* Grouped down GEMM with the routing-weight epilogue (a7):
+ *   y[r, :] = row_weight[r] * (h[r] W_down[e]^T)   (row_weight NULL = 1)
+ *   w_down [E, D, F] in cfg->expert_dtype; s_down NVFP4 scales or NULL
+ *   y      [rows, D] act dtype out */
+moe_status moe_expert_down(const MoEConfig *cfg, int rows, const void *h,
+                           const int32_t *expert_offsets, const void *w_down, const void *s_down,
+                           const float *row_weight, void *y, void *ws, size_t ws_bytes,
+                           moe_stream_t stream);
+
+/* Both expert GEMMs: x_perm -> y_perm through h held in `ws` (a6 + a7). */
+moe_status moe_grouped_swiglu(const MoEConfig *cfg, int rows, const void *x_perm,
+                              const int32_t *expert_offsets, const MoEWeights *w,
+                              const float *row_weight, void *y_perm, void *ws, size_t ws_bytes,
+                              moe_stream_t stream);
+
+/* ---------------------------------------------------------- stage 4: combine */
+
+/* out[t, :] = sum_{j=0..k-1, slot_row[t,j] >= 0} y_perm[slot_row[t, j], :]
+ *             (+ shared_y[t, :] when shared_y != NULL)                  (a9)
+ * Sums in fp32 in the fixed order j = 0..k-1, then the shared term; output in
+ * the act dtype.  Deterministic.  y_perm rows already carry their weights. */
+moe_status moe_combine(const MoEConfig *cfg, int T, const void *y_perm, const int32_t *slot_row,
+                       const void *shared_y, void *out, moe_stream_t stream);
+
+/* ------------------------------------------------------------- whole layer */
+
+/* Bytes of workspace moe_forward needs for T tokens. */
+size_t moe_workspace_size(const MoEConfig *cfg, int T);
+
+/* The whole layer: route, dispatch, experts, shared expert, combine.
+ *   x [T, D], out [T, D] act dtype; image_mask as in moe_route_topk
+ *   topk_idx_out [T, k] int32 or NULL: copy of the routing decision
+ *   expert_counts_out [E] int32 or NULL: assignments per expert before capacity
+ *   ws: workspace of at least moe_workspace_size(cfg, T) bytes
+ * No host synchronisation; per-expert counts never leave the device. */
+moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
+                       const uint8_t *image_mask, void *out, int32_t *topk_idx_out,
+                       int32_t *expert_counts_out, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

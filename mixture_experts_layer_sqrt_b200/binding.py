@@ -1,0 +1,284 @@
+"""Thin ctypes binding of libmoe_b200.so (the C ABI in include/moe.h).
+
+Argument marshalling only: torch tensors provide device memory and the
+current CUDA stream; every step of the layer runs in the library's kernels.
+Importing this module loads the library and raises if it is missing; there is
+no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_float, c_int, c_size_t, c_uint64, c_void_p
+from typing import Dict, Optional
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+
+# enums (include/moe.h)
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE_TIMEOUT = range(6)
+MOE_F32, MOE_BF16, MOE_NVFP4 = range(3)
+MOE_GATE_SOFTMAX_TOPK_RENORM, MOE_GATE_SQRT_SOFTPLUS_RAW = range(2)
+MOE_CLAMP_PREACT, MOE_CLAMP_OUTPUT = range(2)
+
+DTYPES = {"f32": MOE_F32, "bf16": MOE_BF16, "nvfp4": MOE_NVFP4}
+GATES = {"softmax": MOE_GATE_SOFTMAX_TOPK_RENORM, "sqrt_softplus": MOE_GATE_SQRT_SOFTPLUS_RAW}
+CLAMP_MODES = {"preact": MOE_CLAMP_PREACT, "output": MOE_CLAMP_OUTPUT}
+
+
+class MoEConfig(ctypes.Structure):
+    _fields_ = [("num_experts", c_int), ("top_k", c_int), ("expert_capacity", c_int),
+                ("hidden_dim", c_int), ("intermediate_dim", c_int),
+                ("shared_intermediate_dim", c_int), ("gate", c_int), ("swiglu_clamp", c_float),
+                ("clamp_mode", c_int), ("act_dtype", c_int), ("expert_dtype", c_int)]
+
+
+class MoEWeights(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in ("w_router", "w_gate", "w_up", "w_down", "s_gate", "s_up",
+                                        "s_down", "sh_gate", "sh_up", "sh_down", "bias", "bias_vl")]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m mixture_experts_layer_sqrt_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, S = c_void_p, c_int, c_size_t
+    cfgp, wp = POINTER(MoEConfig), POINTER(MoEWeights)
+    sig = {
+        "moe_status_string": (c_char_p, [I]),
+        "moe_version": (c_char_p, []),
+        "moe_expert_capacity": (I, [I, I, I, I, I]),
+        "moe_launch_count": (c_uint64, []),
+        "moe_check_device_status": (I, [P, P]),
+        "moe_route_topk": (I, [cfgp, I, P, wp, P, P, P, P]),
+        "moe_dispatch_workspace_size": (S, [cfgp, I]),
+        "moe_dispatch": (I, [cfgp, I, P, P, P, P, P, P, P, P, P, P, S, P]),
+        "moe_grouped_swiglu_workspace_size": (S, [cfgp, I]),
+        "moe_expert_workspace_size": (S, [cfgp]),
+        "moe_expert_gate_up": (I, [cfgp, I, P, P, P, P, P, P, P, P, S, P]),
+        "moe_expert_down": (I, [cfgp, I, P, P, P, P, P, P, P, S, P]),
+        "moe_grouped_swiglu": (I, [cfgp, I, P, P, wp, P, P, P, S, P]),
+        "moe_combine": (I, [cfgp, I, P, P, P, P, P]),
+        "moe_workspace_size": (S, [cfgp, I]),
+        "moe_forward": (I, [cfgp, I, P, wp, P, P, P, P, P, S, P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+lib = _load()
+
+# Every function the header declares (checked by the tests).
+EXPORTS = ("moe_status_string", "moe_version", "moe_expert_capacity", "moe_launch_count",
+           "moe_check_device_status", "moe_route_topk", "moe_dispatch_workspace_size",
+           "moe_dispatch", "moe_grouped_swiglu_workspace_size", "moe_expert_workspace_size",
+           "moe_expert_gate_up", "moe_expert_down", "moe_grouped_swiglu", "moe_combine",
+           "moe_workspace_size", "moe_forward")
+
+
+def status_string(s: int) -> str:
+    return lib.moe_status_string(s).decode()
+
+
+def version() -> str:
+    return lib.moe_version().decode()
+
+
+def launch_count() -> int:
+    return int(lib.moe_launch_count())
+
+
+def expert_capacity(T: int, k: int, E: int, cf_num: int, cf_den: int) -> int:
+    return int(lib.moe_expert_capacity(T, k, E, cf_num, cf_den))
+
+
+def _check(st: int, where: str):
+    if st != MOE_OK:
+        raise MoEError(st, where)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def make_config(E: int, k: int, D: int, F: int, capacity: int = 0, Fs: int = 0, gate="softmax",
+                clamp: float = 0.0, clamp_mode="preact", act="bf16", expert="bf16") -> MoEConfig:
+    return MoEConfig(E, k, capacity, D, F, Fs, GATES[gate], clamp, CLAMP_MODES[clamp_mode],
+                     DTYPES[act], DTYPES[expert])
+
+
+def make_weights(t: Dict[str, Optional[torch.Tensor]]) -> MoEWeights:
+    """MoEWeights from device tensors keyed like the struct fields (missing = NULL)."""
+    return MoEWeights(*[_p(t.get(n)) for n, _ in MoEWeights._fields_])
+
+
+def workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zeroed device workspace (the status word must start at zero)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+# ------------------------------------------------------------------ stages
+
+def route_topk(cfg: MoEConfig, x: torch.Tensor, w: MoEWeights, image_mask=None,
+               topk_idx=None, topk_w=None, stream=None):
+    T = x.shape[0]
+    if topk_idx is None:
+        topk_idx = torch.empty((T, cfg.top_k), dtype=torch.int32, device=x.device)
+    if topk_w is None:
+        topk_w = torch.empty((T, cfg.top_k), dtype=torch.float32, device=x.device)
+    _check(lib.moe_route_topk(ctypes.byref(cfg), T, _p(x), ctypes.byref(w), _p(image_mask),
+                              _p(topk_idx), _p(topk_w), _stream(stream)), "moe_route_topk")
+    return topk_idx, topk_w
+
+
+def dispatch(cfg: MoEConfig, x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,
+             out: Optional[Dict[str, torch.Tensor]] = None, ws: Optional[torch.Tensor] = None,
+             stream=None) -> Dict[str, torch.Tensor]:
+    T, D, E, k = x.shape[0], cfg.hidden_dim, cfg.num_experts, cfg.top_k
+    dev = x.device
+    o = out or dict(
+        expert_counts=torch.empty(E, dtype=torch.int32, device=dev),
+        expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+        slot_row=torch.empty((T, k), dtype=torch.int32, device=dev),
+        row_token=torch.empty(T * k, dtype=torch.int32, device=dev),
+        row_weight=torch.empty(T * k, dtype=torch.float32, device=dev),
+        x_perm=torch.empty((T * k, D), dtype=x.dtype, device=dev))
+    if ws is None:
+        ws = workspace(lib.moe_dispatch_workspace_size(ctypes.byref(cfg), T), dev)
+    _check(lib.moe_dispatch(ctypes.byref(cfg), T, _p(topk_idx), _p(topk_w), _p(x),
+                            _p(o["expert_counts"]), _p(o["expert_offsets"]), _p(o["slot_row"]),
+                            _p(o["row_token"]), _p(o["row_weight"]), _p(o["x_perm"]), _p(ws),
+                            ws.numel(), _stream(stream)), "moe_dispatch")
+    return o
+
+
+def expert_gate_up(cfg: MoEConfig, x_perm: torch.Tensor, offsets: Optional[torch.Tensor], w_gate, w_up,
+                   s_gate=None, s_up=None, h=None, ws=None, rows=None, stream=None) -> torch.Tensor:
+    rows = x_perm.shape[0] if rows is None else rows
+    if h is None:
+        h = torch.empty((rows, cfg.intermediate_dim), dtype=x_perm.dtype, device=x_perm.device)
+    if ws is None:
+        ws = workspace(lib.moe_expert_workspace_size(ctypes.byref(cfg)), x_perm.device)
+    _check(lib.moe_expert_gate_up(ctypes.byref(cfg), rows, _p(x_perm), _p(offsets), _p(w_gate), _p(w_up),
+                                  _p(s_gate), _p(s_up), _p(h), _p(ws), ws.numel(), _stream(stream)),
+           "moe_expert_gate_up")
+    return h
+
+
+def expert_down(cfg: MoEConfig, h: torch.Tensor, offsets: Optional[torch.Tensor], w_down, s_down=None,
+                row_weight=None, y=None, ws=None, rows=None, stream=None) -> torch.Tensor:
+    rows = h.shape[0] if rows is None else rows
+    if y is None:
+        y = torch.empty((rows, cfg.hidden_dim), dtype=h.dtype, device=h.device)
+    if ws is None:
+        ws = workspace(lib.moe_expert_workspace_size(ctypes.byref(cfg)), h.device)
+    _check(lib.moe_expert_down(ctypes.byref(cfg), rows, _p(h), _p(offsets), _p(w_down), _p(s_down),
+                               _p(row_weight), _p(y), _p(ws), ws.numel(), _stream(stream)),
+           "moe_expert_down")
+    return y
+
+
+def grouped_swiglu(cfg: MoEConfig, x_perm: torch.Tensor, offsets, w: MoEWeights, row_weight=None,
+                   y=None, ws=None, stream=None) -> torch.Tensor:
+    rows = x_perm.shape[0]
+    if y is None:
+        y = torch.empty((rows, cfg.hidden_dim), dtype=x_perm.dtype, device=x_perm.device)
+    if ws is None:
+        ws = workspace(lib.moe_grouped_swiglu_workspace_size(ctypes.byref(cfg), rows), x_perm.device)
+    _check(lib.moe_grouped_swiglu(ctypes.byref(cfg), rows, _p(x_perm), _p(offsets), ctypes.byref(w),
+                                  _p(row_weight), _p(y), _p(ws), ws.numel(), _stream(stream)),
+           "moe_grouped_swiglu")
+    return y
+
+
+def combine(cfg: MoEConfig, y_perm: torch.Tensor, slot_row: torch.Tensor, T: int, shared_y=None,
+            out=None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((T, cfg.hidden_dim), dtype=y_perm.dtype, device=y_perm.device)
+    _check(lib.moe_combine(ctypes.byref(cfg), T, _p(y_perm), _p(slot_row), _p(shared_y), _p(out),
+                           _stream(stream)), "moe_combine")
+    return out
+
+
+def workspace_size(cfg: MoEConfig, T: int) -> int:
+    return int(lib.moe_workspace_size(ctypes.byref(cfg), T))
+
+
+def dispatch_workspace_size(cfg: MoEConfig, T: int) -> int:
+    return int(lib.moe_dispatch_workspace_size(ctypes.byref(cfg), T))
+
+
+def expert_workspace_size(cfg: MoEConfig) -> int:
+    return int(lib.moe_expert_workspace_size(ctypes.byref(cfg)))
+
+
+def grouped_swiglu_workspace_size(cfg: MoEConfig, rows: int) -> int:
+    return int(lib.moe_grouped_swiglu_workspace_size(ctypes.byref(cfg), rows))
+
+
+def forward(cfg: MoEConfig, x: torch.Tensor, w: MoEWeights, ws: torch.Tensor, image_mask=None,
+            out=None, topk_idx_out=None, expert_counts_out=None, stream=None) -> torch.Tensor:
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, cfg.hidden_dim), dtype=x.dtype, device=x.device)
+    _check(lib.moe_forward(ctypes.byref(cfg), T, _p(x), ctypes.byref(w), _p(image_mask), _p(out),
+                           _p(topk_idx_out), _p(expert_counts_out), _p(ws), ws.numel(), _stream(stream)),
+           "moe_forward")
+    return out
+
+
+def check_device_status(ws: torch.Tensor, stream=None):
+    _check(lib.moe_check_device_status(_p(ws), _stream(stream)), "device status")
+
+
+# ------------------------------------------------------------------ layer
+
+class MoELayer:
+    """A layer whose weights live on the device; forward() is one moe_forward call.
+
+    ``forward_host`` is the end-to-end path: pinned host tokens in, host
+    output back, copies included.
+    """
+
+    def __init__(self, cfg: MoEConfig, weights: Dict[str, Optional[torch.Tensor]], max_tokens: int,
+                 device="cuda"):
+        self.cfg = cfg
+        self.weights = weights            # keeps the tensors alive
+        self.w = make_weights(weights)
+        self.max_tokens = max_tokens
+        self.ws = workspace(workspace_size(cfg, max_tokens), device)
+        self.device = device
+
+    def forward(self, x: torch.Tensor, image_mask=None, out=None, topk_idx_out=None,
+                expert_counts_out=None, stream=None) -> torch.Tensor:
+        if x.shape[0] > self.max_tokens:
+            raise ValueError("more tokens than the workspace was sized for")
+        return forward(self.cfg, x, self.w, self.ws, image_mask, out, topk_idx_out, expert_counts_out, stream)
+
+    def forward_host(self, x_host: torch.Tensor, out_host: torch.Tensor, image_mask_host=None,
+                     x_dev=None, out_dev=None, mask_dev=None) -> torch.Tensor:
+        """Host (pinned) x -> device -> moe_forward -> host out, on the current stream."""
+        x_dev = x_dev if x_dev is not None else torch.empty_like(x_host, device=self.device)
+        x_dev.copy_(x_host, non_blocking=True)
+        if image_mask_host is not None:
+            mask_dev = mask_dev if mask_dev is not None else torch.empty_like(image_mask_host, device=self.device)
+            mask_dev.copy_(image_mask_host, non_blocking=True)
+        out_dev = self.forward(x_dev, mask_dev, out_dev)
+        out_host.copy_(out_dev, non_blocking=True)
+        return out_host

@@ -1,0 +1,220 @@
+// Dispatch: group assignments by expert in token order, apply the expert
+// capacity, and gather the rows of x into expert-contiguous order.
+//
+// ops-transformer MoE walkthrough: MoEForward step 3 ("find the tokens routed
+// to expert e; Gather") and 坑一 (tokens beyond the expert capacity are
+// dropped); Echo MoE quick reference, "Dispatch".
+//
+// Four kernels, no global atomics:
+//   hist    one block per chunk of kChunkTokens tokens: per-chunk expert counts
+//           (shared-memory counters) -> chunk_cnt[c][e]
+//   scan    one block: per expert, exclusive scan of chunk_cnt over chunks
+//           (in place), total count, kept = min(count, C), offsets = prefix of kept
+//   maps    one block per chunk: the rank of each assignment among its
+//           expert's assignments in token order (warp match + per-warp
+//           running counters), -> slot_row, row_token, row_weight
+//   gather  x_perm[r] = x[row_token[r]] with 16-byte vector copies
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+static_assert(kChunkTokens == kWarps * 32, "one warp per 32 tokens of a chunk");
+
+__global__ void __launch_bounds__(kThreads) hist_kernel(int T, int E, int k,
+                                                        const int32_t *__restrict__ topk_idx,
+                                                        int32_t *__restrict__ chunk_cnt) {
+  extern __shared__ int32_t cnt[];  // [E]
+  for (int e = threadIdx.x; e < E; e += kThreads) cnt[e] = 0;
+  __syncthreads();
+  const long a0 = (long)blockIdx.x * kChunkTokens * k;
+  const long a1 = min((long)T * k, a0 + (long)kChunkTokens * k);
+  for (long a = a0 + threadIdx.x; a < a1; a += kThreads) {
+    int e = topk_idx[a];
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kThreads) chunk_cnt[(long)blockIdx.x * E + e] = cnt[e];
+}
+
+// Block-wide exclusive scan of one int per thread (1024 threads).
+__device__ int block_exclusive_scan(int v, int *warp_sums, int &total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    int n = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += n;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int ws = warp_sums[lane];
+    int wi = ws;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      int n = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += n;
+    }
+    warp_sums[lane] = wi - ws;  // exclusive prefix of warp sums
+    if (lane == 31) warp_sums[32] = wi;
+  }
+  __syncthreads();
+  int r = warp_sums[warp] + incl - v;
+  total = warp_sums[32];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(1024) scan_kernel(int n_chunks, int E, int capacity,
+                                                    int32_t *__restrict__ chunk_cnt,
+                                                    int32_t *__restrict__ expert_counts,
+                                                    int32_t *__restrict__ expert_offsets) {
+  __shared__ int warp_sums[33];
+  int carry = 0;
+  for (int e0 = 0; e0 < E; e0 += 1024) {
+    const int e = e0 + threadIdx.x;
+    int kept = 0;
+    if (e < E) {
+      int run = 0;
+      for (int c = 0; c < n_chunks; ++c) {
+        int v = chunk_cnt[(long)c * E + e];
+        chunk_cnt[(long)c * E + e] = run;  // exclusive base of chunk c within expert e
+        run += v;
+      }
+      expert_counts[e] = run;
+      kept = (capacity > 0 && run > capacity) ? capacity : run;
+    }
+    int total;
+    int off = block_exclusive_scan(kept, warp_sums, total);
+    if (e < E) expert_offsets[e] = carry + off;
+    carry += total;
+  }
+  if (threadIdx.x == 0) expert_offsets[E] = carry;
+}
+
+__global__ void __launch_bounds__(kThreads) maps_kernel(int T, int E, int k, int capacity,
+                                                        const int32_t *__restrict__ topk_idx,
+                                                        const float *__restrict__ topk_w,
+                                                        const int32_t *__restrict__ chunk_base,
+                                                        const int32_t *__restrict__ expert_offsets,
+                                                        int32_t *__restrict__ slot_row,
+                                                        int32_t *__restrict__ row_token,
+                                                        float *__restrict__ row_weight) {
+  extern __shared__ int32_t run[];  // [kWarps][E]: running position per warp and expert
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int32_t *my = run + warp * E;
+  for (int i = threadIdx.x; i < kWarps * E; i += kThreads) run[i] = 0;
+  __syncthreads();
+
+  // assignments of this warp: tokens [tw, tw + 32), flat items [tw*k, (tw+32)*k)
+  const long tw = (long)blockIdx.x * kChunkTokens + warp * 32;
+  const long a0 = tw * k;
+  const long a_end = min((long)T * k, a0 + 32L * k);
+  // pass 1: per-warp counts per expert
+  for (long a = a0; a < a0 + 32L * k; a += 32) {
+    long ai = a + lane;
+    int e = ai < a_end ? topk_idx[ai] : -1;
+    if (e >= E) e = -1;
+    unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && (__ffs(peers) - 1) == lane) my[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // warps' bases: chunk base + counts of the lower warps of this chunk
+  for (int e = threadIdx.x; e < E; e += kThreads) {
+    int r = chunk_base[(long)blockIdx.x * E + e];
+    for (int w = 0; w < kWarps; ++w) {
+      int v = run[w * E + e];
+      run[w * E + e] = r;
+      r += v;
+    }
+  }
+  __syncthreads();
+  // pass 2: position of every assignment within its expert, in token order
+  const unsigned lt = (1u << lane) - 1u;
+  for (long a = a0; a < a0 + 32L * k; a += 32) {
+    long ai = a + lane;
+    int e = ai < a_end ? topk_idx[ai] : -1;
+    if (e >= E) e = -1;
+    unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (ai < a_end && e < 0) slot_row[ai] = -1;  // invalid expert index: treated as dropped
+    if (e >= 0) {
+      int pos = my[e] + __popc(peers & lt);
+      if (capacity <= 0 || pos < capacity) {
+        int row = expert_offsets[e] + pos;
+        slot_row[ai] = row;
+        row_token[row] = (int32_t)(ai / k);
+        row_weight[row] = topk_w[ai];
+      } else {
+        slot_row[ai] = -1;
+      }
+    }
+    __syncwarp();
+    if (e >= 0 && (__ffs(peers) - 1) == lane) my[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// One warp per row: x_perm[r] = x[row_token[r]], lanes stride over 16-byte vectors.
+template <typename TA>
+__global__ void __launch_bounds__(256) gather_kernel(int max_rows, int D,
+                                                     const int32_t *__restrict__ expert_offsets,
+                                                     int E, const int32_t *__restrict__ row_token,
+                                                     const TA *__restrict__ x,
+                                                     TA *__restrict__ x_perm) {
+  constexpr int V = Vec16<TA>::N;
+  const int R = min(expert_offsets[E], max_rows);
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += warps) {
+    const TA *src = x + (long)row_token[r] * D;
+    TA *dst = x_perm + (long)r * D;
+#pragma unroll 4
+    for (int c = lane * V; c < D; c += 32 * V) store16(dst + c, load16(src + c));
+  }
+}
+
+}  // namespace
+
+moe_status launch_dispatch(const MoEConfig &c, int T, const int32_t *topk_idx, const float *topk_w,
+                           const void *x, int32_t *expert_counts, int32_t *expert_offsets,
+                           int32_t *slot_row, int32_t *row_token, float *row_weight, void *x_perm,
+                           int32_t *chunk_cnt, cudaStream_t s) {
+  const int E = c.num_experts, k = c.top_k;
+  const int nch = num_chunks(T);
+  if (T == 0) {
+    // still publish empty counts and offsets
+    MOE_CUDA_TRY(cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * E, s));
+    MOE_CUDA_TRY(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), s));
+    return MOE_OK;
+  }
+  hist_kernel<<<nch, kThreads, E * sizeof(int32_t), s>>>(T, E, k, topk_idx, chunk_cnt);
+  MOE_LAUNCH_CHECK();
+  scan_kernel<<<1, 1024, 0, s>>>(nch, E, c.expert_capacity, chunk_cnt, expert_counts, expert_offsets);
+  MOE_LAUNCH_CHECK();
+  size_t maps_smem = (size_t)kWarps * E * sizeof(int32_t);
+  MOE_CUDA_TRY(cudaFuncSetAttribute(maps_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)maps_smem));
+  maps_kernel<<<nch, kThreads, maps_smem, s>>>(T, E, k, c.expert_capacity, topk_idx, topk_w, chunk_cnt,
+                                               expert_offsets, slot_row, row_token, row_weight);
+  MOE_LAUNCH_CHECK();
+  int dev = 0, sms = 148;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const int max_rows = T * k;
+  if (c.act_dtype == MOE_F32) {
+    gather_kernel<float><<<sms * 8, 256, 0, s>>>(max_rows, c.hidden_dim, expert_offsets, E, row_token,
+                                                 (const float *)x, (float *)x_perm);
+  } else {
+    gather_kernel<__nv_bfloat16><<<sms * 8, 256, 0, s>>>(max_rows, c.hidden_dim, expert_offsets, E,
+                                                         row_token, (const __nv_bfloat16 *)x,
+                                                         (__nv_bfloat16 *)x_perm);
+  }
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+}  // namespace moe

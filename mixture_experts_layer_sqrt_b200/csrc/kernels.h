@@ -1,0 +1,47 @@
+// Host-side launchers of the kernels (internal to libmoe_b200).
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// Tokens per dispatch chunk: the histogram and permute kernels work on
+// chunks of this many consecutive tokens.
+constexpr int kChunkTokens = 256;
+inline int num_chunks(int T) { return (T + kChunkTokens - 1) / kChunkTokens; }
+
+// route.cu ---------------------------------------------------------------
+moe_status launch_route(const MoEConfig &c, int T, const void *x, const void *w_router,
+                        const float *bias, const float *bias_vl, const uint8_t *image_mask,
+                        int32_t *topk_idx, float *topk_w, cudaStream_t s);
+
+// dispatch.cu ------------------------------------------------------------
+// chunk_cnt: [num_chunks(T), E] int32 scratch.
+moe_status launch_dispatch(const MoEConfig &c, int T, const int32_t *topk_idx, const float *topk_w,
+                           const void *x, int32_t *expert_counts, int32_t *expert_offsets,
+                           int32_t *slot_row, int32_t *row_token, float *row_weight, void *x_perm,
+                           int32_t *chunk_cnt, cudaStream_t s);
+
+// gemm_simt.cu -----------------------------------------------------------
+// Grouped GEMMs on CUDA cores (fp32 FMA), any shape.  act: F32 or BF16 for
+// activations and weights alike.
+moe_status launch_gate_up_simt(const MoEConfig &c, int rows, const void *a,
+                               const int32_t *offsets, const void *w_gate, const void *w_up,
+                               int F, void *h, cudaStream_t s);
+moe_status launch_down_simt(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
+                            const void *w_down, int F, const float *row_weight, void *y,
+                            cudaStream_t s);
+
+// dequant.cu -------------------------------------------------------------
+// n_elems values (a multiple of 16): packed [n/2] bytes + scales [n/16] -> bf16 [n].
+moe_status launch_dequant_nvfp4(const void *packed, const void *scales, long n_elems, void *out,
+                                cudaStream_t s);
+
+// combine.cu -------------------------------------------------------------
+moe_status launch_combine(const MoEConfig &c, int T, const void *y_perm, const int32_t *slot_row,
+                          const void *shared_y, void *out, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,85 @@
+"""Helpers for the GPU-vs-oracle parity tests (not a test module).
+
+The GPU side goes through the C ABI (binding); the oracle side through
+oracle/moe_oracle.py.  Both read the same stored arrays from synth.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle.moe_oracle as O
+from mixture_experts_layer_sqrt_b200 import synth
+
+NEAR_TIE = 1e-4        # selection-key gap below which a token counts as a near-tie
+F32_RTOL = 1e-5        # fp32 layer: |err_i| <= 1e-5 * max(|ref_i|, rms(ref))
+BF16_RMS_TOL = 2e-2    # bf16 / FP4 layer: max |err| <= 2e-2 * rms(ref)
+ROUTE_W_RTOL = 1e-5    # routing weights, every dtype
+
+
+def small(name: str) -> synth.MoEProblem:
+    """A shrunken copy of workload `name` that keeps its features (gate, dtypes,
+    capacity, bias, shared expert) and spans several 128x128 tiles with ragged
+    tails, small enough for the oracle to finish in seconds."""
+    p = synth.PROBLEMS[name]
+    if name == "tiny_f32":
+        return p
+    kw = dict(T=300, D=512, F=384)
+    if name == "capacity_bf16":
+        kw.update(E=6)
+    elif name == "finegrained_bf16":
+        kw.update(E=16, k=4)
+    elif name == "sqrt_fp4":
+        kw.update(E=12, k=3, Fs=256)
+    else:
+        kw.update(E=6)
+    return p.with_(name=name + "_small", **kw)
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    t = t.detach().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.float().numpy().astype(np.float64)
+    return t.numpy()
+
+
+def oracle_layer(p: synth.MoEProblem, arrays) -> O.StoredLayer:
+    return O.StoredLayer(arrays, p.act, p.wdtype)
+
+
+def oracle_route(p: synth.MoEProblem, L: O.StoredLayer, arrays):
+    logits = O.router_logits(L.x(), L.w_router())
+    idx, w, keys = O.route(logits, p.k, p.gate, arrays.get("bias"), arrays.get("bias_vl"), arrays.get("image_mask"))
+    return logits, idx, w, keys
+
+
+def near_ties(keys: np.ndarray, k: int) -> np.ndarray:
+    """Tokens where any adjacent gap among the k+1 largest keys is below NEAR_TIE
+    (the k-th vs (k+1)-th gap decides the set; the others the slot order)."""
+    srt = -np.sort(-keys, axis=1)[:, :min(k + 1, keys.shape[1])]
+    gaps = srt[:, :-1] - srt[:, 1:]
+    return (gaps < NEAR_TIE).any(axis=1) if gaps.shape[1] else np.zeros(keys.shape[0], bool)
+
+
+def check_route(p, idx_g: np.ndarray, w_g: np.ndarray, logits, idx_o, keys, bias=None):
+    """Indices bit-exact except near-ties; weights of the GPU's own selection
+    within ROUTE_W_RTOL of the oracle's weights for that selection."""
+    nt = near_ties(keys, p.k)
+    diff = (idx_g != idx_o).any(axis=1)
+    bad = diff & ~nt
+    assert not bad.any(), f"{bad.sum()} tokens routed differently with no near-tie, e.g. {np.nonzero(bad)[0][:5]}"
+    w_ref = O.route_weights(logits, idx_g.astype(np.int64), p.gate, bias if p.gate == "softmax" else None)
+    np.testing.assert_allclose(w_g, w_ref, rtol=ROUTE_W_RTOL, atol=1e-7)
+    return int(diff.sum()), int(nt.sum())
+
+
+def assert_close_layer(p, got: np.ndarray, ref: np.ndarray, what: str):
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    err = np.abs(got - ref)
+    if p.act == "f32":
+        lim = F32_RTOL * np.maximum(np.abs(ref), rms)
+        bad = err > lim
+        assert not bad.any(), f"{what}: {bad.sum()} elements above 1e-5 rel, max ratio {(err / lim).max():.3g}"
+    else:
+        assert err.max() <= BF16_RMS_TOL * rms, f"{what}: max|err| {err.max():.4g} > 2e-2 * rms {rms:.4g}"
+    return float(err.max() / max(rms, 1e-30))

@@ -1,0 +1,299 @@
+"""GPU parity: every stage through the C ABI against the float64 oracle.
+
+Small shrunken copies of the five workloads (several tiles, ragged tails) are
+checked element by element; the full-size workloads on sampled tokens (routing
+and dispatch on every token).  Tolerances: indices, counts, rows and copies
+bit-exact (near-ties excepted and reported); routing weights 1e-5 relative;
+fp32 layer 1e-5 relative; bf16/FP4 layer max|err| <= 2e-2 * rms(oracle).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.moe_oracle as O
+from mixture_experts_layer_sqrt_b200 import synth
+from tests import harness as H
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ["tiny_f32", "mixtral_bf16", "capacity_bf16", "finegrained_bf16", "sqrt_fp4"]
+
+
+@pytest.fixture(scope="module")
+def B():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from mixture_experts_layer_sqrt_b200 import build
+    build.build()
+    from mixture_experts_layer_sqrt_b200 import binding
+    return binding
+
+
+@pytest.fixture(scope="module")
+def W(B):
+    from mixture_experts_layer_sqrt_b200 import workload
+    return workload
+
+
+class Case:
+    """One problem: stored arrays, the device copies and the oracle view."""
+
+    def __init__(self, B, W, p, arrays=None, clamp_mode="preact"):
+        self.p = p
+        self.a = arrays if arrays is not None else synth.generate(p)
+        self.cfg = W.config_of(p, clamp_mode)
+        self.clamp_mode = clamp_mode
+        self.wt = W.device_weights(p, self.a)
+        self.w = B.make_weights(self.wt)
+        self.x = W.to_torch(self.a["x"])
+        self.mask = W.to_torch(self.a.get("image_mask"))
+        self.L = H.oracle_layer(p, self.a)
+        self.C = self.cfg.expert_capacity
+
+    def shared_cfg(self, B):
+        p = self.p
+        return B.make_config(E=1, k=1, D=p.D, F=p.Fs, clamp=p.clamp, clamp_mode=self.clamp_mode,
+                             act=p.act, expert=p.act)
+
+
+def _stages(B, c: Case):
+    """Run route, dispatch, gate/up, down, shared expert and combine one by one."""
+    p = c.p
+    idx, w = B.route_topk(c.cfg, c.x, c.w, c.mask)
+    d = B.dispatch(c.cfg, c.x, idx, w)
+    s = {k: c.wt.get(k) for k in ("s_gate", "s_up", "s_down")}
+    h = B.expert_gate_up(c.cfg, d["x_perm"], d["expert_offsets"], c.wt["w_gate"], c.wt["w_up"], s["s_gate"], s["s_up"])
+    y = B.expert_down(c.cfg, h, d["expert_offsets"], c.wt["w_down"], s["s_down"], d["row_weight"])
+    sh = None
+    if p.Fs:
+        sc = c.shared_cfg(B)
+        hs = B.expert_gate_up(sc, c.x, None, c.wt["sh_gate"], c.wt["sh_up"])
+        sh = B.expert_down(sc, hs, None, c.wt["sh_down"])
+    out = B.combine(c.cfg, y, d["slot_row"], p.T, shared_y=sh)
+    torch.cuda.synchronize()
+    return dict(idx=idx, w=w, h=h, y=y, sh=sh, out=out, **d)
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_stages_small(B, W, name):
+    p = H.small(name)
+    c = Case(B, W, p)
+    g = _stages(B, c)
+    idx_g, w_g = H.to_np(g["idx"]), H.to_np(g["w"])
+
+    # a1-a2 route
+    logits, idx_o, w_o, keys = H.oracle_route(p, c.L, c.a)
+    flips, ties = H.check_route(p, idx_g, w_g, logits, idx_o, keys, c.a.get("bias"))
+    print(f"{p.name}: near-ties {ties}, flipped {flips}")
+
+    # a3-a5 dispatch, conditioned on the GPU's selection: bit-exact
+    d = O.dispatch(idx_g.astype(np.int64), p.E, c.C)
+    R = int(d["offsets"][-1])
+    np.testing.assert_array_equal(H.to_np(g["expert_counts"]), d["counts"])
+    np.testing.assert_array_equal(H.to_np(g["expert_offsets"]), d["offsets"])
+    np.testing.assert_array_equal(H.to_np(g["slot_row"]), d["slot_row"])
+    np.testing.assert_array_equal(H.to_np(g["row_token"])[:R], d["row_token"])
+    np.testing.assert_array_equal(H.to_np(g["row_weight"])[:R], w_g[d["row_token"], d["row_slot"]])
+    xp = g["x_perm"][:R].cpu()
+    assert torch.equal(xp, c.x.cpu()[torch.from_numpy(d["row_token"])])
+    if c.C:
+        assert d["drops"] > 0 or p.name.startswith("tiny")
+
+    # a6 gate/up + SwiGLU epilogue, per expert on the GPU's rows
+    x64 = c.L.x()
+    h_g = H.to_np(g["h"])[:R]
+    h_ref = np.zeros_like(h_g)
+    y_ref = np.zeros((R, p.D))
+    for e in range(p.E):
+        r0, r1 = d["offsets"][e], d["offsets"][e + 1]
+        if r1 == r0:
+            continue
+        wg, wu, wd = c.L.expert(e)
+        h_ref[r0:r1] = O.swiglu_hidden(x64[d["row_token"][r0:r1]], wg, wu, p.clamp, c.clamp_mode)
+        # a7 down + weight epilogue, fed with the GPU's own h
+        y_ref[r0:r1] = w_g[d["row_token"][r0:r1], d["row_slot"][r0:r1], None] * (h_g[r0:r1] @ wd.T)
+    H.assert_close_layer(p, h_g, h_ref, "h")
+    y_g = H.to_np(g["y"])[:R]
+    H.assert_close_layer(p, y_g, y_ref, "y_perm")
+
+    # a8 shared expert
+    sh_g = None
+    if p.Fs:
+        sh_g = H.to_np(g["sh"])
+        H.assert_close_layer(p, sh_g, O.swiglu(x64, *c.L.shared(), p.clamp, c.clamp_mode), "shared")
+
+    # a9 combine of the GPU's y (and shared): fp32 sums, one rounding
+    ref = np.zeros((p.T, p.D))
+    for t in range(p.T):
+        for j in range(p.k):
+            r = d["slot_row"][t, j]
+            if r >= 0:
+                ref[t] += y_g[r]
+    if sh_g is not None:
+        ref += sh_g
+    out_g = H.to_np(g["out"])
+    tol = 2.0 ** -8 if p.act == "bf16" else 1e-6
+    assert np.all(np.abs(out_g - ref) <= tol * np.abs(ref) + 1e-6 * np.sqrt(np.mean(ref ** 2)))
+
+    # whole layer vs the oracle (conditioned on the GPU's selection)
+    o = O.moe_forward(x64, logits, idx_g.astype(np.int64), O.route_weights(logits, idx_g.astype(np.int64), p.gate,
+                      c.a.get("bias") if p.gate == "softmax" else None), c.L.expert, p.E, c.C, p.clamp,
+                      c.clamp_mode, c.L.shared())
+    rel = H.assert_close_layer(p, out_g, o["out"], "out")
+    print(f"{p.name}: out max|err|/rms = {rel:.3g}")
+
+    # moe_forward gives the staged result bit for bit
+    ws = B.workspace(B.workspace_size(c.cfg, p.T))
+    out_f = B.forward(c.cfg, c.x, c.w, ws, c.mask)
+    torch.cuda.synchronize()
+    B.check_device_status(ws)
+    assert torch.equal(out_f, g["out"])
+
+
+def _full_forward_check(B, W, name, n_sample):
+    p = synth.PROBLEMS[name]
+    c = Case(B, W, p)
+    T = p.T
+    ws = B.workspace(B.workspace_size(c.cfg, T))
+    idx_t = torch.empty((T, p.k), dtype=torch.int32, device="cuda")
+    cnt_t = torch.empty(p.E, dtype=torch.int32, device="cuda")
+    out = B.forward(c.cfg, c.x, c.w, ws, c.mask, topk_idx_out=idx_t, expert_counts_out=cnt_t)
+    torch.cuda.synchronize()
+    B.check_device_status(ws)
+    # staged route + dispatch for the per-stage maps
+    idx_g_t, w_g_t = B.route_topk(c.cfg, c.x, c.w, c.mask)
+    dg = B.dispatch(c.cfg, c.x, idx_g_t, w_g_t)
+    torch.cuda.synchronize()
+    idx_g, w_g = H.to_np(idx_g_t), H.to_np(w_g_t)
+    assert np.array_equal(idx_g, H.to_np(idx_t))
+
+    logits, idx_o, w_o, keys = H.oracle_route(p, c.L, c.a)
+    flips, ties = H.check_route(p, idx_g, w_g, logits, idx_o, keys, c.a.get("bias"))
+    d = O.dispatch(idx_g.astype(np.int64), p.E, c.C)
+    R = int(d["offsets"][-1])
+    np.testing.assert_array_equal(H.to_np(cnt_t), d["counts"])
+    np.testing.assert_array_equal(H.to_np(dg["expert_offsets"]), d["offsets"])
+    np.testing.assert_array_equal(H.to_np(dg["slot_row"]), d["slot_row"])
+    np.testing.assert_array_equal(H.to_np(dg["row_token"])[:R], d["row_token"])
+    rows = np.random.default_rng(99).choice(R, size=min(R, 512), replace=False)
+    xs = dg["x_perm"][torch.from_numpy(rows).cuda()].cpu()
+    assert torch.equal(xs, c.x[torch.from_numpy(d["row_token"][rows]).cuda()].cpu())
+    if c.C:
+        print(f"{name}: capacity {c.C}, drops {d['drops']}")
+        assert d["drops"] > 0
+
+    rng = np.random.default_rng(7)
+    toks = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=n_sample, replace=False)]))
+    w_sel = O.route_weights(logits, idx_g.astype(np.int64), p.gate, c.a.get("bias") if p.gate == "softmax" else None)
+    o = O.moe_forward(c.L.x(), logits, idx_g.astype(np.int64), w_sel, c.L.expert, p.E, c.C, p.clamp, "preact",
+                      c.L.shared(), tokens=toks)
+    got = H.to_np(out[torch.from_numpy(toks).cuda()])
+    rel = H.assert_close_layer(p, got, o["out"], "out")
+    print(f"{name}: near-ties {ties}, flipped {flips}, sampled {len(toks)} tokens, max|err|/rms {rel:.3g}")
+
+
+@pytest.mark.parametrize("name,n_sample", [("tiny_f32", 64), ("mixtral_bf16", 48), ("capacity_bf16", 48),
+                                           ("finegrained_bf16", 32), ("sqrt_fp4", 24)])
+def test_full_size_sampled(B, W, name, n_sample):
+    _full_forward_check(B, W, name, n_sample)
+    torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------- edge cases
+
+def _edge_case(B, W, p, bias=None, capacity=None, clamp_mode="preact", x_scale=None):
+    a = synth.generate(p)
+    if bias is not None:
+        a["bias"] = bias.astype(np.float32)
+    if x_scale is not None:
+        xf = O.decode_act(a["x"], p.act) * x_scale
+        a["x"] = xf.astype(np.float32) if p.act == "f32" else synth.f32_to_bf16_bits(xf.astype(np.float32))
+    c = Case(B, W, p, a, clamp_mode)
+    if capacity is not None:
+        c.cfg.expert_capacity = capacity
+        c.C = capacity
+    g = _stages(B, c)
+    idx_g = H.to_np(g["idx"]).astype(np.int64)
+    logits, idx_o, w_o, keys = H.oracle_route(p, c.L, a)
+    H.check_route(p, idx_g, H.to_np(g["w"]), logits, idx_o, keys, a.get("bias"))
+    d = O.dispatch(idx_g, p.E, c.C)
+    np.testing.assert_array_equal(H.to_np(g["slot_row"]), d["slot_row"])
+    np.testing.assert_array_equal(H.to_np(g["expert_offsets"]), d["offsets"])
+    w_sel = O.route_weights(logits, idx_g, p.gate, a.get("bias") if p.gate == "softmax" else None)
+    o = O.moe_forward(c.L.x(), logits, idx_g, w_sel, c.L.expert, p.E, c.C, p.clamp, clamp_mode, c.L.shared())
+    H.assert_close_layer(p, H.to_np(g["out"]), o["out"], "out")
+    return g, d
+
+
+BASE = synth.MoEProblem("edge", T=300, D=512, F=384, E=6, k=2, seed=11)
+
+
+@pytest.mark.parametrize("T", [1, 2, 37, 129, 257])
+def test_ragged_token_counts(B, W, T):
+    _edge_case(B, W, BASE.with_(T=T))
+
+
+def test_expert_with_no_tokens(B, W):
+    bias = np.zeros(6)
+    bias[3] = -100.0
+    g, d = _edge_case(B, W, BASE, bias=bias)
+    assert d["counts"][3] == 0
+
+
+def test_all_tokens_one_expert(B, W):
+    bias = np.zeros(6)
+    bias[4] = 100.0
+    g, d = _edge_case(B, W, BASE.with_(k=1), bias=bias)
+    assert d["counts"][4] == BASE.T
+
+
+def test_capacity_one(B, W):
+    g, d = _edge_case(B, W, BASE, capacity=1)
+    assert d["drops"] == BASE.T * 2 - 6
+
+
+def test_k_equals_E(B, W):
+    _edge_case(B, W, BASE.with_(E=4, k=4))
+
+
+def test_shapes_off_the_tile_grid(B, W):
+    _edge_case(B, W, BASE.with_(T=77, D=200, F=104))
+
+
+def test_fp32_shapes_off_the_tile_grid(B, W):
+    _edge_case(B, W, synth.PROBLEMS["tiny_f32"].with_(T=45, D=72, F=40, E=5, k=3))
+
+
+def test_clamp_fires_both_modes(B, W):
+    p = synth.PROBLEMS["sqrt_fp4"].with_(T=200, D=256, F=256, E=8, k=2, Fs=128)
+    _edge_case(B, W, p, x_scale=20.0, clamp_mode="preact")
+    _edge_case(B, W, p, x_scale=20.0, clamp_mode="output")
+
+
+def test_deterministic_and_canaries(B, W):
+    p = H.small("finegrained_bf16")
+    c = Case(B, W, p)
+    ws = B.workspace(B.workspace_size(c.cfg, p.T))
+    G = 4096  # guard elements on each side of the output
+    outs = []
+    for _ in range(3):
+        buf = torch.full((p.T * p.D + 2 * G,), 7.25, dtype=torch.bfloat16, device="cuda")
+        out = buf[G:G + p.T * p.D].view(p.T, p.D)
+        idx = torch.full((p.T * p.k + 2 * G,), -77, dtype=torch.int32, device="cuda")
+        B.forward(c.cfg, c.x, c.w, ws, c.mask, out=out, topk_idx_out=idx[G:G + p.T * p.k].view(p.T, p.k))
+        torch.cuda.synchronize()
+        assert torch.all(buf[:G] == 7.25) and torch.all(buf[-G:] == 7.25)
+        assert torch.all(idx[:G] == -77) and torch.all(idx[-G:] == -77)
+        outs.append(out.clone())
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+    B.check_device_status(ws)
+
+
+def test_zero_tokens(B, W):
+    p = H.small("mixtral_bf16")
+    c = Case(B, W, p)
+    ws = B.workspace(B.workspace_size(c.cfg, p.T))
+    x0 = c.x[:0]
+    out = B.forward(c.cfg, x0, c.w, ws)
+    assert out.shape == (0, p.D)
