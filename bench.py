@@ -174,9 +174,9 @@ def run_ours(args, p, rank, world, local_rank):
                 row_weight=torch.empty(T * k, dtype=torch.float32, device=dev),
                 x_perm=torch.empty((T * k, D), dtype=act, device=dev))
     h = torch.empty((max(T * k * p.F, T * p.Fs),), dtype=act, device=dev)
-    y = torch.empty((T * k, D), dtype=act, device=dev)
-    shy = torch.empty((T, D), dtype=act, device=dev) if p.Fs else None
-    out = torch.empty((T, D), dtype=act, device=dev)
+    y = torch.empty((T * k, D), dtype=torch.float32, device=dev)
+    shy = torch.empty((T, D), dtype=torch.float32, device=dev) if p.Fs else None
+    out = torch.empty((T, D), dtype=torch.float32, device=dev)
     ws_d = B.workspace(B.dispatch_workspace_size(cfg, T), dev)
     ws_e = B.workspace(B.expert_workspace_size(cfg), dev)
     scfg = B.make_config(E=1, k=1, D=D, F=max(p.Fs, 1), clamp=p.clamp, act=p.act, expert=p.act) if p.Fs else None
@@ -242,10 +242,10 @@ def run_ours(args, p, rank, world, local_rank):
     layer = B.MoELayer(cfg, wt, T, dev)
     x_h = WL.to_torch(arrays["x"], "cpu", pin=True)
     m_h = WL.to_torch(arrays.get("image_mask"), "cpu", pin=True)
-    out_h = torch.empty((T, D), dtype=act).pin_memory()
+    out_h = torch.empty((T, D), dtype=torch.float32).pin_memory()
     x_d = torch.empty_like(x_h, device=dev)
     m_d = torch.empty_like(m_h, device=dev) if m_h is not None else None
-    out_d = torch.empty((T, D), dtype=act, device=dev)
+    out_d = torch.empty((T, D), dtype=torch.float32, device=dev)
     for _ in range(max(1, args.warmup)):
         layer.forward_host(x_h, out_h, m_h, x_d, out_d, m_d)
     torch.cuda.synchronize()
@@ -280,6 +280,7 @@ def run_ours(args, p, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32" if p.act == "f32" else "bf16", "data": "synthetic",
         "config": {"workload": describe(p), "tokens_per_gpu": T, "rows_after_capacity": rows,
+                   "out_dtype": "f32",
                    "parallelism": f"dp{world} (independent token batches, replicated weights)",
                    "l2": "inputs larger than L2: expert weights %.2f GB streamed every step" % (layer_bytes(p) / 1e9)},
         "latency_ms": {"p50": float(np.percentile(per_step, 50)), "p95": float(np.percentile(per_step, 95)),

@@ -80,10 +80,14 @@ typedef struct {
   moe_gate gate;
   float swiglu_clamp;          /* L; 0 = no clamp */
   moe_clamp_mode clamp_mode;
-  moe_dtype act_dtype;         /* x, router weights, shared-expert weights, every
-                                  intermediate and out: MOE_F32 or MOE_BF16 */
+  moe_dtype act_dtype;         /* x, router weights, shared-expert weights, x_perm and
+                                  the SwiGLU hidden h: MOE_F32 or MOE_BF16 */
   moe_dtype expert_dtype;      /* routed expert weights: MOE_F32 (only with F32
                                   activations), MOE_BF16 or MOE_NVFP4 (BF16 activations) */
+  moe_dtype out_dtype;         /* layer output: MOE_F32 or MOE_BF16.  The expert outputs
+                                  y are always fp32, so the only rounding after the down
+                                  projection is this final store (a bf16 store alone is
+                                  up to 2^-8 relative) */
 } MoEConfig;
 
 /* Weights.  Matrices are in nn.Linear layout (out_features x in_features), so
@@ -186,14 +190,15 @@ moe_status moe_expert_gate_up(const MoEConfig *cfg, int rows, const void *x_perm
 
 /* Grouped down GEMM with the routing-weight epilogue (a7):
  *   y[r, :] = row_weight[r] * (h[r] W_down[e]^T)   (row_weight NULL = 1)
+ *   h      [rows, F] act dtype
  *   w_down [E, D, F] in cfg->expert_dtype; s_down NVFP4 scales or NULL
- *   y      [rows, D] act dtype out */
+ *   y      [rows, D] float out */
 moe_status moe_expert_down(const MoEConfig *cfg, int rows, const void *h,
                            const int32_t *expert_offsets, const void *w_down, const void *s_down,
                            const float *row_weight, void *y, void *ws, size_t ws_bytes,
                            moe_stream_t stream);
 
-/* Both expert GEMMs: x_perm -> y_perm through h held in `ws` (a6 + a7). */
+/* Both expert GEMMs: x_perm -> y_perm (float [rows, D]) through h held in `ws` (a6 + a7). */
 moe_status moe_grouped_swiglu(const MoEConfig *cfg, int rows, const void *x_perm,
                               const int32_t *expert_offsets, const MoEWeights *w,
                               const float *row_weight, void *y_perm, void *ws, size_t ws_bytes,
@@ -203,8 +208,9 @@ moe_status moe_grouped_swiglu(const MoEConfig *cfg, int rows, const void *x_perm
 
 /* out[t, :] = sum_{j=0..k-1, slot_row[t,j] >= 0} y_perm[slot_row[t, j], :]
  *             (+ shared_y[t, :] when shared_y != NULL)                  (a9)
- * Sums in fp32 in the fixed order j = 0..k-1, then the shared term; output in
- * the act dtype.  Deterministic.  y_perm rows already carry their weights. */
+ * y_perm [>= max slot_row + 1, D] float (rows already carry their weights),
+ * shared_y [T, D] float or NULL, out [T, D] in cfg->out_dtype.  Sums in fp32
+ * in the fixed order j = 0..k-1, then the shared term.  Deterministic. */
 moe_status moe_combine(const MoEConfig *cfg, int T, const void *y_perm, const int32_t *slot_row,
                        const void *shared_y, void *out, moe_stream_t stream);
 
@@ -214,7 +220,7 @@ moe_status moe_combine(const MoEConfig *cfg, int T, const void *y_perm, const in
 size_t moe_workspace_size(const MoEConfig *cfg, int T);
 
 /* The whole layer: route, dispatch, experts, shared expert, combine.
- *   x [T, D], out [T, D] act dtype; image_mask as in moe_route_topk
+ *   x [T, D] act dtype, out [T, D] cfg->out_dtype; image_mask as in moe_route_topk
  *   topk_idx_out [T, k] int32 or NULL: copy of the routing decision
  *   expert_counts_out [E] int32 or NULL: assignments per expert before capacity
  *   ws: workspace of at least moe_workspace_size(cfg, T) bytes

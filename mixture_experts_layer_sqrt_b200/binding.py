@@ -31,7 +31,8 @@ class MoEConfig(ctypes.Structure):
     _fields_ = [("num_experts", c_int), ("top_k", c_int), ("expert_capacity", c_int),
                 ("hidden_dim", c_int), ("intermediate_dim", c_int),
                 ("shared_intermediate_dim", c_int), ("gate", c_int), ("swiglu_clamp", c_float),
-                ("clamp_mode", c_int), ("act_dtype", c_int), ("expert_dtype", c_int)]
+                ("clamp_mode", c_int), ("act_dtype", c_int), ("expert_dtype", c_int),
+                ("out_dtype", c_int)]
 
 
 class MoEWeights(ctypes.Structure):
@@ -118,9 +119,13 @@ def _stream(stream=None):
 
 
 def make_config(E: int, k: int, D: int, F: int, capacity: int = 0, Fs: int = 0, gate="softmax",
-                clamp: float = 0.0, clamp_mode="preact", act="bf16", expert="bf16") -> MoEConfig:
+                clamp: float = 0.0, clamp_mode="preact", act="bf16", expert="bf16", out="f32") -> MoEConfig:
     return MoEConfig(E, k, capacity, D, F, Fs, GATES[gate], clamp, CLAMP_MODES[clamp_mode],
-                     DTYPES[act], DTYPES[expert])
+                     DTYPES[act], DTYPES[expert], DTYPES[out])
+
+
+def out_torch_dtype(cfg: MoEConfig):
+    return torch.float32 if cfg.out_dtype == MOE_F32 else torch.bfloat16
 
 
 def make_weights(t: Dict[str, Optional[torch.Tensor]]) -> MoEWeights:
@@ -185,7 +190,7 @@ def expert_down(cfg: MoEConfig, h: torch.Tensor, offsets: Optional[torch.Tensor]
                 row_weight=None, y=None, ws=None, rows=None, stream=None) -> torch.Tensor:
     rows = h.shape[0] if rows is None else rows
     if y is None:
-        y = torch.empty((rows, cfg.hidden_dim), dtype=h.dtype, device=h.device)
+        y = torch.empty((rows, cfg.hidden_dim), dtype=torch.float32, device=h.device)
     if ws is None:
         ws = workspace(lib.moe_expert_workspace_size(ctypes.byref(cfg)), h.device)
     _check(lib.moe_expert_down(ctypes.byref(cfg), rows, _p(h), _p(offsets), _p(w_down), _p(s_down),
@@ -198,7 +203,7 @@ def grouped_swiglu(cfg: MoEConfig, x_perm: torch.Tensor, offsets, w: MoEWeights,
                    y=None, ws=None, stream=None) -> torch.Tensor:
     rows = x_perm.shape[0]
     if y is None:
-        y = torch.empty((rows, cfg.hidden_dim), dtype=x_perm.dtype, device=x_perm.device)
+        y = torch.empty((rows, cfg.hidden_dim), dtype=torch.float32, device=x_perm.device)
     if ws is None:
         ws = workspace(lib.moe_grouped_swiglu_workspace_size(ctypes.byref(cfg), rows), x_perm.device)
     _check(lib.moe_grouped_swiglu(ctypes.byref(cfg), rows, _p(x_perm), _p(offsets), ctypes.byref(w),
@@ -210,7 +215,7 @@ def grouped_swiglu(cfg: MoEConfig, x_perm: torch.Tensor, offsets, w: MoEWeights,
 def combine(cfg: MoEConfig, y_perm: torch.Tensor, slot_row: torch.Tensor, T: int, shared_y=None,
             out=None, stream=None) -> torch.Tensor:
     if out is None:
-        out = torch.empty((T, cfg.hidden_dim), dtype=y_perm.dtype, device=y_perm.device)
+        out = torch.empty((T, cfg.hidden_dim), dtype=out_torch_dtype(cfg), device=y_perm.device)
     _check(lib.moe_combine(ctypes.byref(cfg), T, _p(y_perm), _p(slot_row), _p(shared_y), _p(out),
                            _stream(stream)), "moe_combine")
     return out
@@ -236,7 +241,7 @@ def forward(cfg: MoEConfig, x: torch.Tensor, w: MoEWeights, ws: torch.Tensor, im
             out=None, topk_idx_out=None, expert_counts_out=None, stream=None) -> torch.Tensor:
     T = x.shape[0]
     if out is None:
-        out = torch.empty((T, cfg.hidden_dim), dtype=x.dtype, device=x.device)
+        out = torch.empty((T, cfg.hidden_dim), dtype=out_torch_dtype(cfg), device=x.device)
     _check(lib.moe_forward(ctypes.byref(cfg), T, _p(x), ctypes.byref(w), _p(image_mask), _p(out),
                            _p(topk_idx_out), _p(expert_counts_out), _p(ws), ws.numel(), _stream(stream)),
            "moe_forward")

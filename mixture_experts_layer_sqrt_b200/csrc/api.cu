@@ -45,6 +45,7 @@ moe_status validate_cfg(const MoEConfig *c) {
     return MOE_ERR_INVALID_ARG;
   if (!(c->swiglu_clamp >= 0.0f)) return MOE_ERR_INVALID_ARG;
   if (c->clamp_mode != MOE_CLAMP_PREACT && c->clamp_mode != MOE_CLAMP_OUTPUT) return MOE_ERR_INVALID_ARG;
+  if (c->out_dtype != MOE_F32 && c->out_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (c->act_dtype == MOE_F32) {
     if (c->expert_dtype != MOE_F32) return MOE_ERR_UNSUPPORTED;
   } else if (c->act_dtype == MOE_BF16) {
@@ -146,8 +147,8 @@ ForwardWs carve_forward(Carve &cv, const MoEConfig &c, int T) {
   size_t hrows = Tk * c.intermediate_dim;
   if ((size_t)T * c.shared_intermediate_dim > hrows) hrows = (size_t)T * c.shared_intermediate_dim;
   w.h = cv.take<char>(hrows * as);
-  w.y_perm = cv.take<char>(Tk * D * as);
-  w.sh_y = c.shared_intermediate_dim ? cv.take<char>((size_t)T * D * as) : nullptr;
+  w.y_perm = cv.take<float>(Tk * D);
+  w.sh_y = c.shared_intermediate_dim ? cv.take<float>((size_t)T * D) : nullptr;
   w.ex.status = w.status;
   w.ex.wexp = nullptr;
   if (c.expert_dtype == MOE_NVFP4)

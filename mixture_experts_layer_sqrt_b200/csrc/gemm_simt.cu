@@ -18,7 +18,7 @@ namespace {
 
 constexpr int BM = 64, BN = 64, BK = 16;
 
-template <typename TIn, bool GATED>
+template <typename TIn, typename TOut, bool GATED>
 __global__ void __launch_bounds__(256) grouped_gemm_simt(int rows, int K, int N,
                                                          const int32_t *__restrict__ offsets, int E,
                                                          const TIn *__restrict__ A,
@@ -26,7 +26,7 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt(int rows, int K, int N,
                                                          const TIn *__restrict__ B1, float clamp,
                                                          int clamp_mode,
                                                          const float *__restrict__ row_weight,
-                                                         TIn *__restrict__ out) {
+                                                         TOut *__restrict__ out) {
   __shared__ float As[BK][BM + 4];
   __shared__ float Bs0[BK][BN + 4];
   __shared__ float Bs1[GATED ? BK : 1][BN + 4];
@@ -107,20 +107,20 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt(int rows, int K, int N,
       float v;
       if (GATED) v = swiglu_h(acc0[i][j], acc1[i][j], clamp, clamp_mode);
       else v = acc0[i][j] * rw;
-      out[(long)row * N + col] = from_f32<TIn>(v);
+      out[(long)row * N + col] = from_f32<TOut>(v);
     }
   }
 }
 
-template <typename TIn, bool GATED>
+template <typename TIn, typename TOut, bool GATED>
 void launch_one(int rows, int K, int N, const int32_t *offsets, int E, const void *A,
                 const void *B0, const void *B1, float clamp, int clamp_mode,
                 const float *row_weight, void *out, cudaStream_t s) {
   long mt = (rows + BM - 1) / BM + (offsets ? E : 0);
   dim3 grid((unsigned)mt, (N + BN - 1) / BN);
-  grouped_gemm_simt<TIn, GATED><<<grid, 256, 0, s>>>(rows, K, N, offsets, E, (const TIn *)A,
-                                                     (const TIn *)B0, (const TIn *)B1, clamp,
-                                                     clamp_mode, row_weight, (TIn *)out);
+  grouped_gemm_simt<TIn, TOut, GATED><<<grid, 256, 0, s>>>(rows, K, N, offsets, E, (const TIn *)A,
+                                                           (const TIn *)B0, (const TIn *)B1, clamp,
+                                                           clamp_mode, row_weight, (TOut *)out);
 }
 
 }  // namespace
@@ -131,10 +131,10 @@ moe_status launch_gate_up_simt(const MoEConfig &c, int rows, const void *a,
   if (rows == 0) return MOE_OK;
   const int E = offsets ? c.num_experts : 1;
   if (c.act_dtype == MOE_F32)
-    launch_one<float, true>(rows, c.hidden_dim, F, offsets, E, a, w_gate, w_up, c.swiglu_clamp,
+    launch_one<float, float, true>(rows, c.hidden_dim, F, offsets, E, a, w_gate, w_up, c.swiglu_clamp,
                             c.clamp_mode, nullptr, h, s);
   else
-    launch_one<__nv_bfloat16, true>(rows, c.hidden_dim, F, offsets, E, a, w_gate, w_up,
+    launch_one<__nv_bfloat16, __nv_bfloat16, true>(rows, c.hidden_dim, F, offsets, E, a, w_gate, w_up,
                                     c.swiglu_clamp, c.clamp_mode, nullptr, h, s);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
@@ -146,10 +146,10 @@ moe_status launch_down_simt(const MoEConfig &c, int rows, const void *h, const i
   if (rows == 0) return MOE_OK;
   const int E = offsets ? c.num_experts : 1;
   if (c.act_dtype == MOE_F32)
-    launch_one<float, false>(rows, F, c.hidden_dim, offsets, E, h, w_down, nullptr, 0.0f, 0,
+    launch_one<float, float, false>(rows, F, c.hidden_dim, offsets, E, h, w_down, nullptr, 0.0f, 0,
                              row_weight, y, s);
   else
-    launch_one<__nv_bfloat16, false>(rows, F, c.hidden_dim, offsets, E, h, w_down, nullptr, 0.0f,
+    launch_one<__nv_bfloat16, float, false>(rows, F, c.hidden_dim, offsets, E, h, w_down, nullptr, 0.0f,
                                      0, row_weight, y, s);
   MOE_LAUNCH_CHECK();
   return MOE_OK;

@@ -20,9 +20,9 @@ def capacity_of(p: MoEProblem) -> int:
     return B.expert_capacity(p.T, p.k, p.E, f.numerator, f.denominator)
 
 
-def config_of(p: MoEProblem, clamp_mode: str = "preact") -> B.MoEConfig:
+def config_of(p: MoEProblem, clamp_mode: str = "preact", out: str = "f32") -> B.MoEConfig:
     return B.make_config(E=p.E, k=p.k, D=p.D, F=p.F, capacity=capacity_of(p), Fs=p.Fs, gate=p.gate,
-                         clamp=p.clamp, clamp_mode=clamp_mode, act=p.act, expert=p.wdtype)
+                         clamp=p.clamp, clamp_mode=clamp_mode, act=p.act, expert=p.wdtype, out=out)
 
 
 def to_torch(a: Optional[np.ndarray], device="cuda", pin=False) -> Optional[torch.Tensor]:

@@ -73,6 +73,28 @@ def check_route(p, idx_g: np.ndarray, w_g: np.ndarray, logits, idx_o, keys, bias
     return int(diff.sum()), int(nt.sum())
 
 
+def assert_close_h(p, got: np.ndarray, ref: np.ndarray, what: str = "h"):
+    """The SwiGLU hidden h is stored in the act dtype: bf16 adds one rounding of
+    at most 2^-8 relative (RNE), on top of fp32 accumulation error."""
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    err = np.abs(got - ref)
+    if p.act == "f32":
+        lim = F32_RTOL * np.maximum(np.abs(ref), rms)
+    else:
+        lim = 2.0 ** -8 * np.abs(ref) + 1e-3 * rms
+    bad = err > lim
+    assert not bad.any(), f"{what}: {bad.sum()} elements out of bound, max ratio {(err / lim).max():.3g}"
+
+
+def assert_close_f32(got: np.ndarray, ref: np.ndarray, what: str, rtol: float = F32_RTOL):
+    """fp32 results computed from the GPU's own (exactly known) inputs."""
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    err = np.abs(got - ref)
+    lim = rtol * np.maximum(np.abs(ref), rms)
+    bad = err > lim
+    assert not bad.any(), f"{what}: {bad.sum()} elements above {rtol} rel, max ratio {(err / lim).max():.3g}"
+
+
 def assert_close_layer(p, got: np.ndarray, ref: np.ndarray, what: str):
     rms = float(np.sqrt(np.mean(ref ** 2)))
     err = np.abs(got - ref)
