@@ -113,6 +113,14 @@ def _p(t: Optional[torch.Tensor]):
     return None if t is None else t.data_ptr()
 
 
+def _expect(t: Optional[torch.Tensor], shape, dtype, what: str):
+    """Buffers handed to the library must match what it will write."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{what}: expected contiguous {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return s.cuda_stream
@@ -191,6 +199,9 @@ def expert_down(cfg: MoEConfig, h: torch.Tensor, offsets: Optional[torch.Tensor]
     rows = h.shape[0] if rows is None else rows
     if y is None:
         y = torch.empty((rows, cfg.hidden_dim), dtype=torch.float32, device=h.device)
+    _expect(y, (y.shape[0], cfg.hidden_dim), torch.float32, "y")
+    if y.shape[0] < rows:
+        raise ValueError("y has fewer rows than `rows`")
     if ws is None:
         ws = workspace(lib.moe_expert_workspace_size(ctypes.byref(cfg)), h.device)
     _check(lib.moe_expert_down(ctypes.byref(cfg), rows, _p(h), _p(offsets), _p(w_down), _p(s_down),
@@ -216,6 +227,8 @@ def combine(cfg: MoEConfig, y_perm: torch.Tensor, slot_row: torch.Tensor, T: int
             out=None, stream=None) -> torch.Tensor:
     if out is None:
         out = torch.empty((T, cfg.hidden_dim), dtype=out_torch_dtype(cfg), device=y_perm.device)
+    _expect(out, (T, cfg.hidden_dim), out_torch_dtype(cfg), "out")
+    _expect(y_perm, (y_perm.shape[0], cfg.hidden_dim), torch.float32, "y_perm")
     _check(lib.moe_combine(ctypes.byref(cfg), T, _p(y_perm), _p(slot_row), _p(shared_y), _p(out),
                            _stream(stream)), "moe_combine")
     return out
@@ -242,6 +255,9 @@ def forward(cfg: MoEConfig, x: torch.Tensor, w: MoEWeights, ws: torch.Tensor, im
     T = x.shape[0]
     if out is None:
         out = torch.empty((T, cfg.hidden_dim), dtype=out_torch_dtype(cfg), device=x.device)
+    _expect(out, (T, cfg.hidden_dim), out_torch_dtype(cfg), "out")
+    _expect(topk_idx_out, (T, cfg.top_k), torch.int32, "topk_idx_out")
+    _expect(expert_counts_out, (cfg.num_experts,), torch.int32, "expert_counts_out")
     _check(lib.moe_forward(ctypes.byref(cfg), T, _p(x), ctypes.byref(w), _p(image_mask), _p(out),
                            _p(topk_idx_out), _p(expert_counts_out), _p(ws), ws.numel(), _stream(stream)),
            "moe_forward")

@@ -95,6 +95,8 @@ moe_status run_gate_up(const MoEConfig &c, int rows, const void *a, const int32_
     wu = ws.wexp + n;
     cc.expert_dtype = MOE_BF16;
   }
+  if (tc_shapes_ok(cc, c.intermediate_dim))
+    return launch_gate_up_tc(cc, rows, a, offsets, wg, wu, c.intermediate_dim, h, ws.status, s);
   return launch_gate_up_simt(cc, rows, a, offsets, wg, wu, c.intermediate_dim, h, s);
 }
 
@@ -109,6 +111,8 @@ moe_status run_down(const MoEConfig &c, int rows, const void *h, const int32_t *
     wd = ws.wexp;
     cc.expert_dtype = MOE_BF16;
   }
+  if (tc_shapes_ok(cc, c.intermediate_dim))
+    return launch_down_tc(cc, rows, h, offsets, wd, c.intermediate_dim, row_weight, (float *)y, ws.status, s);
   return launch_down_simt(cc, rows, h, offsets, wd, c.intermediate_dim, row_weight, y, s);
 }
 

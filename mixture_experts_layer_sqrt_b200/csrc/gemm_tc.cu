@@ -1,0 +1,457 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// "FFN、SwiGLU 与 MoE" sec. 2: y = W_down[SiLU(W_gate x) * (W_up x)]; the
+// ops-transformer MoE walkthrough (优化三) packs every expert's rows into one
+// irregular matmul launch.  Here one persistent kernel covers all experts:
+//
+//   gate/up (GATED):  for the rows of expert e, D[128 x 256] accumulates
+//                     x_perm[rows] . [W_gate[e] rows n0..n0+127 ; W_up[e] rows n0..n0+127]^T,
+//                     so TMEM columns 0..127 hold g and 128..255 hold u; the
+//                     epilogue forms h = SiLU(clip g) * clip u and stores bf16.
+//   down:             D[128 x 256] = h[rows] . W_down[e][n0..n0+255]^T; the
+//                     epilogue scales row r by row_weight[r] and stores fp32.
+//
+// Structure (one CTA per SM, 192 threads):
+//   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (bf16, 128-byte
+//               swizzle) per k-block into a 4-stage ring guarded by mbarriers.
+//   warp 1      TMEM owner and MMA issuer: one thread issues 4 tcgen05.mma
+//               (M=128, N=256, K=16) per k-block and commits each stage back
+//               to the producer; two 256-column fp32 accumulators let the
+//               epilogue of tile i overlap the MMAs of tile i+1.
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
+//               output row per thread), fused SwiGLU or routing weight, store.
+//
+// Tiles never straddle two experts: expert e owns ceil(rows_e / 128) m-blocks;
+// the tile list (expert-major, then n-block, then m-block, so the CTAs in
+// flight share weight tiles through L2) is derived on the device from
+// expert_offsets, so the host never reads a count.  Rows past the expert's
+// segment are computed from whatever lies there and never stored.
+//
+// Every wait is bounded: after kWaitLimitNs the waiting thread records
+// MOE_ERR_DEVICE_TIMEOUT in the status word, raises a CTA-wide abort flag and
+// every role winds down (copies drained, TMEM freed) instead of hanging.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;          // rows per tile (TMEM lanes)
+constexpr int BN = 256;          // MMA N (accumulator columns)
+constexpr int BK = 64;           // one 128-byte swizzle row of bf16
+constexpr int STAGES = 4;
+constexpr int UMMA_K = 16;
+constexpr int A_BYTES = BM * BK * 2;         // 16 KB
+constexpr int B_BYTES = BN * BK * 2;         // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t TMEM_COLS = 2 * BN;       // two accumulators
+constexpr int MAX_E = 1024;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s
+constexpr int kThreads = 192;
+
+struct Smem {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int tile_start[MAX_E + 1];
+};
+
+struct Params {
+  int rows;                  // rows of A and of the output
+  int K;                     // reduction length
+  int N;                     // output columns (F for gate/up, D for down)
+  int E;                     // groups
+  int n_tiles;               // output-column tiles per m-block
+  const int32_t *offsets;    // [E+1] row offsets, or null: one group of `rows` rows
+  void *out;                 // h (bf16) or y (fp32), [rows, N]
+  const float *row_weight;   // down only, nullable
+  float clamp;
+  int clamp_mode;
+  int *status;
+};
+
+// Bounded wait; false if the CTA is aborting (this thread may have started it).
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Smem &sm, int *status) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (true) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*(volatile int *)&sm.abort) return false;
+    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+      *(volatile int *)&sm.abort = 1;
+      atomicExch(status, kDevTimeout);
+      return false;
+    }
+  }
+}
+
+// Bounded wait used while winding down: ignores the abort flag (copies and
+// MMAs already issued must land before shared memory or TMEM is released).
+__device__ __forceinline__ void drain_bar(uint64_t *bar, uint32_t parity, int *status) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    if (ptx::globaltimer_ns() - t0 > kDrainLimitNs) {
+      atomicExch(status, kDevTimeout);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ int seg_begin(const Params &p, int e) { return p.offsets ? p.offsets[e] : 0; }
+__device__ __forceinline__ int seg_end(const Params &p, int e) {
+  int v = p.offsets ? p.offsets[e + 1] : p.rows;
+  return v < p.rows ? v : p.rows;
+}
+
+struct Tile {
+  int e, m0, end, n_blk;
+};
+
+// Largest e with tile_start[e] <= t (empty experts share the next start).
+__device__ __forceinline__ Tile decode_tile(const Params &p, const Smem &sm, int t) {
+  int lo = 0, hi = p.E - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (sm.tile_start[mid] <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  const int e = lo;
+  const int local = t - sm.tile_start[e];
+  const int m_tiles = (sm.tile_start[e + 1] - sm.tile_start[e]) / p.n_tiles;
+  Tile r;
+  r.e = e;
+  r.n_blk = local / m_tiles;
+  r.m0 = seg_begin(p, e) + (local - r.n_blk * m_tiles) * BM;
+  r.end = seg_end(p, e);
+  return r;
+}
+
+template <bool GATED>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                    const __grid_constant__ CUtensorMap tmB1, const Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // stage buffers first, 1024-byte aligned (the swizzle atoms need it)
+  uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t *stage_a = base;
+  uint8_t *stage_b = base + STAGES * A_BYTES;
+  Smem &sm = *reinterpret_cast<Smem *>(base + STAGES * STAGE_BYTES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- setup: barriers, TMEM, tile schedule
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(&sm.full[s], 1);
+      ptx::mbar_init(&sm.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(&sm.tmem_full[a], 1);
+      ptx::mbar_init(&sm.tmem_empty[a], 4);
+    }
+    ptx::mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    ptx::fence_mbar_init();
+    ptx::fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB0);
+    if (GATED) ptx::prefetch_tmap(&tmB1);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&sm.tmem_base, TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  if (warp == 2) {
+    // tile_start[e] = sum over e' < e of ceil(rows_e' / BM) * n_tiles
+    int carry = 0;
+    for (int e0 = 0; e0 < p.E; e0 += 32) {
+      const int e = e0 + lane;
+      int v = 0;
+      if (e < p.E) {
+        int n = seg_end(p, e) - seg_begin(p, e);
+        v = n > 0 ? (n + BM - 1) / BM * p.n_tiles : 0;
+      }
+      int incl = v;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (e < p.E) sm.tile_start[e] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) sm.tile_start[p.E] = carry;
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = sm.tmem_base;
+  const int total_tiles = sm.tile_start[p.E];
+  const int k_blocks = (p.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    // ================================================= TMA producer
+    uint32_t last_parity[STAGES];
+    bool used[STAGES];
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s) {
+      used[s] = false;
+      last_parity[s] = 0;
+    }
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const Tile tl = decode_tile(p, sm, t);
+        for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!wait_bar(&sm.empty[s], ph ^ 1u, sm, p.status)) { ok = false; break; }
+          ptx::mbar_arrive_expect_tx(&sm.full[s], STAGE_BYTES);
+          const int k0 = kb * BK;
+          ptx::tma_load_2d(stage_a + s * A_BYTES, &tmA, &sm.full[s], k0, tl.m0);
+          uint8_t *b = stage_b + s * B_BYTES;
+          if (GATED) {
+            const int n0 = tl.n_blk * (BN / 2);
+            ptx::tma_load_3d(b, &tmB0, &sm.full[s], k0, n0, tl.e);
+            ptx::tma_load_3d(b + B_BYTES / 2, &tmB1, &sm.full[s], k0, n0, tl.e);
+          } else {
+            const int n0 = tl.n_blk * BN;
+            ptx::tma_load_3d(b, &tmB0, &sm.full[s], k0, n0, tl.e);
+            ptx::tma_load_3d(b + B_BYTES / 2, &tmB0, &sm.full[s], k0, n0 + BN / 2, tl.e);
+          }
+          used[s] = true;
+          last_parity[s] = ph;
+        }
+      }
+      // drain: every issued copy has landed before shared memory is released
+      for (int s = 0; s < STAGES; ++s)
+        if (used[s]) drain_bar(&sm.full[s], last_parity[s], p.status);
+    }
+  } else if (warp == 1) {
+    // ================================================= MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, BN);
+      uint32_t it = 0;
+      int i = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++i) {
+        const int acc = i & 1;
+        const uint32_t aph = (i >> 1) & 1u;
+        if (!wait_bar(&sm.tmem_empty[acc], aph ^ 1u, sm, p.status)) break;
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!wait_bar(&sm.full[s], ph, sm, p.status)) { ok = false; break; }
+          ptx::tc_fence_after();
+          const uint32_t a_addr = ptx::smem_addr(stage_a + s * A_BYTES);
+          const uint32_t b_addr = ptx::smem_addr(stage_b + s * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            const uint64_t ad = ptx::desc_kmajor_sw128(a_addr + k * UMMA_K * 2);
+            const uint64_t bd = ptx::desc_kmajor_sw128(b_addr + k * UMMA_K * 2);
+            ptx::mma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          }
+          ptx::mma_commit(&sm.empty[s]);
+        }
+        if (!ok) break;
+        ptx::mma_commit(&sm.tmem_full[acc]);
+      }
+      // drain: all issued MMAs complete before TMEM is released
+      ptx::mma_commit(&sm.drain);
+      drain_bar(&sm.drain, 0, p.status);
+    }
+  } else {
+    // ================================================= epilogue (warps 2..5)
+    const int q = warp & 3;                 // TMEM lane quadrant this warp may access
+    const int row_in_tile = q * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    int i = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++i) {
+      const Tile tl = decode_tile(p, sm, t);
+      const int acc = i & 1;
+      const uint32_t aph = (i >> 1) & 1u;
+      if (!wait_bar(&sm.tmem_full[acc], aph, sm, p.status)) break;
+      ptx::tc_fence_after();
+      const uint32_t tbase = tmem_base + lane_addr + acc * BN;
+      const int row = tl.m0 + row_in_tile;
+      const bool live = row < tl.end;
+      if (GATED) {
+        const int ncol0 = tl.n_blk * (BN / 2);
+        __nv_bfloat16 *hrow = (__nv_bfloat16 *)p.out + (long)row * p.N + ncol0;
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t g[32], u[32];
+          ptx::tmem_ld32(tbase + c, g);
+          ptx::tmem_ld32(tbase + BN / 2 + c, u);
+          ptx::tmem_ld_wait();
+          if (live) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              float h0 = swiglu_h(__uint_as_float(g[2 * j]), __uint_as_float(u[2 * j]), p.clamp, p.clamp_mode);
+              float h1 = swiglu_h(__uint_as_float(g[2 * j + 1]), __uint_as_float(u[2 * j + 1]), p.clamp,
+                                  p.clamp_mode);
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(h0, h1);
+              pk[j] = *reinterpret_cast<uint32_t *>(&b2);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(hrow + c);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          }
+        }
+      } else {
+        const int ncol0 = tl.n_blk * BN;
+        const float rw = (live && p.row_weight) ? p.row_weight[row] : 1.0f;
+        float *yrow = (float *)p.out + (long)row * p.N + ncol0;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t v[32];
+          ptx::tmem_ld32(tbase + c, v);
+          ptx::tmem_ld_wait();
+          if (live) {
+            float4 *dst = reinterpret_cast<float4 *>(yrow + c);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              dst[j] = make_float4(__uint_as_float(v[4 * j]) * rw, __uint_as_float(v[4 * j + 1]) * rw,
+                                   __uint_as_float(v[4 * j + 2]) * rw, __uint_as_float(v[4 * j + 3]) * rw);
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&sm.tmem_empty[acc]);
+    }
+  }
+
+  // ---- teardown
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// bf16 tensor [d2][d1][d0] (d0 contiguous) with a {64, 128, 1} box, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  cuuint32_t box[3] = {BK, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d2 > 1 ? 3 : 2, const_cast<void *>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool GATED>
+moe_status launch_tc(const Params &p, const void *a, const void *b0, const void *b1, int Nw, cudaStream_t s) {
+  // A: [rows, K]; B: [E, Nw, K] (rank 3 even for one group)
+  CUtensorMap ta, tb0, tb1;
+  if (!make_map(&ta, a, (uint64_t)p.K, (uint64_t)p.rows, 1)) return MOE_ERR_CUDA;
+  // weights always rank 3 so the kernel's 3-D loads match
+  auto fn = encode_fn();
+  auto map3 = [&](CUtensorMap *m, const void *ptr) {
+    cuuint64_t dims[3] = {(cuuint64_t)p.K, (cuuint64_t)Nw, (cuuint64_t)p.E};
+    cuuint64_t strides[2] = {(cuuint64_t)p.K * 2, (cuuint64_t)p.K * Nw * 2};
+    cuuint32_t box[3] = {BK, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  };
+  if (!map3(&tb0, b0)) return MOE_ERR_CUDA;
+  if (GATED) {
+    if (!map3(&tb1, b1)) return MOE_ERR_CUDA;
+  } else {
+    tb1 = tb0;
+  }
+  int dev = 0, sms = 148;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const long ub = ((long)(p.rows + BM - 1) / BM + (p.offsets ? p.E : 0)) * p.n_tiles;
+  const int grid = (int)(ub < sms ? ub : sms);
+  if (grid <= 0) return MOE_OK;
+  const size_t smem = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Smem);
+  auto kern = tc_grouped_gemm<GATED>;
+  MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  kern<<<grid, kThreads, smem, s>>>(ta, tb0, tb1, p);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+}  // namespace
+
+bool tc_shapes_ok(const MoEConfig &c, int F) {
+  return c.act_dtype == MOE_BF16 && c.hidden_dim % BN == 0 && F % 128 == 0 && c.hidden_dim % BK == 0 &&
+         encode_fn() != nullptr;
+}
+
+moe_status launch_gate_up_tc(const MoEConfig &c, int rows, const void *a, const int32_t *offsets,
+                             const void *w_gate, const void *w_up, int F, void *h, int *status,
+                             cudaStream_t s) {
+  if (rows == 0) return MOE_OK;
+  Params p;
+  p.rows = rows;
+  p.K = c.hidden_dim;
+  p.N = F;
+  p.E = offsets ? c.num_experts : 1;
+  p.n_tiles = F / (BN / 2);
+  p.offsets = offsets;
+  p.out = h;
+  p.row_weight = nullptr;
+  p.clamp = c.swiglu_clamp;
+  p.clamp_mode = c.clamp_mode;
+  p.status = status;
+  return launch_tc<true>(p, a, w_gate, w_up, F, s);
+}
+
+moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
+                          const void *w_down, int F, const float *row_weight, float *y, int *status,
+                          cudaStream_t s) {
+  if (rows == 0) return MOE_OK;
+  Params p;
+  p.rows = rows;
+  p.K = F;
+  p.N = c.hidden_dim;
+  p.E = offsets ? c.num_experts : 1;
+  p.n_tiles = c.hidden_dim / BN;
+  p.offsets = offsets;
+  p.out = y;
+  p.row_weight = row_weight;
+  p.clamp = 0.0f;
+  p.clamp_mode = 0;
+  p.status = status;
+  return launch_tc<false>(p, h, w_down, nullptr, c.hidden_dim, s);
+}
+
+}  // namespace moe

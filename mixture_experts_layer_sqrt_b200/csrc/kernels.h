@@ -35,6 +35,17 @@ moe_status launch_down_simt(const MoEConfig &c, int rows, const void *h, const i
                             const void *w_down, int F, const float *row_weight, void *y,
                             cudaStream_t s);
 
+// gemm_tc.cu -------------------------------------------------------------
+// Grouped GEMMs on tcgen05 tensor cores (bf16 in, fp32 accumulate).  Usable
+// when tc_shapes_ok(): bf16 activations, D % 256 == 0, F % 128 == 0.
+bool tc_shapes_ok(const MoEConfig &c, int F);
+moe_status launch_gate_up_tc(const MoEConfig &c, int rows, const void *a, const int32_t *offsets,
+                             const void *w_gate, const void *w_up, int F, void *h, int *status,
+                             cudaStream_t s);
+moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
+                          const void *w_down, int F, const float *row_weight, float *y, int *status,
+                          cudaStream_t s);
+
 // dequant.cu -------------------------------------------------------------
 // n_elems values (a multiple of 16): packed [n/2] bytes + scales [n/16] -> bf16 [n].
 moe_status launch_dequant_nvfp4(const void *packed, const void *scales, long n_elems, void *out,

@@ -289,7 +289,7 @@ def test_deterministic_and_canaries(B, W):
     G = 4096  # guard elements on each side of the output
     outs = []
     for _ in range(3):
-        buf = torch.full((p.T * p.D + 2 * G,), 7.25, dtype=torch.bfloat16, device="cuda")
+        buf = torch.full((p.T * p.D + 2 * G,), 7.25, dtype=torch.float32, device="cuda")
         out = buf[G:G + p.T * p.D].view(p.T, p.D)
         idx = torch.full((p.T * p.k + 2 * G,), -77, dtype=torch.int32, device="cuda")
         B.forward(c.cfg, c.x, c.w, ws, c.mask, out=out, topk_idx_out=idx[G:G + p.T * p.k].view(p.T, p.k))
@@ -299,6 +299,16 @@ def test_deterministic_and_canaries(B, W):
         outs.append(out.clone())
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
     B.check_device_status(ws)
+
+
+def test_binding_rejects_mismatched_out(B, W):
+    p = H.small("mixtral_bf16")
+    c = Case(B, W, p)
+    ws = B.workspace(B.workspace_size(c.cfg, p.T))
+    with pytest.raises(ValueError):
+        B.forward(c.cfg, c.x, c.w, ws, out=torch.empty((p.T, p.D), dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(ValueError):
+        B.forward(c.cfg, c.x, c.w, ws, out=torch.empty((p.T - 1, p.D), dtype=torch.float32, device="cuda"))
 
 
 def test_zero_tokens(B, W):
