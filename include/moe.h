@@ -168,6 +168,28 @@ moe_status moe_dispatch(const MoEConfig *cfg, int T, const int32_t *topk_idx, co
                         int32_t *slot_row, int32_t *row_token, float *row_weight, void *x_perm,
                         void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Dispatch for callers that cannot allocate device memory on their call path
+ * (a plugin inside an inference engine that offers no workspace, a serving
+ * loop that may not call cudaMalloc, a program whose memory is all owned by
+ * another allocator).  No counterpart on the pages: it is moe_dispatch with
+ * the per-chunk histogram scratch taken from a fixed array inside the library
+ * (MOE_DISPATCH_NOALLOC_MAX_SCRATCH_INTS int32, 1 MiB, held on every GPU that
+ * loads the library until exit) instead of `ws`.  Same arguments, layouts and
+ * results as moe_dispatch otherwise.
+ *  - Returns MOE_ERR_UNSUPPORTED when ceil(T / 256) * E exceeds the limit,
+ *    MOE_ERR_INVALID_ARG for a bad config or pointer, MOE_ERR_CUDA if the
+ *    array's device address cannot be obtained.
+ *  - The first call on a device looks up the array's address on that device
+ *    (cudaGetSymbolAddress); make it before any stream capture.
+ *  - All calls share the one array: calls that overlap on the GPU race and
+ *    must be serialised by the caller.  No entry needs clearing between calls.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+#define MOE_DISPATCH_NOALLOC_MAX_SCRATCH_INTS 262144
+moe_status moe_dispatch_noalloc(const MoEConfig *cfg, int T, const int32_t *topk_idx,
+                                const float *topk_w, const void *x, int32_t *expert_counts,
+                                int32_t *expert_offsets, int32_t *slot_row, int32_t *row_token,
+                                float *row_weight, void *x_perm, moe_stream_t stream);
+
 /* ---------------------------------------------------------- stage 3: experts */
 
 /* Bytes of workspace moe_grouped_swiglu needs for up to `rows` rows. */

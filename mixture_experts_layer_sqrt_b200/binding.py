@@ -62,6 +62,7 @@ def _load() -> ctypes.CDLL:
         "moe_route_topk": (I, [cfgp, I, P, wp, P, P, P, P]),
         "moe_dispatch_workspace_size": (S, [cfgp, I]),
         "moe_dispatch": (I, [cfgp, I, P, P, P, P, P, P, P, P, P, P, S, P]),
+        "moe_dispatch_noalloc": (I, [cfgp, I, P, P, P, P, P, P, P, P, P, P]),
         "moe_grouped_swiglu_workspace_size": (S, [cfgp, I]),
         "moe_expert_workspace_size": (S, [cfgp]),
         "moe_expert_gate_up": (I, [cfgp, I, P, P, P, P, P, P, P, P, S, P]),
@@ -83,7 +84,7 @@ lib = _load()
 # Every function the header declares (checked by the tests).
 EXPORTS = ("moe_status_string", "moe_version", "moe_expert_capacity", "moe_launch_count",
            "moe_check_device_status", "moe_route_topk", "moe_dispatch_workspace_size",
-           "moe_dispatch", "moe_grouped_swiglu_workspace_size", "moe_expert_workspace_size",
+           "moe_dispatch", "moe_dispatch_noalloc", "moe_grouped_swiglu_workspace_size", "moe_expert_workspace_size",
            "moe_expert_gate_up", "moe_expert_down", "moe_grouped_swiglu", "moe_combine",
            "moe_workspace_size", "moe_forward")
 
@@ -178,6 +179,25 @@ def dispatch(cfg: MoEConfig, x: torch.Tensor, topk_idx: torch.Tensor, topk_w: to
                             _p(o["expert_counts"]), _p(o["expert_offsets"]), _p(o["slot_row"]),
                             _p(o["row_token"]), _p(o["row_weight"]), _p(o["x_perm"]), _p(ws),
                             ws.numel(), _stream(stream)), "moe_dispatch")
+    return o
+
+
+def dispatch_noalloc(cfg: MoEConfig, x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,
+                     out: Optional[Dict[str, torch.Tensor]] = None, stream=None) -> Dict[str, torch.Tensor]:
+    """moe_dispatch_noalloc: dispatch with the library's own fixed scratch, no workspace."""
+    T, D, E, k = x.shape[0], cfg.hidden_dim, cfg.num_experts, cfg.top_k
+    dev = x.device
+    o = out or dict(
+        expert_counts=torch.empty(E, dtype=torch.int32, device=dev),
+        expert_offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+        slot_row=torch.empty((T, k), dtype=torch.int32, device=dev),
+        row_token=torch.empty(T * k, dtype=torch.int32, device=dev),
+        row_weight=torch.empty(T * k, dtype=torch.float32, device=dev),
+        x_perm=torch.empty((T * k, D), dtype=x.dtype, device=dev))
+    _check(lib.moe_dispatch_noalloc(ctypes.byref(cfg), T, _p(topk_idx), _p(topk_w), _p(x),
+                                    _p(o["expert_counts"]), _p(o["expert_offsets"]), _p(o["slot_row"]),
+                                    _p(o["row_token"]), _p(o["row_weight"]), _p(o["x_perm"]),
+                                    _stream(stream)), "moe_dispatch_noalloc")
     return o
 
 
