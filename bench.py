@@ -184,21 +184,29 @@ def run_ours(args, p, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     hF = h[:T * k * p.F].view(T * k, p.F)
 
-    def step(ev=None):
-        B.route_topk(cfg, x, w, mask, idx, tw)
-        B.dispatch(cfg, x, idx, tw, disp, ws_d)
+    def mark(ev, i):
         if ev is not None:
-            ev[0].record(stream)
+            ev[i].record(stream)
+
+    # events: 0 | route | 1 | dispatch | 2 | gate/up | 3 | down | 4 | shared | 5 | combine | 6
+    def step(ev=None):
+        mark(ev, 0)
+        B.route_topk(cfg, x, w, mask, idx, tw)
+        mark(ev, 1)
+        B.dispatch(cfg, x, idx, tw, disp, ws_d)
+        mark(ev, 2)
         B.expert_gate_up(cfg, disp["x_perm"], disp["expert_offsets"], wt["w_gate"], wt["w_up"],
                          wt.get("s_gate"), wt.get("s_up"), hF, ws_e)
-        if ev is not None:
-            ev[1].record(stream)
+        mark(ev, 3)
         B.expert_down(cfg, hF, disp["expert_offsets"], wt["w_down"], wt.get("s_down"), disp["row_weight"], y, ws_e)
+        mark(ev, 4)
         if p.Fs:
             hs = h[:T * p.Fs].view(T, p.Fs)
             B.expert_gate_up(scfg, x, None, wt["sh_gate"], wt["sh_up"], None, None, hs, ws_s)
             B.expert_down(scfg, hs, None, wt["sh_down"], None, None, shy, ws_s)
+        mark(ev, 5)
         B.combine(cfg, y, disp["slot_row"], T, shy, out)
+        mark(ev, 6)
 
     for _ in range(args.warmup):
         step()
@@ -216,7 +224,7 @@ def run_ours(args, p, rank, world, local_rank):
     torch.cuda.synchronize()
     n0 = B.launch_count()
     step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    g_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    g_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
     step_ev[0].record(stream)
     for i in range(args.steps):
         step(g_ev[i])
@@ -228,7 +236,9 @@ def run_ours(args, p, rank, world, local_rank):
     clocks = sampler.stop() if sampler else None
     total_ms = step_ev[0].elapsed_time(step_ev[-1])
     per_step = [step_ev[i].elapsed_time(step_ev[i + 1]) for i in range(args.steps)]
-    gemm_ms = sum(a.elapsed_time(b) for a, b in g_ev) / args.steps
+    names = ["route", "dispatch", "gate_up", "down", "shared", "combine"]
+    stage_ms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in g_ev) / args.steps for i, n in enumerate(names)}
+    gemm_ms = stage_ms["gate_up"]
     B.check_device_status(ws_e)
     t_max = total_ms
     if dist:
@@ -243,7 +253,9 @@ def run_ours(args, p, rank, world, local_rank):
         e2e = run_e2e(args, B, WL, cfg, wt, arrays, T, D, dev, stream, dist)
     if rank != 0:
         return None
-    return report(args, p, world, rows, value, ms, per_step, gemm_ms, e2e, n_launch, clocks)
+    res = report(args, p, world, rows, value, ms, per_step, gemm_ms, e2e, n_launch, clocks)
+    res["stage_ms"] = stage_ms
+    return res
 
 
 def run_e2e(args, B, WL, cfg, wt, arrays, T, D, dev, stream, dist):

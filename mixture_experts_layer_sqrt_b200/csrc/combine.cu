@@ -27,6 +27,7 @@ __global__ void __launch_bounds__(256) combine_kernel(int T, int D, int k,
     int rows[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) rows[j] = j < k ? slot_row[(long)t * k + j] : -1;
+#pragma unroll 4
     for (int c = lane * V; c < D; c += 32 * V) {
       float acc[V];
 #pragma unroll

@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(256) gather_kernel(int max_rows, int D,
   for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += warps) {
     const TA *src = x + (long)row_token[r] * D;
     TA *dst = x_perm + (long)r * D;
-#pragma unroll 4
+#pragma unroll 8
     for (int c = lane * V; c < D; c += 32 * V) store16(dst + c, load16(src + c));
   }
 }

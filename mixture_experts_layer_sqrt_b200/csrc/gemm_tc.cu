@@ -4,33 +4,44 @@
 // ops-transformer MoE walkthrough (优化三) packs every expert's rows into one
 // irregular matmul launch.  Here one persistent kernel covers all experts:
 //
-//   gate/up (GATED):  for the rows of expert e, D[128 x 256] accumulates
+//   gate/up (GATED):  for the rows of expert e, D[rows x 256] accumulates
 //                     x_perm[rows] . [W_gate[e] rows n0..n0+127 ; W_up[e] rows n0..n0+127]^T,
 //                     so TMEM columns 0..127 hold g and 128..255 hold u; the
 //                     epilogue forms h = SiLU(clip g) * clip u and stores bf16.
-//   down:             D[128 x 256] = h[rows] . W_down[e][n0..n0+255]^T; the
+//   down:             D[rows x 256] = h[rows] . W_down[e][n0..n0+255]^T; the
 //                     epilogue scales row r by row_weight[r] and stores fp32.
 //
-// Structure (one CTA per SM, 192 threads):
-//   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (bf16, 128-byte
-//               swizzle) per k-block into a 4-stage ring guarded by mbarriers.
-//   warp 1      TMEM owner and MMA issuer: one thread issues 4 tcgen05.mma
-//               (M=128, N=256, K=16) per k-block and commits each stage back
-//               to the producer; two 256-column fp32 accumulators let the
-//               epilogue of tile i overlap the MMAs of tile i+1.
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
-//               output row per thread), fused SwiGLU or routing weight, store.
+// Two tile shapes:
+//   single (PAIR=false)  one CTA per 128x256 tile: A 128x64 + B 256x64 per
+//                        k-block, 4 stages, tcgen05.mma.cta_group::1 M=128.
+//   pair   (PAIR=true)   a cluster of 2 CTAs per 256x256 tile: each CTA stages
+//                        its own 128 rows of A and half of B (128x64 each), the
+//                        leader issues tcgen05.mma.cta_group::2 M=256 and its
+//                        commits arrive on both CTAs' barriers; each CTA's TMEM
+//                        holds its 128 rows.  Half the operand bytes per SM
+//                        and 6 stages.  Used when experts have many rows.
 //
-// Tiles never straddle two experts: expert e owns ceil(rows_e / 128) m-blocks;
-// the tile list (expert-major, then n-block, then m-block, so the CTAs in
-// flight share weight tiles through L2) is derived on the device from
+// Roles (192 threads per CTA):
+//   warp 0      TMA producer into the stage ring guarded by mbarriers.
+//   warp 1      TMEM owner; one thread (the leader's, for pairs) issues the
+//               MMAs: 4 x K=16 per 64-wide k-block, then commits the stage
+//               back to the producers; two 256-column fp32 accumulators let
+//               the epilogue of tile i overlap the MMAs of tile i+1.
+//   warps 2-5   epilogue: tcgen05.ld (one TMEM lane = one output row per
+//               thread), fused SwiGLU or routing weight, global store.
+//
+// Tiles never straddle two experts: expert e owns ceil(rows_e / tile_rows)
+// m-blocks; the tile list (expert-major, then n-block, then m-block, so the
+// CTAs in flight share weight tiles through L2) is derived on the device from
 // expert_offsets, so the host never reads a count.  Rows past the expert's
 // segment are computed from whatever lies there and never stored.
 //
 // Every wait is bounded: after kWaitLimitNs the waiting thread records
-// MOE_ERR_DEVICE_TIMEOUT in the status word, raises a CTA-wide abort flag and
-// every role winds down (copies drained, TMEM freed) instead of hanging.
+// MOE_ERR_DEVICE_TIMEOUT in the status word, raises the abort flag (in both
+// CTAs of a pair) and every role winds down (copies and MMAs drained, TMEM
+// freed) instead of hanging.
 #include <cudaTypedefs.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -39,23 +50,30 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128;          // rows per tile (TMEM lanes)
+constexpr int BM = 128;          // rows per CTA (TMEM lanes)
 constexpr int BN = 256;          // MMA N (accumulator columns)
 constexpr int BK = 64;           // one 128-byte swizzle row of bf16
-constexpr int STAGES = 4;
 constexpr int UMMA_K = 16;
 constexpr int A_BYTES = BM * BK * 2;         // 16 KB
-constexpr int B_BYTES = BN * BK * 2;         // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t TMEM_COLS = 2 * BN;       // two accumulators
 constexpr int MAX_E = 1024;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s
 constexpr int kThreads = 192;
 
+template <bool PAIR>
+struct Cfg {
+  static constexpr int TILE_M = PAIR ? 2 * BM : BM;         // output rows per tile
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;         // B rows staged per CTA
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr uint32_t TX_BYTES = PAIR ? 2 * STAGE_BYTES : STAGE_BYTES;  // per leader barrier phase
+};
+
 struct Smem {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[6];
+  uint64_t empty[6];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t drain;
@@ -78,15 +96,22 @@ struct Params {
   int *status;
 };
 
+template <bool PAIR>
+__device__ __forceinline__ void raise_abort(Smem &sm, uint32_t rank) {
+  *(volatile int *)&sm.abort = 1;
+  if (PAIR) ptx::st_cluster_u32(ptx::map_to_rank(&sm.abort, rank ^ 1u), 1u);
+}
+
 // Bounded wait; false if the CTA is aborting (this thread may have started it).
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Smem &sm, int *status) {
+template <bool PAIR>
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Smem &sm, int *status, uint32_t rank) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   while (true) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if (*(volatile int *)&sm.abort) return false;
     if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
-      *(volatile int *)&sm.abort = 1;
+      raise_abort<PAIR>(sm, rank);
       atomicExch(status, kDevTimeout);
       return false;
     }
@@ -105,6 +130,12 @@ __device__ __forceinline__ void drain_bar(uint64_t *bar, uint32_t parity, int *s
   }
 }
 
+__device__ __forceinline__ void spin_ns(uint64_t ns) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (ptx::globaltimer_ns() - t0 < ns) {
+  }
+}
+
 __device__ __forceinline__ int seg_begin(const Params &p, int e) { return p.offsets ? p.offsets[e] : 0; }
 __device__ __forceinline__ int seg_end(const Params &p, int e) {
   int v = p.offsets ? p.offsets[e + 1] : p.rows;
@@ -116,7 +147,7 @@ struct Tile {
 };
 
 // Largest e with tile_start[e] <= t (empty experts share the next start).
-__device__ __forceinline__ Tile decode_tile(const Params &p, const Smem &sm, int t) {
+__device__ __forceinline__ Tile decode_tile(const Params &p, const Smem &sm, int t, int tile_m) {
   int lo = 0, hi = p.E - 1;
   while (lo < hi) {
     int mid = (lo + hi + 1) >> 1;
@@ -129,33 +160,38 @@ __device__ __forceinline__ Tile decode_tile(const Params &p, const Smem &sm, int
   Tile r;
   r.e = e;
   r.n_blk = local / m_tiles;
-  r.m0 = seg_begin(p, e) + (local - r.n_blk * m_tiles) * BM;
+  r.m0 = seg_begin(p, e) + (local - r.n_blk * m_tiles) * tile_m;
   r.end = seg_end(p, e);
   return r;
 }
 
-template <bool GATED>
+template <bool GATED, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const Params p) {
+  using C = Cfg<PAIR>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // stage buffers first, 1024-byte aligned (the swizzle atoms need it)
   uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *stage_a = base;
-  uint8_t *stage_b = base + STAGES * A_BYTES;
-  Smem &sm = *reinterpret_cast<Smem *>(base + STAGES * STAGE_BYTES);
+  uint8_t *stage_b = base + C::STAGES * A_BYTES;
+  Smem &sm = *reinterpret_cast<Smem *>(base + C::STAGES * C::STAGE_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;  // tile-processing unit
+  const int n_units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   // ---- setup: barriers, TMEM, tile schedule
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < C::STAGES; ++s) {
       ptx::mbar_init(&sm.full[s], 1);
       ptx::mbar_init(&sm.empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&sm.tmem_full[a], 1);
-      ptx::mbar_init(&sm.tmem_empty[a], 4);
+      ptx::mbar_init(&sm.tmem_empty[a], PAIR ? 8 : 4);  // epilogue warps of both CTAs
     }
     ptx::mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -168,18 +204,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (GATED) ptx::prefetch_tmap(&tmB1);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(&sm.tmem_base, TMEM_COLS);
-    ptx::tmem_relinquish();
+    if (PAIR) {
+      ptx::tmem_alloc_pair(&sm.tmem_base, TMEM_COLS);
+      ptx::tmem_relinquish_pair();
+    } else {
+      ptx::tmem_alloc(&sm.tmem_base, TMEM_COLS);
+      ptx::tmem_relinquish();
+    }
   }
   if (warp == 2) {
-    // tile_start[e] = sum over e' < e of ceil(rows_e' / BM) * n_tiles
+    // tile_start[e] = sum over e' < e of ceil(rows_e' / TILE_M) * n_tiles
     int carry = 0;
     for (int e0 = 0; e0 < p.E; e0 += 32) {
       const int e = e0 + lane;
       int v = 0;
       if (e < p.E) {
         int n = seg_end(p, e) - seg_begin(p, e);
-        v = n > 0 ? (n + BM - 1) / BM * p.n_tiles : 0;
+        v = n > 0 ? (n + C::TILE_M - 1) / C::TILE_M * p.n_tiles : 0;
       }
       int incl = v;
 #pragma unroll
@@ -193,97 +234,121 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) sm.tile_start[p.E] = carry;
   }
   ptx::tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  if (PAIR) ptx::cluster_sync();  // the peer's copies may target the leader's barriers from here on
+  else __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = sm.tmem_base;
   const int total_tiles = sm.tile_start[p.E];
   const int k_blocks = (p.K + BK - 1) / BK;
 
   if (warp == 0) {
-    // ================================================= TMA producer
-    uint32_t last_parity[STAGES];
-    bool used[STAGES];
-#pragma unroll
-    for (int s = 0; s < STAGES; ++s) {
-      used[s] = false;
-      last_parity[s] = 0;
-    }
+    // ================================================= TMA producer (both CTAs)
     if (lane == 0) {
+      uint32_t last_parity[C::STAGES];
+      bool used[C::STAGES];
+#pragma unroll
+      for (int s = 0; s < C::STAGES; ++s) {
+        used[s] = false;
+        last_parity[s] = 0;
+      }
       uint32_t it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
-        const Tile tl = decode_tile(p, sm, t);
+      for (int t = unit; t < total_tiles && ok; t += n_units) {
+        const Tile tl = decode_tile(p, sm, t, C::TILE_M);
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1u;
-          if (!wait_bar(&sm.empty[s], ph ^ 1u, sm, p.status)) { ok = false; break; }
-          ptx::mbar_arrive_expect_tx(&sm.full[s], STAGE_BYTES);
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1u;
+          if (!wait_bar<PAIR>(&sm.empty[s], ph ^ 1u, sm, p.status, rank)) { ok = false; break; }
           const int k0 = kb * BK;
-          ptx::tma_load_2d(stage_a + s * A_BYTES, &tmA, &sm.full[s], k0, tl.m0);
-          uint8_t *b = stage_b + s * B_BYTES;
-          if (GATED) {
-            const int n0 = tl.n_blk * (BN / 2);
-            ptx::tma_load_3d(b, &tmB0, &sm.full[s], k0, n0, tl.e);
-            ptx::tma_load_3d(b + B_BYTES / 2, &tmB1, &sm.full[s], k0, n0, tl.e);
+          uint8_t *a = stage_a + s * A_BYTES;
+          uint8_t *b = stage_b + s * C::B_BYTES;
+          if (PAIR) {
+            const uint32_t bar = ptx::map_to_rank(&sm.full[s], 0);   // the leader's barrier
+            if (leader) ptx::mbar_arrive_expect_tx(&sm.full[s], C::TX_BYTES);
+            ptx::tma_load_2d_pair(a, &tmA, bar, k0, tl.m0 + (int)rank * BM);
+            if (GATED) {
+              ptx::tma_load_3d_pair(b, rank == 0 ? &tmB0 : &tmB1, bar, k0, tl.n_blk * (BN / 2), tl.e);
+            } else {
+              ptx::tma_load_3d_pair(b, &tmB0, bar, k0, tl.n_blk * BN + (int)rank * (BN / 2), tl.e);
+            }
           } else {
-            const int n0 = tl.n_blk * BN;
-            ptx::tma_load_3d(b, &tmB0, &sm.full[s], k0, n0, tl.e);
-            ptx::tma_load_3d(b + B_BYTES / 2, &tmB0, &sm.full[s], k0, n0 + BN / 2, tl.e);
+            ptx::mbar_arrive_expect_tx(&sm.full[s], C::TX_BYTES);
+            ptx::tma_load_2d(a, &tmA, &sm.full[s], k0, tl.m0);
+            if (GATED) {
+              const int n0 = tl.n_blk * (BN / 2);
+              ptx::tma_load_3d(b, &tmB0, &sm.full[s], k0, n0, tl.e);
+              ptx::tma_load_3d(b + C::B_BYTES / 2, &tmB1, &sm.full[s], k0, n0, tl.e);
+            } else {
+              const int n0 = tl.n_blk * BN;
+              ptx::tma_load_3d(b, &tmB0, &sm.full[s], k0, n0, tl.e);
+              ptx::tma_load_3d(b + C::B_BYTES / 2, &tmB0, &sm.full[s], k0, n0 + BN / 2, tl.e);
+            }
           }
           used[s] = true;
           last_parity[s] = ph;
         }
       }
-      // drain: every issued copy has landed before shared memory is released
-      for (int s = 0; s < STAGES; ++s)
-        if (used[s]) drain_bar(&sm.full[s], last_parity[s], p.status);
+      // drain: every issued copy has landed before shared memory is released.
+      // The leader's barriers count both CTAs' bytes; a peer that stopped early
+      // gives its last copies time to land.
+      if (leader) {
+        for (int s = 0; s < C::STAGES; ++s)
+          if (used[s]) drain_bar(&sm.full[s], last_parity[s], p.status);
+      } else if (!ok) {
+        spin_ns(1000000);
+      }
     }
   } else if (warp == 1) {
-    // ================================================= MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, BN);
+    // ================================================= MMA issuer (leader)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = ptx::idesc_bf16_f32(C::TILE_M, BN);
       uint32_t it = 0;
       int i = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++i) {
+      for (int t = unit; t < total_tiles && ok; t += n_units, ++i) {
         const int acc = i & 1;
         const uint32_t aph = (i >> 1) & 1u;
-        if (!wait_bar(&sm.tmem_empty[acc], aph ^ 1u, sm, p.status)) break;
+        if (!wait_bar<PAIR>(&sm.tmem_empty[acc], aph ^ 1u, sm, p.status, rank)) break;
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1u;
-          if (!wait_bar(&sm.full[s], ph, sm, p.status)) { ok = false; break; }
+          const int s = it % C::STAGES;
+          const uint32_t ph = (it / C::STAGES) & 1u;
+          if (!wait_bar<PAIR>(&sm.full[s], ph, sm, p.status, rank)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t a_addr = ptx::smem_addr(stage_a + s * A_BYTES);
-          const uint32_t b_addr = ptx::smem_addr(stage_b + s * B_BYTES);
+          const uint32_t b_addr = ptx::smem_addr(stage_b + s * C::B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / UMMA_K; ++k) {
             const uint64_t ad = ptx::desc_kmajor_sw128(a_addr + k * UMMA_K * 2);
             const uint64_t bd = ptx::desc_kmajor_sw128(b_addr + k * UMMA_K * 2);
-            ptx::mma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+            if (PAIR) ptx::mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0);
+            else ptx::mma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0);
           }
-          ptx::mma_commit(&sm.empty[s]);
+          if (PAIR) ptx::mma_commit_pair_mc(&sm.empty[s], 0x3);
+          else ptx::mma_commit(&sm.empty[s]);
         }
         if (!ok) break;
-        ptx::mma_commit(&sm.tmem_full[acc]);
+        if (PAIR) ptx::mma_commit_pair_mc(&sm.tmem_full[acc], 0x3);
+        else ptx::mma_commit(&sm.tmem_full[acc]);
       }
       // drain: all issued MMAs complete before TMEM is released
-      ptx::mma_commit(&sm.drain);
+      if (PAIR) ptx::mma_commit_pair(&sm.drain);
+      else ptx::mma_commit(&sm.drain);
       drain_bar(&sm.drain, 0, p.status);
     }
   } else {
     // ================================================= epilogue (warps 2..5)
     const int q = warp & 3;                 // TMEM lane quadrant this warp may access
-    const int row_in_tile = q * 32 + lane;
+    const int row_in_tile = (int)rank * BM + q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     int i = 0;
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++i) {
-      const Tile tl = decode_tile(p, sm, t);
+    for (int t = unit; t < total_tiles; t += n_units, ++i) {
+      const Tile tl = decode_tile(p, sm, t, C::TILE_M);
       const int acc = i & 1;
       const uint32_t aph = (i >> 1) & 1u;
-      if (!wait_bar(&sm.tmem_full[acc], aph, sm, p.status)) break;
+      if (!wait_bar<PAIR>(&sm.tmem_full[acc], aph, sm, p.status, rank)) break;
       ptx::tc_fence_after();
       const uint32_t tbase = tmem_base + lane_addr + acc * BN;
       const int row = tl.m0 + row_in_tile;
@@ -332,16 +397,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&sm.tmem_empty[acc]);
+      if (lane == 0) {
+        if (PAIR && !leader) ptx::mbar_arrive_cluster(ptx::map_to_rank(&sm.tmem_empty[acc], 0));
+        else ptx::mbar_arrive(&sm.tmem_empty[acc]);
+      }
     }
   }
 
   // ---- teardown
   ptx::tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  if (PAIR) ptx::cluster_sync();  // neither CTA leaves while the pair's copies, MMAs or arrivals are pending
+  else __syncthreads();
   if (warp == 1) {
+    __syncwarp();
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+    if (PAIR) ptx::tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else ptx::tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -359,54 +431,87 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// bf16 tensor [d2][d1][d0] (d0 contiguous) with a {64, 128, 1} box, 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2) {
+// bf16 tensor of rank 2 ([d1][d0]) or 3 ([d2][d1][d0]), d0 contiguous, box
+// {64, 128(, 1)}, 128-byte swizzle, zero fill outside the tensor.
+bool make_map(CUtensorMap *m, const void *ptr, int rank, uint64_t d0, uint64_t d1, uint64_t d2) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {d0, d1, d2};
   cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
   cuuint32_t box[3] = {BK, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d2 > 1 ? 3 : 2, const_cast<void *>(ptr), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-template <bool GATED>
+struct DevInfo {
+  int sms = 0;
+  int pair_clusters = 0;  // co-resident CTA pairs of the pair kernels
+};
+
+template <bool GATED, bool PAIR>
+size_t smem_bytes() {
+  return 1024 + (size_t)Cfg<PAIR>::STAGES * Cfg<PAIR>::STAGE_BYTES + sizeof(Smem);
+}
+
+template <bool GATED, bool PAIR>
 moe_status launch_tc(const Params &p, const void *a, const void *b0, const void *b1, int Nw, cudaStream_t s) {
   // A: [rows, K]; B: [E, Nw, K] (rank 3 even for one group)
   CUtensorMap ta, tb0, tb1;
-  if (!make_map(&ta, a, (uint64_t)p.K, (uint64_t)p.rows, 1)) return MOE_ERR_CUDA;
-  // weights always rank 3 so the kernel's 3-D loads match
-  auto fn = encode_fn();
-  auto map3 = [&](CUtensorMap *m, const void *ptr) {
-    cuuint64_t dims[3] = {(cuuint64_t)p.K, (cuuint64_t)Nw, (cuuint64_t)p.E};
-    cuuint64_t strides[2] = {(cuuint64_t)p.K * 2, (cuuint64_t)p.K * Nw * 2};
-    cuuint32_t box[3] = {BK, 128, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-  };
-  if (!map3(&tb0, b0)) return MOE_ERR_CUDA;
+  if (!make_map(&ta, a, 2, (uint64_t)p.K, (uint64_t)p.rows, 1)) return MOE_ERR_CUDA;
+  if (!make_map(&tb0, b0, 3, (uint64_t)p.K, (uint64_t)Nw, (uint64_t)p.E)) return MOE_ERR_CUDA;
   if (GATED) {
-    if (!map3(&tb1, b1)) return MOE_ERR_CUDA;
+    if (!make_map(&tb1, b1, 3, (uint64_t)p.K, (uint64_t)Nw, (uint64_t)p.E)) return MOE_ERR_CUDA;
   } else {
     tb1 = tb0;
   }
   int dev = 0, sms = 148;
   MOE_CUDA_TRY(cudaGetDevice(&dev));
   MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  const long ub = ((long)(p.rows + BM - 1) / BM + (p.offsets ? p.E : 0)) * p.n_tiles;
-  const int grid = (int)(ub < sms ? ub : sms);
-  if (grid <= 0) return MOE_OK;
-  const size_t smem = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Smem);
-  auto kern = tc_grouped_gemm<GATED>;
+  const size_t smem = smem_bytes<GATED, PAIR>();
+  auto kern = tc_grouped_gemm<GATED, PAIR>;
   MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  kern<<<grid, kThreads, smem, s>>>(ta, tb0, tb1, p);
+  constexpr int TM = Cfg<PAIR>::TILE_M;
+  const long ub = ((long)(p.rows + TM - 1) / TM + (p.offsets ? p.E : 0)) * p.n_tiles;  // tile upper bound
+  if (ub <= 0) return MOE_OK;
+  if (!PAIR) {
+    const int grid = (int)(ub < sms ? ub : sms);
+    kern<<<grid, kThreads, smem, s>>>(ta, tb0, tb1, p);
+  } else {
+    cudaLaunchConfig_t lc = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.blockDim = dim3(kThreads);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = s;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    lc.gridDim = dim3(2);
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &lc) != cudaSuccess || clusters <= 0) clusters = sms / 2;
+    const long units = ub < clusters ? ub : clusters;
+    lc.gridDim = dim3((unsigned)(2 * units));
+    MOE_CUDA_TRY(cudaLaunchKernelEx(&lc, kern, ta, tb0, tb1, p));
+  }
   MOE_LAUNCH_CHECK();
   return MOE_OK;
+}
+
+// Pairs pay off only when groups are so large that the padding of their last
+// 256-row tile is negligible (measured under the power cap, extra padded rows
+// cost more than the pair saves on operand traffic).  The
+// environment variable MOE_TC_TILE = 128 | 256 overrides the choice (for
+// tuning; both paths compute the same result).
+bool use_pair(int rows, int E) {
+  const char *env = getenv("MOE_TC_TILE");
+  if (env && env[0] == '1') return false;
+  if (env && env[0] == '2') return true;
+  return rows >= 2048L * E;
 }
 
 }  // namespace
@@ -432,7 +537,8 @@ moe_status launch_gate_up_tc(const MoEConfig &c, int rows, const void *a, const 
   p.clamp = c.swiglu_clamp;
   p.clamp_mode = c.clamp_mode;
   p.status = status;
-  return launch_tc<true>(p, a, w_gate, w_up, F, s);
+  if (use_pair(rows, p.E)) return launch_tc<true, true>(p, a, w_gate, w_up, F, s);
+  return launch_tc<true, false>(p, a, w_gate, w_up, F, s);
 }
 
 moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
@@ -451,7 +557,8 @@ moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int
   p.clamp = 0.0f;
   p.clamp_mode = 0;
   p.status = status;
-  return launch_tc<false>(p, h, w_down, nullptr, c.hidden_dim, s);
+  if (use_pair(rows, p.E)) return launch_tc<false, true>(p, h, w_down, nullptr, c.hidden_dim, s);
+  return launch_tc<false, false>(p, h, w_down, nullptr, c.hidden_dim, s);
 }
 
 }  // namespace moe

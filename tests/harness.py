@@ -20,7 +20,14 @@ ROUTE_W_RTOL = 1e-5    # routing weights, every dtype
 def small(name: str) -> synth.MoEProblem:
     """A shrunken copy of workload `name` that keeps its features (gate, dtypes,
     capacity, bias, shared expert) and spans several 128x128 tiles with ragged
-    tails, small enough for the oracle to finish in seconds."""
+    tails, small enough for the oracle to finish in seconds.
+
+    A "_pair" suffix gives enough rows per group (>= 2048) for the expert GEMMs
+    to take the CTA-pair (256-row tile) path."""
+    if name == "mixtral_bf16_pair":
+        return synth.PROBLEMS["mixtral_bf16"].with_(name=name, T=4200, D=512, F=384, E=4)
+    if name == "sqrt_fp4_pair":
+        return synth.PROBLEMS["sqrt_fp4"].with_(name=name, T=2100, D=512, F=384, E=12, k=3, Fs=256)
     p = synth.PROBLEMS[name]
     if name == "tiny_f32":
         return p

@@ -19,6 +19,7 @@ from tests import harness as H
 pytestmark = pytest.mark.gpu
 
 NAMES = ["tiny_f32", "mixtral_bf16", "capacity_bf16", "finegrained_bf16", "sqrt_fp4"]
+SMALL_NAMES = NAMES + ["mixtral_bf16_pair", "sqrt_fp4_pair"]
 
 
 @pytest.fixture(scope="module")
@@ -75,7 +76,7 @@ def _stages(B, c: Case):
     return dict(idx=idx, w=w, h=h, y=y, sh=sh, out=out, **d)
 
 
-@pytest.mark.parametrize("name", NAMES)
+@pytest.mark.parametrize("name", SMALL_NAMES)
 def test_stages_small(B, W, name):
     p = H.small(name)
     c = Case(B, W, p)
