@@ -46,11 +46,12 @@ class MoEError(RuntimeError):
         super().__init__(f"{where}: {status_string(status)}")
 
 
-def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with "
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads a build of libmoe_b200.so and declares its C signatures."""
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
                           "`python -m mixture_experts_layer_sqrt_b200.build` (nvcc, sm_100a)")
-    lib = ctypes.CDLL(LIB_PATH)
+    lib = ctypes.CDLL(path)
     P, I, S = c_void_p, c_int, c_size_t
     cfgp, wp = POINTER(MoEConfig), POINTER(MoEWeights)
     sig = {
@@ -79,7 +80,7 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-lib = _load()
+lib = load_library()
 
 # Every function the header declares (checked by the tests).
 EXPORTS = ("moe_status_string", "moe_version", "moe_expert_capacity", "moe_launch_count",
@@ -311,6 +312,52 @@ class MoELayer:
         if x.shape[0] > self.max_tokens:
             raise ValueError("more tokens than the workspace was sized for")
         return forward(self.cfg, x, self.w, self.ws, image_mask, out, topk_idx_out, expert_counts_out, stream)
+
+    def forward_host_batches(self, xs_host, outs_host, masks_host=None) -> None:
+        """Forward a sequence of pinned host batches, copies overlapped with compute.
+
+        Batch i's host-to-device copy runs on its own stream ahead of the
+        compute, and batch i's device-to-host copy on a third stream behind
+        it, so while batch i computes, batch i+1 is uploading and batch i-1
+        downloading; two device buffers alternate.  Every batch is still
+        copied in and out.  Asynchronous: synchronise before reading outs_host.
+        """
+        n = len(xs_host)
+        if n == 0:
+            return
+        comp = torch.cuda.current_stream()
+        if not hasattr(self, "_h2d"):
+            self._h2d, self._d2h = torch.cuda.Stream(), torch.cuda.Stream()
+        h2d, d2h = self._h2d, self._d2h
+        T, D = xs_host[0].shape
+        odt = out_torch_dtype(self.cfg)
+        x_dev = [torch.empty((T, D), dtype=xs_host[0].dtype, device=self.device) for _ in range(2)]
+        o_dev = [torch.empty((T, D), dtype=odt, device=self.device) for _ in range(2)]
+        m_dev = [None, None]
+        if masks_host is not None:
+            m_dev = [torch.empty_like(masks_host[0], device=self.device) for _ in range(2)]
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_free = [torch.cuda.Event() for _ in range(2)]
+        for i in range(n):
+            b = i % 2
+            if i >= 2:
+                h2d.wait_event(ev_done[b])          # batch i-2 no longer reads x_dev[b]
+            with torch.cuda.stream(h2d):
+                x_dev[b].copy_(xs_host[i], non_blocking=True)
+                if masks_host is not None:
+                    m_dev[b].copy_(masks_host[i], non_blocking=True)
+                ev_in[b].record(h2d)
+            comp.wait_event(ev_in[b])
+            if i >= 2:
+                comp.wait_event(ev_free[b])         # batch i-2's result has left o_dev[b]
+            self.forward(x_dev[b], m_dev[b], o_dev[b])
+            ev_done[b].record(comp)
+            d2h.wait_event(ev_done[b])
+            with torch.cuda.stream(d2h):
+                outs_host[i].copy_(o_dev[b], non_blocking=True)
+                ev_free[b].record(d2h)
+        comp.wait_stream(d2h)
 
     def forward_host(self, x_host: torch.Tensor, out_host: torch.Tensor, image_mask_host=None,
                      x_dev=None, out_dev=None, mask_dev=None) -> torch.Tensor:

@@ -1,6 +1,7 @@
 // C ABI of libmoe_b200: argument checks, workspace layout and the order of
 // the stage kernels.  Every compute step runs in the kernels of this library.
 #include <limits.h>
+#include <stdlib.h>
 
 #include <atomic>
 
@@ -76,7 +77,7 @@ ExpertWs carve_expert(Carve &cv, const MoEConfig &c) {
   w.status = cv.take<int>(kStatusBytes / sizeof(int));
   w.wexp = nullptr;
   if (c.expert_dtype == MOE_NVFP4)
-    w.wexp = cv.take<__nv_bfloat16>(2ull * c.num_experts * c.intermediate_dim * c.hidden_dim);
+    w.wexp = cv.take<__nv_bfloat16>(3ull * c.num_experts * c.intermediate_dim * c.hidden_dim);
   return w;
 }
 
@@ -116,6 +117,44 @@ moe_status run_down(const MoEConfig &c, int rows, const void *h, const int32_t *
   return launch_down_simt(cc, rows, h, offsets, wd, c.intermediate_dim, row_weight, y, s);
 }
 
+// The expert projections run as two tensor-core launches; MOE_EXPERTS_FUSED=1
+// selects the single persistent launch instead (same results, bit for bit).
+bool fused_requested() {
+  const char *e = getenv("MOE_EXPERTS_FUSED");
+  return e && e[0] == '1';
+}
+
+// Both expert projections: x_perm -> h -> y.  On the tensor-core path one
+// fused persistent launch; otherwise the CUDA-core kernels one after the other.
+moe_status run_experts(const MoEConfig &c, int rows, const void *a, const int32_t *offsets, const void *wg,
+                       const void *wu, const void *wd, const void *sg, const void *su, const void *sd,
+                       const float *row_weight, void *h, void *y, const ExpertWs &ws, int *sched,
+                       cudaStream_t s) {
+  MoEConfig cc = c;
+  if (c.expert_dtype == MOE_NVFP4) {
+    const long n = (long)c.num_experts * c.intermediate_dim * c.hidden_dim;
+    moe_status st;
+    if ((st = launch_dequant_nvfp4(wg, sg, n, ws.wexp, s)) != MOE_OK) return st;
+    if ((st = launch_dequant_nvfp4(wu, su, n, ws.wexp + n, s)) != MOE_OK) return st;
+    if ((st = launch_dequant_nvfp4(wd, sd, n, ws.wexp + 2 * n, s)) != MOE_OK) return st;
+    wg = ws.wexp;
+    wu = ws.wexp + n;
+    wd = ws.wexp + 2 * n;
+    cc.expert_dtype = MOE_BF16;
+  }
+  if (tc_shapes_ok(cc, c.intermediate_dim)) {
+    if (fused_requested())
+      return launch_experts_fused_tc(cc, rows, a, offsets, wg, wu, wd, row_weight, h, (float *)y, ws.status,
+                                     sched, s);
+    moe_status st = launch_gate_up_tc(cc, rows, a, offsets, wg, wu, c.intermediate_dim, h, ws.status, s);
+    if (st != MOE_OK) return st;
+    return launch_down_tc(cc, rows, h, offsets, wd, c.intermediate_dim, row_weight, (float *)y, ws.status, s);
+  }
+  moe_status st = launch_gate_up_simt(cc, rows, a, offsets, wg, wu, c.intermediate_dim, h, s);
+  if (st != MOE_OK) return st;
+  return launch_down_simt(cc, rows, h, offsets, wd, c.intermediate_dim, row_weight, y, s);
+}
+
 // The shared expert viewed as a one-expert layer of width F_s in the act dtype.
 MoEConfig shared_cfg(const MoEConfig &c) {
   MoEConfig sc = c;
@@ -129,6 +168,7 @@ MoEConfig shared_cfg(const MoEConfig &c) {
 // ---- whole-layer workspace
 struct ForwardWs {
   int *status;
+  int *sched;
   int32_t *topk_idx, *counts, *offsets, *slot_row, *row_token, *chunk_cnt;
   float *topk_w, *row_weight;
   void *x_perm, *h, *y_perm, *sh_y;
@@ -139,6 +179,12 @@ ForwardWs carve_forward(Carve &cv, const MoEConfig &c, int T) {
   const size_t Tk = (size_t)T * c.top_k, E = c.num_experts, D = c.hidden_dim;
   const size_t as = act_size(c);
   w.status = cv.take<int>(kStatusBytes / sizeof(int));
+  size_t ns = fused_sched_ints(c, (int)Tk, true);
+  if (c.shared_intermediate_dim) {
+    const size_t ns2 = fused_sched_ints(c, T, false);
+    if (ns2 > ns) ns = ns2;
+  }
+  w.sched = cv.take<int>(ns);
   w.topk_idx = cv.take<int32_t>(Tk);
   w.topk_w = cv.take<float>(Tk);
   w.counts = cv.take<int32_t>(E);
@@ -156,7 +202,7 @@ ForwardWs carve_forward(Carve &cv, const MoEConfig &c, int T) {
   w.ex.status = w.status;
   w.ex.wexp = nullptr;
   if (c.expert_dtype == MOE_NVFP4)
-    w.ex.wexp = cv.take<__nv_bfloat16>(2ull * c.num_experts * c.intermediate_dim * D);
+    w.ex.wexp = cv.take<__nv_bfloat16>(3ull * c.num_experts * c.intermediate_dim * D);
   return w;
 }
 
@@ -257,6 +303,7 @@ size_t moe_grouped_swiglu_workspace_size(const MoEConfig *cfg, int rows) {
   Carve cv(nullptr);
   carve_expert(cv, *cfg);
   cv.take<char>((size_t)rows * cfg->intermediate_dim * act_size(*cfg));
+  cv.take<int>(fused_sched_ints(*cfg, rows, true));
   return align_up(cv.off, 256);
 }
 
@@ -315,10 +362,9 @@ moe_status moe_grouped_swiglu(const MoEConfig *cfg, int rows, const void *x_perm
   Carve cv(ws);
   ExpertWs ew = carve_expert(cv, *cfg);
   void *h = cv.take<char>((size_t)rows * cfg->intermediate_dim * act_size(*cfg));
-  cudaStream_t s = (cudaStream_t)stream;
-  st = run_gate_up(*cfg, rows, x_perm, expert_offsets, w->w_gate, w->w_up, w->s_gate, w->s_up, h, ew, s);
-  if (st != MOE_OK) return st;
-  return run_down(*cfg, rows, h, expert_offsets, w->w_down, w->s_down, row_weight, y_perm, ew, s);
+  int *sched = cv.take<int>(fused_sched_ints(*cfg, rows, true));
+  return run_experts(*cfg, rows, x_perm, expert_offsets, w->w_gate, w->w_up, w->w_down, w->s_gate, w->s_up,
+                     w->s_down, row_weight, h, y_perm, ew, sched, (cudaStream_t)stream);
 }
 
 moe_status moe_combine(const MoEConfig *cfg, int T, const void *y_perm, const int32_t *slot_row,
@@ -368,17 +414,13 @@ moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeig
   if ((st = launch_dispatch(c, T, idx, f.topk_w, x, counts, f.offsets, f.slot_row, f.row_token,
                             f.row_weight, f.x_perm, f.chunk_cnt, s)) != MOE_OK)
     return st;
-  if ((st = run_gate_up(c, rows, f.x_perm, f.offsets, w->w_gate, w->w_up, w->s_gate, w->s_up, f.h,
-                        f.ex, s)) != MOE_OK)
-    return st;
-  if ((st = run_down(c, rows, f.h, f.offsets, w->w_down, w->s_down, f.row_weight, f.y_perm, f.ex,
-                     s)) != MOE_OK)
+  if ((st = run_experts(c, rows, f.x_perm, f.offsets, w->w_gate, w->w_up, w->w_down, w->s_gate, w->s_up,
+                        w->s_down, f.row_weight, f.h, f.y_perm, f.ex, f.sched, s)) != MOE_OK)
     return st;
   if (c.shared_intermediate_dim) {
     const MoEConfig sc = shared_cfg(c);
-    if ((st = run_gate_up(sc, T, x, nullptr, w->sh_gate, w->sh_up, nullptr, nullptr, f.h, f.ex, s)) != MOE_OK)
-      return st;
-    if ((st = run_down(sc, T, f.h, nullptr, w->sh_down, nullptr, nullptr, f.sh_y, f.ex, s)) != MOE_OK)
+    if ((st = run_experts(sc, T, x, nullptr, w->sh_gate, w->sh_up, w->sh_down, nullptr, nullptr, nullptr, nullptr,
+                          f.h, f.sh_y, f.ex, f.sched, s)) != MOE_OK)
       return st;
   }
   return launch_combine(c, T, f.y_perm, f.slot_row, f.sh_y, out, s);

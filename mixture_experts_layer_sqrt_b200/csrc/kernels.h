@@ -46,6 +46,15 @@ moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int
                           const void *w_down, int F, const float *row_weight, float *y, int *status,
                           cudaStream_t s);
 
+// Both projections in one persistent launch (gate/up tiles, then down tiles
+// that wait for their m-block of h).  sched: fused_sched_ints() ints of
+// scratch, zeroed by the launcher.
+size_t fused_sched_ints(const MoEConfig &c, int rows, bool grouped);
+moe_status launch_experts_fused_tc(const MoEConfig &c, int rows, const void *x_perm, const int32_t *offsets,
+                                   const void *w_gate, const void *w_up, const void *w_down,
+                                   const float *row_weight, void *h, float *y, int *status, int *sched,
+                                   cudaStream_t s);
+
 // dequant.cu -------------------------------------------------------------
 // n_elems values (a multiple of 16): packed [n/2] bytes + scales [n/16] -> bf16 [n].
 moe_status launch_dequant_nvfp4(const void *packed, const void *scales, long n_elems, void *out,

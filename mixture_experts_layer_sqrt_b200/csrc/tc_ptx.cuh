@@ -196,6 +196,20 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t *bar) {
                : "memory");
 }
 
+// ------------------------------------------- cross-CTA flags in global memory
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const int *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(int *p, int v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Orders this thread's generic-proxy global accesses with async-proxy (TMA) ones.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ---------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor of a K-major tile written by TMA with the
 // 128-byte swizzle: rows of 128 bytes (64 bf16), 8-row groups 1024 bytes

@@ -118,6 +118,16 @@ def test_stages_small(B, W, name):
     y_g = H.to_np(g["y"][:R])
     H.assert_close_f32(y_g, y_ref, "y_perm")
 
+    # both projections in one call (the fused persistent kernel on the tensor-core
+    # path): the same tiles as the staged kernels, so the same bits when both use
+    # 128-row tiles; within the fp32 bound otherwise
+    y2 = B.grouped_swiglu(c.cfg, g["x_perm"], g["expert_offsets"], c.w, g["row_weight"])
+    torch.cuda.synchronize()
+    if p.name.endswith("_pair"):
+        H.assert_close_f32(H.to_np(y2[:R]), y_ref, "grouped_swiglu")
+    else:
+        assert torch.equal(y2[:R], g["y"][:R])
+
     # a8 shared expert
     sh_g = None
     if p.Fs:
@@ -143,12 +153,15 @@ def test_stages_small(B, W, name):
     rel = H.assert_close_layer(p, out_g, o["out"], "out")
     print(f"{p.name}: out max|err|/rms = {rel:.3g}")
 
-    # moe_forward gives the staged result bit for bit
+    # moe_forward gives the staged result bit for bit (same tile shapes)
     ws = B.workspace(B.workspace_size(c.cfg, p.T))
     out_f = B.forward(c.cfg, c.x, c.w, ws, c.mask)
     torch.cuda.synchronize()
     B.check_device_status(ws)
-    assert torch.equal(out_f, g["out"])
+    if p.name.endswith("_pair"):
+        H.assert_close_layer(p, H.to_np(out_f), o["out"], "forward")
+    else:
+        assert torch.equal(out_f, g["out"])
 
     # a bf16 output is the fp32 output rounded once (RNE: at most 2^-8 relative)
     c.cfg.out_dtype = B.MOE_BF16
@@ -310,6 +323,42 @@ def test_binding_rejects_mismatched_out(B, W):
         B.forward(c.cfg, c.x, c.w, ws, out=torch.empty((p.T, p.D), dtype=torch.bfloat16, device="cuda"))
     with pytest.raises(ValueError):
         B.forward(c.cfg, c.x, c.w, ws, out=torch.empty((p.T - 1, p.D), dtype=torch.float32, device="cuda"))
+
+
+@pytest.mark.parametrize("name", ["mixtral_bf16", "finegrained_bf16", "sqrt_fp4"])
+def test_fused_expert_kernel_matches(B, W, name, monkeypatch):
+    # the single persistent launch (gate/up tiles, then down tiles waiting on
+    # their m-block of h) gives the two-launch result bit for bit
+    p = H.small(name)
+    c = Case(B, W, p)
+    ws = B.workspace(B.workspace_size(c.cfg, p.T))
+    ref = B.forward(c.cfg, c.x, c.w, ws, c.mask)
+    torch.cuda.synchronize()
+    monkeypatch.setenv("MOE_EXPERTS_FUSED", "1")
+    got = B.forward(c.cfg, c.x, c.w, ws, c.mask)
+    torch.cuda.synchronize()
+    B.check_device_status(ws)
+    assert torch.equal(got, ref)
+
+
+def test_host_batches_overlapped_copies(B, W):
+    # pinned host batches through the overlapped-copy path give the same
+    # outputs as one forward per device batch
+    p = H.small("sqrt_fp4")
+    c = Case(B, W, p)
+    layer = B.MoELayer(c.cfg, c.wt, p.T)
+    xs, refs = [], []
+    for i in range(3):
+        xb = W.to_torch(synth.generate(p.with_(seed=p.seed + 100 + i), experts=False)["x"])
+        refs.append(layer.forward(xb, c.mask).cpu())
+        xs.append(xb.cpu().pin_memory())
+    masks = [c.mask.cpu().pin_memory()] * 3
+    outs = [torch.empty((p.T, p.D), dtype=torch.float32).pin_memory() for _ in range(3)]
+    layer.forward_host_batches(xs, outs, masks)
+    torch.cuda.synchronize()
+    B.check_device_status(layer.ws)
+    for o, r in zip(outs, refs):
+        assert torch.equal(o, r)
 
 
 def test_zero_tokens(B, W):
