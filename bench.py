@@ -177,6 +177,7 @@ def run_ours(args, p, rank, world, local_rank):
     y = torch.empty((T * k, D), dtype=torch.float32, device=dev)
     shy = torch.empty((T, D), dtype=torch.float32, device=dev) if p.Fs else None
     out = torch.empty((T, D), dtype=torch.float32, device=dev)
+    ws_r = B.workspace(256, dev)
     ws_d = B.workspace(B.dispatch_workspace_size(cfg, T), dev)
     ws_e = B.workspace(B.expert_workspace_size(cfg), dev)
     scfg = B.make_config(E=1, k=1, D=D, F=max(p.Fs, 1), clamp=p.clamp, act=p.act, expert=p.act) if p.Fs else None
@@ -192,7 +193,7 @@ def run_ours(args, p, rank, world, local_rank):
     # events: 0 | route | 1 | dispatch | 2 | gate/up | 3 | down | 4 | shared | 5 | combine | 6
     def step(ev=None):
         mark(ev, 0)
-        B.route_topk(cfg, x, w, mask, idx, tw)
+        B.route_topk(cfg, x, w, mask, idx, tw, ws_r)
         mark(ev, 1)
         B.dispatch(cfg, x, idx, tw, disp, ws_d)
         mark(ev, 2)
@@ -213,6 +214,7 @@ def run_ours(args, p, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
     B.check_device_status(ws_e)
+    B.check_device_status(ws_r)
     rows = int(disp["expert_offsets"][-1].item())
 
     dist = None

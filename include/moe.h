@@ -132,6 +132,9 @@ moe_status moe_check_device_status(void *ws, moe_stream_t stream);
 
 /* ------------------------------------------------------------ stage 1: route */
 
+/* Bytes of workspace moe_route_topk needs (its device status word). */
+size_t moe_route_workspace_size(const MoEConfig *cfg, int T);
+
 /* Router GEMM + gate + top-k for T tokens (a1-a2).
  *   x          [T, D] act dtype
  *   w->w_router, w->bias, w->bias_vl as in MoEWeights (other fields unused)
@@ -140,10 +143,13 @@ moe_status moe_check_device_status(void *ws, moe_stream_t stream);
  *              equal keys ordered by lower expert index
  *   topk_w     [T, k] float out: the multipliers (renormalised softmax, or raw
  *              sqrt(softplus(s)))
- * Logits are accumulated in fp32 (ops-transformer walkthrough, 坑三). */
+ *   ws         >= moe_route_workspace_size(cfg, T) bytes (status word)
+ * Logits are accumulated in fp32 (ops-transformer walkthrough, 坑三); with
+ * bf16 activations and 32 < E <= 512 they are computed on the tensor cores and
+ * never leave the SM. */
 moe_status moe_route_topk(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
-                          const uint8_t *image_mask, int32_t *topk_idx, float *topk_w,
-                          moe_stream_t stream);
+                          const uint8_t *image_mask, int32_t *topk_idx, float *topk_w, void *ws,
+                          size_t ws_bytes, moe_stream_t stream);
 
 /* --------------------------------------------------------- stage 2: dispatch */
 

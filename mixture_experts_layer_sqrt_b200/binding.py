@@ -60,7 +60,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_expert_capacity": (I, [I, I, I, I, I]),
         "moe_launch_count": (c_uint64, []),
         "moe_check_device_status": (I, [P, P]),
-        "moe_route_topk": (I, [cfgp, I, P, wp, P, P, P, P]),
+        "moe_route_workspace_size": (S, [cfgp, I]),
+        "moe_route_topk": (I, [cfgp, I, P, wp, P, P, P, P, S, P]),
         "moe_dispatch_workspace_size": (S, [cfgp, I]),
         "moe_dispatch": (I, [cfgp, I, P, P, P, P, P, P, P, P, P, P, S, P]),
         "moe_dispatch_noalloc": (I, [cfgp, I, P, P, P, P, P, P, P, P, P, P]),
@@ -84,7 +85,7 @@ lib = load_library()
 
 # Every function the header declares (checked by the tests).
 EXPORTS = ("moe_status_string", "moe_version", "moe_expert_capacity", "moe_launch_count",
-           "moe_check_device_status", "moe_route_topk", "moe_dispatch_workspace_size",
+           "moe_check_device_status", "moe_route_workspace_size", "moe_route_topk", "moe_dispatch_workspace_size",
            "moe_dispatch", "moe_dispatch_noalloc", "moe_grouped_swiglu_workspace_size", "moe_expert_workspace_size",
            "moe_expert_gate_up", "moe_expert_down", "moe_grouped_swiglu", "moe_combine",
            "moe_workspace_size", "moe_forward")
@@ -151,14 +152,16 @@ def workspace(nbytes: int, device=None) -> torch.Tensor:
 # ------------------------------------------------------------------ stages
 
 def route_topk(cfg: MoEConfig, x: torch.Tensor, w: MoEWeights, image_mask=None,
-               topk_idx=None, topk_w=None, stream=None):
+               topk_idx=None, topk_w=None, ws=None, stream=None):
     T = x.shape[0]
     if topk_idx is None:
         topk_idx = torch.empty((T, cfg.top_k), dtype=torch.int32, device=x.device)
     if topk_w is None:
         topk_w = torch.empty((T, cfg.top_k), dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = workspace(lib.moe_route_workspace_size(ctypes.byref(cfg), T), x.device)
     _check(lib.moe_route_topk(ctypes.byref(cfg), T, _p(x), ctypes.byref(w), _p(image_mask),
-                              _p(topk_idx), _p(topk_w), _stream(stream)), "moe_route_topk")
+                              _p(topk_idx), _p(topk_w), _p(ws), ws.numel(), _stream(stream)), "moe_route_topk")
     return topk_idx, topk_w
 
 

@@ -252,15 +252,22 @@ moe_status moe_check_device_status(void *ws, moe_stream_t stream) {
   return MOE_OK;
 }
 
+size_t moe_route_workspace_size(const MoEConfig *cfg, int T) {
+  if (validate_cfg(cfg) != MOE_OK || T < 0) return 0;
+  return kStatusBytes;
+}
+
 moe_status moe_route_topk(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
-                          const uint8_t *image_mask, int32_t *topk_idx, float *topk_w,
-                          moe_stream_t stream) {
+                          const uint8_t *image_mask, int32_t *topk_idx, float *topk_w, void *ws,
+                          size_t ws_bytes, moe_stream_t stream) {
   moe_status st = validate_cfg(cfg);
   if (st != MOE_OK) return st;
   if ((st = validate_tokens(cfg, T)) != MOE_OK) return st;
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_route_workspace_size(cfg, T)) return MOE_ERR_WORKSPACE;
   if (T == 0) return MOE_OK;
   if (!w || !ok_ptr(x) || !ok_ptr(w->w_router) || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
-  return launch_route(*cfg, T, x, w->w_router, w->bias, w->bias_vl, image_mask, topk_idx, topk_w,
+  return launch_route(*cfg, T, x, w->w_router, w->bias, w->bias_vl, image_mask, topk_idx, topk_w, (int *)ws,
                       (cudaStream_t)stream);
 }
 
@@ -409,7 +416,8 @@ moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeig
   int32_t *counts = expert_counts_out ? expert_counts_out : f.counts;
   const int rows = T * c.top_k;
 
-  if ((st = launch_route(c, T, x, w->w_router, w->bias, w->bias_vl, image_mask, idx, f.topk_w, s)) != MOE_OK)
+  if ((st = launch_route(c, T, x, w->w_router, w->bias, w->bias_vl, image_mask, idx, f.topk_w, f.status, s)) !=
+      MOE_OK)
     return st;
   if ((st = launch_dispatch(c, T, idx, f.topk_w, x, counts, f.offsets, f.slot_row, f.row_token,
                             f.row_weight, f.x_perm, f.chunk_cnt, s)) != MOE_OK)

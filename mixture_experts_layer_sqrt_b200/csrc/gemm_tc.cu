@@ -932,11 +932,13 @@ moe_status launch_fused(const MoEConfig &c, int rows, const void *x_perm, const 
 // cost more than the pair saves on operand traffic).  The
 // environment variable MOE_TC_TILE = 128 | 256 overrides the choice (for
 // tuning; both paths compute the same result).
-bool use_pair(int rows, int E) {
+bool use_pair(int rows, int E, bool gated) {
   const char *env = getenv("MOE_TC_TILE");
   if (env && env[0] == '1') return false;
   if (env && env[0] == '2') return true;
-  return rows >= 2048L * E;
+  // measured (A/B in one process): gate/up gains only for very large groups;
+  // down, with 3.5x longer tiles and fewer of them, already at ~1000 rows
+  return rows >= (gated ? 2048L : 768L) * E;
 }
 
 }  // namespace
@@ -962,7 +964,7 @@ moe_status launch_gate_up_tc(const MoEConfig &c, int rows, const void *a, const 
   p.clamp = c.swiglu_clamp;
   p.clamp_mode = c.clamp_mode;
   p.status = status;
-  if (use_pair(rows, p.E)) return launch_tc<true, true>(p, a, w_gate, w_up, F, s);
+  if (use_pair(rows, p.E, true)) return launch_tc<true, true>(p, a, w_gate, w_up, F, s);
   return launch_tc<true, false>(p, a, w_gate, w_up, F, s);
 }
 
@@ -982,7 +984,7 @@ moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int
   p.clamp = 0.0f;
   p.clamp_mode = 0;
   p.status = status;
-  if (use_pair(rows, p.E)) return launch_tc<false, true>(p, h, w_down, nullptr, c.hidden_dim, s);
+  if (use_pair(rows, p.E, false)) return launch_tc<false, true>(p, h, w_down, nullptr, c.hidden_dim, s);
   return launch_tc<false, false>(p, h, w_down, nullptr, c.hidden_dim, s);
 }
 

@@ -14,9 +14,16 @@ constexpr int kChunkTokens = 256;
 inline int num_chunks(int T) { return (T + kChunkTokens - 1) / kChunkTokens; }
 
 // route.cu ---------------------------------------------------------------
+// Picks the tensor-core router (route_tc.cu) when route_tc_ok(c), else CUDA cores.
 moe_status launch_route(const MoEConfig &c, int T, const void *x, const void *w_router,
                         const float *bias, const float *bias_vl, const uint8_t *image_mask,
-                        int32_t *topk_idx, float *topk_w, cudaStream_t s);
+                        int32_t *topk_idx, float *topk_w, int *status, cudaStream_t s);
+
+// route_tc.cu ------------------------------------------------------------
+bool route_tc_ok(const MoEConfig &c);
+moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void *w_router, const float *bias,
+                           const float *bias_vl, const uint8_t *image_mask, int32_t *topk_idx, float *topk_w,
+                           int *status, cudaStream_t s);
 
 // dispatch.cu ------------------------------------------------------------
 // chunk_cnt: [num_chunks(T), E] int32 scratch.

@@ -232,8 +232,10 @@ moe_status launch_route_t(const MoEConfig &c, int T, const void *x, const void *
 
 moe_status launch_route(const MoEConfig &c, int T, const void *x, const void *w_router,
                         const float *bias, const float *bias_vl, const uint8_t *image_mask,
-                        int32_t *topk_idx, float *topk_w, cudaStream_t s) {
+                        int32_t *topk_idx, float *topk_w, int *status, cudaStream_t s) {
   if (T == 0) return MOE_OK;
+  if (route_tc_ok(c))
+    return launch_route_tc(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, status, s);
   const int E = c.num_experts;
   if (E <= 32) {  // one token per warp, x row slice in registers
     const size_t smem = (size_t)kFewWarps * E * sizeof(float);

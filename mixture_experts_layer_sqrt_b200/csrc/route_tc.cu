@@ -1,0 +1,310 @@
+// Router GEMM + gate + top-k on the tensor cores, for many experts (32 < E <= 512).
+//
+// logits r = W_r x ("FFN、SwiGLU 与 MoE" sec. 3; ops-transformer MoE walkthrough,
+// 优化一) with fp32 accumulation (坑三), then the gate and a partial top-k
+// selection (优化二) -- here without a heap and without writing the logits to
+// HBM: they stay in TMEM and each epilogue thread streams its token's row out
+// in 32-column chunks into a sorted register list.  Softmax mode: weights
+// are the renormalised softmax of the selected (optionally logit-biased)
+// logits.  Sqrt mode: selection on s + bias / bias_vl, weights
+// sqrt(softplus(s)) of the raw score ("5A · MoE fine-grained" sec. 1, 3).
+//
+// One CTA per 128 tokens, 192 threads: warp 0 loads x (128 x 64) and W_r
+// (E_pad x 64, in 128-row boxes) per k-block with TMA; warp 1 issues
+// tcgen05.mma (M=128, N <= 256 per instruction, two instructions when
+// E_pad > 256) into an fp32 TMEM accumulator of E_pad columns; warps 2-5 own
+// one token (TMEM lane) per thread for the selection.  All waits bounded.
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_ptx.cuh"
+#include "tma_host.h"
+
+namespace moe {
+namespace {
+
+constexpr int RBM = 128;
+constexpr int RBK = 64;
+constexpr int kRThreads = 192;
+constexpr int kMaxEPad = 512;
+constexpr int kMaxStages = 8;
+constexpr uint64_t kRWaitNs = 2000000000ull;
+constexpr uint64_t kRDrainNs = 200000000ull;
+
+struct RParams {
+  int T, D, E, E_pad, k, gate, stages, b_rows;
+  uint32_t tmem_cols;
+  const float *bias;
+  const float *bias_vl;
+  const uint8_t *image_mask;
+  int32_t *topk_idx;
+  float *topk_w;
+  int *status;
+};
+
+struct RSmem {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  uint64_t acc_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  float bias[kMaxEPad];
+  float bias_vl[kMaxEPad];
+};
+
+__device__ __forceinline__ bool rwait(uint64_t *bar, uint32_t parity, RSmem &sm, int *status) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (true) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*(volatile int *)&sm.abort) return false;
+    if (ptx::globaltimer_ns() - t0 > kRWaitNs) {
+      *(volatile int *)&sm.abort = 1;
+      atomicExch(status, kDevTimeout);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void rdrain(uint64_t *bar, uint32_t parity, int *status) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    if (ptx::globaltimer_ns() - t0 > kRDrainNs) {
+      atomicExch(status, kDevTimeout);
+      return;
+    }
+  }
+}
+
+// Insert (v, e, l) into a list sorted by descending key, equal keys ordered by
+// lower expert index; the smallest entry falls off the end.
+template <int KMAX>
+__device__ __forceinline__ void topk_insert(float (&kv)[KMAX], int (&ke)[KMAX], float (&kl)[KMAX], float v, int e,
+                                            float l) {
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    const bool better = v > kv[j] || (v == kv[j] && e < ke[j]);
+    if (better) {
+      const float tv = kv[j], tl = kl[j];
+      const int te = ke[j];
+      kv[j] = v;
+      ke[j] = e;
+      kl[j] = l;
+      v = tv;
+      e = te;
+      l = tl;
+    }
+  }
+}
+
+template <int KMAX>
+__global__ void __launch_bounds__(kRThreads, 1)
+    tc_route_topk(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, const RParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const int a_bytes = RBM * RBK * 2;
+  const int b_bytes = p.b_rows * RBK * 2;
+  const int stage_bytes = a_bytes + b_bytes;
+  RSmem &sm = *reinterpret_cast<RSmem *>(base + (size_t)p.stages * stage_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * RBM;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      ptx::mbar_init(&sm.full[s], 1);
+      ptx::mbar_init(&sm.empty[s], 1);
+    }
+    ptx::mbar_init(&sm.acc_full, 1);
+    ptx::mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    ptx::fence_mbar_init();
+    ptx::fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tmX);
+    ptx::prefetch_tmap(&tmW);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&sm.tmem_base, p.tmem_cols);
+    ptx::tmem_relinquish();
+  }
+  if (warp >= 2) {
+    for (int e = threadIdx.x - 64; e < p.E; e += kRThreads - 64) {
+      sm.bias[e] = p.bias ? p.bias[e] : 0.0f;
+      sm.bias_vl[e] = p.bias_vl ? p.bias_vl[e] : 0.0f;
+    }
+  }
+  ptx::tc_fence_before();
+  __syncwarp();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = sm.tmem_base;
+  const int k_blocks = p.D / RBK;
+  const int n_boxes = p.b_rows / 128;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int last = -1;
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        const int s = kb % p.stages;
+        const uint32_t ph = (kb / p.stages) & 1u;
+        if (!rwait(&sm.empty[s], ph ^ 1u, sm, p.status)) break;
+        ptx::mbar_arrive_expect_tx(&sm.full[s], stage_bytes);
+        uint8_t *a = base + (size_t)s * stage_bytes;
+        ptx::tma_load_2d(a, &tmX, &sm.full[s], kb * RBK, m0);
+        for (int j = 0; j < n_boxes; ++j) ptx::tma_load_2d(a + a_bytes + j * 16384, &tmW, &sm.full[s], kb * RBK, j * 128);
+        last = kb;
+      }
+      // drain the copies still in flight (the last `stages` k-blocks)
+      for (int kb = last - p.stages + 1; kb <= last; ++kb)
+        if (kb >= 0) rdrain(&sm.full[kb % p.stages], (kb / p.stages) & 1u, p.status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const int n0 = p.E_pad < 256 ? p.E_pad : 256;
+      const int n1 = p.E_pad - n0;
+      const uint32_t id0 = ptx::idesc_bf16_f32(RBM, n0);
+      const uint32_t id1 = n1 > 0 ? ptx::idesc_bf16_f32(RBM, n1) : 0u;
+      bool ok = true;
+      for (int kb = 0; kb < k_blocks; ++kb) {
+        const int s = kb % p.stages;
+        const uint32_t ph = (kb / p.stages) & 1u;
+        if (!rwait(&sm.full[s], ph, sm, p.status)) { ok = false; break; }
+        ptx::tc_fence_after();
+        const uint32_t a_addr = ptx::smem_addr(base + (size_t)s * stage_bytes);
+        const uint32_t b_addr = a_addr + a_bytes;
+#pragma unroll
+        for (int k = 0; k < RBK / 16; ++k) {
+          const uint64_t ad = ptx::desc_kmajor_sw128(a_addr + k * 32);
+          ptx::mma_bf16(tmem_base, ad, ptx::desc_kmajor_sw128(b_addr + k * 32), id0, (kb | k) != 0);
+          if (n1 > 0)
+            ptx::mma_bf16(tmem_base + 256, ad, ptx::desc_kmajor_sw128(b_addr + 256 * 128 + k * 32), id1,
+                          (kb | k) != 0);
+        }
+        ptx::mma_commit(&sm.empty[s]);
+      }
+      if (ok) ptx::mma_commit(&sm.acc_full);
+      ptx::mma_commit(&sm.drain);
+      rdrain(&sm.drain, 0, p.status);
+    }
+  } else {
+    // ---- selection: one token (TMEM lane) per thread
+    const int q = warp & 3;
+    const int row = m0 + q * 32 + lane;
+    bool ok = true;
+    if (lane == 0) ok = rwait(&sm.acc_full, 0, sm, p.status);
+    if (__shfl_sync(0xffffffffu, ok, 0)) {
+      ptx::tc_fence_after();
+      const bool live = row < p.T;
+      const bool sqrt_gate = p.gate == MOE_GATE_SQRT_SOFTPLUS_RAW;
+      const float *sel = (sqrt_gate && live && p.bias_vl && p.image_mask && p.image_mask[row]) ? sm.bias_vl : sm.bias;
+      float kv[KMAX], kl[KMAX];
+      int ke[KMAX];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        kv[j] = -INFINITY;
+        kl[j] = 0.0f;
+        ke[j] = 0x7fffffff;
+      }
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16);
+      for (int c = 0; c < p.E_pad; c += 32) {
+        uint32_t v[32];
+        ptx::tmem_ld32(tbase + c, v);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int e = c + j;
+          if (e < p.E) {
+            float l = __uint_as_float(v[j]);
+            if (!sqrt_gate) l += sm.bias[e];  // router logit bias: selection and weight
+            float key = sqrt_gate ? l + sel[e] : l;
+            if (key != key) key = -INFINITY;
+            const bool cand = key > kv[KMAX - 1] || (key == kv[KMAX - 1] && e < ke[KMAX - 1]);
+            if (cand) topk_insert<KMAX>(kv, ke, kl, key, e, l);
+          }
+        }
+      }
+      if (live) {
+        float w[KMAX];
+        if (!sqrt_gate) {
+          float sum = 0.0f;
+#pragma unroll
+          for (int j = 0; j < KMAX; ++j) {
+            w[j] = j < p.k ? expf(kl[j] - kl[0]) : 0.0f;
+            sum += w[j];
+          }
+#pragma unroll
+          for (int j = 0; j < KMAX; ++j) w[j] = w[j] / sum;
+        } else {
+#pragma unroll
+          for (int j = 0; j < KMAX; ++j) w[j] = sqrtf(softplus_f32(kl[j]));
+        }
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+          if (j < p.k) {
+            p.topk_idx[(long)row * p.k + j] = ke[j];
+            p.topk_w[(long)row * p.k + j] = w[j];
+          }
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncwarp();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+}
+
+}  // namespace
+
+bool route_tc_ok(const MoEConfig &c) {
+  return c.act_dtype == MOE_BF16 && c.num_experts > 32 && c.num_experts <= kMaxEPad && c.top_k <= 16 &&
+         c.hidden_dim % RBK == 0 && tma_encode_fn() != nullptr;
+}
+
+moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void *w_router, const float *bias,
+                           const float *bias_vl, const uint8_t *image_mask, int32_t *topk_idx, float *topk_w,
+                           int *status, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  RParams p;
+  p.T = T;
+  p.D = c.hidden_dim;
+  p.E = c.num_experts;
+  p.E_pad = (c.num_experts + 15) / 16 * 16;
+  p.b_rows = (p.E_pad + 127) / 128 * 128;
+  p.k = c.top_k;
+  p.gate = c.gate;
+  uint32_t cols = 32;
+  while (cols < (uint32_t)p.E_pad) cols <<= 1;
+  p.tmem_cols = cols;
+  p.bias = bias;
+  p.bias_vl = bias_vl;
+  p.image_mask = image_mask;
+  p.topk_idx = topk_idx;
+  p.topk_w = topk_w;
+  p.status = status;
+  const int stage_bytes = RBM * RBK * 2 + p.b_rows * RBK * 2;
+  int stages = (192 * 1024) / stage_bytes;
+  p.stages = stages > kMaxStages ? kMaxStages : stages;
+  CUtensorMap tx, tw;
+  if (!tma_map_bf16(&tx, x, 2, (uint64_t)p.D, (uint64_t)T, 1)) return MOE_ERR_CUDA;
+  if (!tma_map_bf16(&tw, w_router, 2, (uint64_t)p.D, (uint64_t)p.E, 1)) return MOE_ERR_CUDA;
+  const size_t smem = 1024 + (size_t)p.stages * stage_bytes + sizeof(RSmem);
+  const dim3 grid((T + RBM - 1) / RBM);
+  if (c.top_k <= 8) {
+    MOE_CUDA_TRY(cudaFuncSetAttribute(tc_route_topk<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    tc_route_topk<8><<<grid, kRThreads, smem, s>>>(tx, tw, p);
+  } else {
+    MOE_CUDA_TRY(cudaFuncSetAttribute(tc_route_topk<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    tc_route_topk<16><<<grid, kRThreads, smem, s>>>(tx, tw, p);
+  }
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+}  // namespace moe

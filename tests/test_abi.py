@@ -86,19 +86,22 @@ def test_workspace_sizes(B):
 def test_invalid_config_rejected_on_host(B, kw, status):
     c = _cfg(B, **kw)
     w = B.MoEWeights()
-    st = B.lib.moe_route_topk(ctypes.byref(c), 4, 16, ctypes.byref(w), None, 16, 16, None)
+    st = B.lib.moe_route_topk(ctypes.byref(c), 4, 16, ctypes.byref(w), None, 16, 16, 16, 256, None)
     assert st == status
 
 
 def test_null_and_misaligned_pointers_rejected(B):
     c = _cfg(B)
     w = B.MoEWeights(w_router=16)
-    assert B.lib.moe_route_topk(ctypes.byref(c), 4, None, ctypes.byref(w), None, 16, 16, None) == B.MOE_ERR_INVALID_ARG
-    assert B.lib.moe_route_topk(ctypes.byref(c), 4, 24, ctypes.byref(w), None, 16, 16, None) == B.MOE_ERR_INVALID_ARG
-    assert B.lib.moe_route_topk(None, 4, 16, ctypes.byref(w), None, 16, 16, None) == B.MOE_ERR_INVALID_ARG
-    assert B.lib.moe_route_topk(ctypes.byref(c), -1, 16, ctypes.byref(w), None, 16, 16, None) == B.MOE_ERR_INVALID_ARG
+    assert B.lib.moe_route_topk(ctypes.byref(c), 4, None, ctypes.byref(w), None, 16, 16, 16, 256, None) == B.MOE_ERR_INVALID_ARG
+    assert B.lib.moe_route_topk(ctypes.byref(c), 4, 24, ctypes.byref(w), None, 16, 16, 16, 256, None) == B.MOE_ERR_INVALID_ARG
+    assert B.lib.moe_route_topk(None, 4, 16, ctypes.byref(w), None, 16, 16, 16, 256, None) == B.MOE_ERR_INVALID_ARG
+    assert B.lib.moe_route_topk(ctypes.byref(c), -1, 16, ctypes.byref(w), None, 16, 16, 16, 256, None) == B.MOE_ERR_INVALID_ARG
     # zero tokens: nothing to do, nothing launched
-    assert B.lib.moe_route_topk(ctypes.byref(c), 0, None, None, None, None, None, None) == B.MOE_OK
+    assert B.lib.moe_route_topk(ctypes.byref(c), 0, None, None, None, None, None, 16, 256, None) == B.MOE_OK
+    # workspace missing or too small
+    assert B.lib.moe_route_topk(ctypes.byref(c), 4, 16, ctypes.byref(w), None, 16, 16, None, 0, None) == B.MOE_ERR_INVALID_ARG
+    assert B.lib.moe_route_topk(ctypes.byref(c), 4, 16, ctypes.byref(w), None, 16, 16, 16, 8, None) == B.MOE_ERR_WORKSPACE
     assert B.lib.moe_combine(ctypes.byref(c), 4, None, 16, None, 16, None) == B.MOE_ERR_INVALID_ARG
 
 

@@ -220,6 +220,25 @@ def test_full_size_sampled(B, W, name, n_sample):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("E,k,gate,bias", [(33, 16, "sqrt_softplus", "uniform"), (48, 4, "softmax", "none"),
+                                           (64, 2, "softmax", "zipf"), (128, 16, "softmax", "none"),
+                                           (300, 6, "sqrt_softplus", "uniform"), (512, 8, "softmax", "none")])
+def test_route_many_experts(B, W, E, k, gate, bias):
+    # the tensor-core router (E > 32): ragged 128-token tiles, padded expert
+    # columns, one or two MMA column blocks, both gates and both biases
+    p = synth.MoEProblem("route", T=300, D=512, F=128, E=E, k=k, gate=gate, bias=bias, seed=21)
+    a = synth.generate(p, experts=False)
+    cfg = W.config_of(p)
+    wt = {n: W.to_torch(a.get(n)) for n in ("w_router", "bias", "bias_vl")}
+    x = W.to_torch(a["x"])
+    idx, w = B.route_topk(cfg, x, B.make_weights(wt), W.to_torch(a.get("image_mask")))
+    torch.cuda.synchronize()
+    L = H.oracle_layer(p, a)
+    logits, idx_o, w_o, keys = H.oracle_route(p, L, a)
+    flips, ties = H.check_route(p, H.to_np(idx), H.to_np(w), logits, idx_o, keys, a.get("bias"))
+    print(f"route E={E} k={k} {gate}: near-ties {ties}, flipped {flips}")
+
+
 # ---------------------------------------------------------------- edge cases
 
 def _edge_case(B, W, p, bias=None, capacity=None, clamp_mode="preact", x_scale=None):
