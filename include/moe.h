@@ -145,8 +145,8 @@ size_t moe_route_workspace_size(const MoEConfig *cfg, int T);
  *              sqrt(softplus(s)))
  *   ws         >= moe_route_workspace_size(cfg, T) bytes (status word)
  * Logits are accumulated in fp32 (ops-transformer walkthrough, 坑三); with
- * bf16 activations and 32 < E <= 512 they are computed on the tensor cores and
- * never leave the SM. */
+ * bf16 activations and 32 < E <= 512 they are computed on the tensor cores
+ * and never leave the SM. */
 moe_status moe_route_topk(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
                           const uint8_t *image_mask, int32_t *topk_idx, float *topk_w, void *ws,
                           size_t ws_bytes, moe_stream_t stream);

@@ -220,12 +220,14 @@ def test_full_size_sampled(B, W, name, n_sample):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("E,k,gate,bias", [(33, 16, "sqrt_softplus", "uniform"), (48, 4, "softmax", "none"),
+@pytest.mark.parametrize("E,k,gate,bias", [(8, 2, "softmax", "none"), (6, 6, "softmax", "zipf"),
+                                           (33, 16, "sqrt_softplus", "uniform"), (48, 4, "softmax", "none"),
                                            (64, 2, "softmax", "zipf"), (128, 16, "softmax", "none"),
                                            (300, 6, "sqrt_softplus", "uniform"), (512, 8, "softmax", "none")])
 def test_route_many_experts(B, W, E, k, gate, bias):
-    # the tensor-core router (E > 32): ragged 128-token tiles, padded expert
-    # columns, one or two MMA column blocks, both gates and both biases
+    # the router on both paths (CUDA cores up to 32 experts, tensor cores
+    # above): ragged 128-token tiles, padded expert columns, one or two MMA
+    # column blocks, k = E, both gates and both biases
     p = synth.MoEProblem("route", T=300, D=512, F=128, E=E, k=k, gate=gate, bias=bias, seed=21)
     a = synth.generate(p, experts=False)
     cfg = W.config_of(p)
