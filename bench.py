@@ -177,7 +177,7 @@ def run_ours(args, p, rank, world, local_rank):
     y = torch.empty((T * k, D), dtype=torch.float32, device=dev)
     shy = torch.empty((T, D), dtype=torch.float32, device=dev) if p.Fs else None
     out = torch.empty((T, D), dtype=torch.float32, device=dev)
-    ws_r = B.workspace(256, dev)
+    ws_r = B.workspace(B.route_workspace_size(cfg, T), dev)
     ws_d = B.workspace(B.dispatch_workspace_size(cfg, T), dev)
     ws_e = B.workspace(B.expert_workspace_size(cfg), dev)
     scfg = B.make_config(E=1, k=1, D=D, F=max(p.Fs, 1), clamp=p.clamp, act=p.act, expert=p.act) if p.Fs else None

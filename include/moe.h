@@ -166,7 +166,9 @@ size_t moe_dispatch_workspace_size(const MoEConfig *cfg, int T);
  *   slot_row       [T, k] int32 out: row of (t, j), or -1 if dropped
  *   row_token      [T*k] int32 out: token of each row (first R valid)
  *   row_weight     [T*k] float out: topk_w of each row (first R valid)
- *   x_perm         [T*k, D] act dtype out: x_perm[r] = x[row_token[r]], r < R
+ *   x_perm         [T*k, D] act dtype out: x_perm[r] = x[row_token[r]], r < R;
+ *                  or NULL: only the maps are built (moe_expert_gate_up can
+ *                  gather the rows from x itself), and x may then be NULL
  *   ws             >= moe_dispatch_workspace_size(cfg, T) bytes
  * Deterministic: no global atomics; counts and rows are identical run to run. */
 moe_status moe_dispatch(const MoEConfig *cfg, int T, const int32_t *topk_idx, const float *topk_w,
@@ -204,16 +206,23 @@ size_t moe_grouped_swiglu_workspace_size(const MoEConfig *cfg, int rows);
 size_t moe_expert_workspace_size(const MoEConfig *cfg);
 
 /* Grouped gate/up GEMM with the SwiGLU epilogue (a6).  For every expert e and
- * row r in [expert_offsets[e], expert_offsets[e+1]):
- *   h[r, :] = SiLU(clip(x_perm[r] W_gate[e]^T)) * clip(x_perm[r] W_up[e]^T)
+ * row r in [expert_offsets[e], expert_offsets[e+1]), with A[r] the r-th input row:
+ *   h[r, :] = SiLU(clip(A[r] W_gate[e]^T)) * clip(A[r] W_up[e]^T)
  * (clip per cfg->swiglu_clamp / clamp_mode), fp32 accumulation, stored in the
  * act dtype.  expert_offsets == NULL means one group of `rows` rows using
  * expert 0's weights.  `rows` bounds every offset (R <= rows).
+ *   a, row_token  row_token == NULL: A = a, dense [rows, D] (x_perm).
+ *                 Otherwise A[r] = a[row_token[r]] with a = x [a_rows, D] and
+ *                 row_token the map from moe_dispatch: the rows are gathered
+ *                 by the GEMM's own loads and no x_perm is needed.  On the
+ *                 tensor-core path the gather issues one TMA copy per 4 rows x
+ *                 64 columns, slower than moe_dispatch's gather plus a dense
+ *                 A at large sizes; moe_forward uses the dense form.
  *   w_gate/w_up [E, F, D] in cfg->expert_dtype; s_gate/s_up NVFP4 scales or NULL
  *   h           [rows, F] out */
-moe_status moe_expert_gate_up(const MoEConfig *cfg, int rows, const void *x_perm,
-                              const int32_t *expert_offsets, const void *w_gate, const void *w_up,
-                              const void *s_gate, const void *s_up, void *h, void *ws,
+moe_status moe_expert_gate_up(const MoEConfig *cfg, int rows, const void *a, int a_rows,
+                              const int32_t *row_token, const int32_t *expert_offsets, const void *w_gate,
+                              const void *w_up, const void *s_gate, const void *s_up, void *h, void *ws,
                               size_t ws_bytes, moe_stream_t stream);
 
 /* Grouped down GEMM with the routing-weight epilogue (a7):

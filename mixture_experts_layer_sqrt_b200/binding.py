@@ -67,7 +67,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_dispatch_noalloc": (I, [cfgp, I, P, P, P, P, P, P, P, P, P, P]),
         "moe_grouped_swiglu_workspace_size": (S, [cfgp, I]),
         "moe_expert_workspace_size": (S, [cfgp]),
-        "moe_expert_gate_up": (I, [cfgp, I, P, P, P, P, P, P, P, P, S, P]),
+        "moe_expert_gate_up": (I, [cfgp, I, P, I, P, P, P, P, P, P, P, P, S, P]),
         "moe_expert_down": (I, [cfgp, I, P, P, P, P, P, P, P, S, P]),
         "moe_grouped_swiglu": (I, [cfgp, I, P, P, wp, P, P, P, S, P]),
         "moe_combine": (I, [cfgp, I, P, P, P, P, P]),
@@ -167,7 +167,8 @@ def route_topk(cfg: MoEConfig, x: torch.Tensor, w: MoEWeights, image_mask=None,
 
 def dispatch(cfg: MoEConfig, x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,
              out: Optional[Dict[str, torch.Tensor]] = None, ws: Optional[torch.Tensor] = None,
-             stream=None) -> Dict[str, torch.Tensor]:
+             stream=None, gather: bool = True) -> Dict[str, torch.Tensor]:
+    """gather=False builds the row maps only (x_perm None): the gate/up GEMM gathers from x."""
     T, D, E, k = x.shape[0], cfg.hidden_dim, cfg.num_experts, cfg.top_k
     dev = x.device
     o = out or dict(
@@ -176,7 +177,7 @@ def dispatch(cfg: MoEConfig, x: torch.Tensor, topk_idx: torch.Tensor, topk_w: to
         slot_row=torch.empty((T, k), dtype=torch.int32, device=dev),
         row_token=torch.empty(T * k, dtype=torch.int32, device=dev),
         row_weight=torch.empty(T * k, dtype=torch.float32, device=dev),
-        x_perm=torch.empty((T * k, D), dtype=x.dtype, device=dev))
+        x_perm=torch.empty((T * k, D), dtype=x.dtype, device=dev) if gather else None)
     if ws is None:
         ws = workspace(lib.moe_dispatch_workspace_size(ctypes.byref(cfg), T), dev)
     _check(lib.moe_dispatch(ctypes.byref(cfg), T, _p(topk_idx), _p(topk_w), _p(x),
@@ -205,15 +206,18 @@ def dispatch_noalloc(cfg: MoEConfig, x: torch.Tensor, topk_idx: torch.Tensor, to
     return o
 
 
-def expert_gate_up(cfg: MoEConfig, x_perm: torch.Tensor, offsets: Optional[torch.Tensor], w_gate, w_up,
-                   s_gate=None, s_up=None, h=None, ws=None, rows=None, stream=None) -> torch.Tensor:
-    rows = x_perm.shape[0] if rows is None else rows
+def expert_gate_up(cfg: MoEConfig, a: torch.Tensor, offsets: Optional[torch.Tensor], w_gate, w_up,
+                   s_gate=None, s_up=None, h=None, ws=None, rows=None, row_token=None, stream=None) -> torch.Tensor:
+    """a = x_perm (dense rows), or with row_token: a = x and row r is a[row_token[r]]."""
+    if rows is None:
+        rows = row_token.shape[0] if row_token is not None else a.shape[0]
     if h is None:
-        h = torch.empty((rows, cfg.intermediate_dim), dtype=x_perm.dtype, device=x_perm.device)
+        h = torch.empty((rows, cfg.intermediate_dim), dtype=a.dtype, device=a.device)
     if ws is None:
-        ws = workspace(lib.moe_expert_workspace_size(ctypes.byref(cfg)), x_perm.device)
-    _check(lib.moe_expert_gate_up(ctypes.byref(cfg), rows, _p(x_perm), _p(offsets), _p(w_gate), _p(w_up),
-                                  _p(s_gate), _p(s_up), _p(h), _p(ws), ws.numel(), _stream(stream)),
+        ws = workspace(lib.moe_expert_workspace_size(ctypes.byref(cfg)), a.device)
+    _check(lib.moe_expert_gate_up(ctypes.byref(cfg), rows, _p(a), a.shape[0], _p(row_token), _p(offsets),
+                                  _p(w_gate), _p(w_up), _p(s_gate), _p(s_up), _p(h), _p(ws), ws.numel(),
+                                  _stream(stream)),
            "moe_expert_gate_up")
     return h
 
@@ -268,6 +272,10 @@ def dispatch_workspace_size(cfg: MoEConfig, T: int) -> int:
 
 def expert_workspace_size(cfg: MoEConfig) -> int:
     return int(lib.moe_expert_workspace_size(ctypes.byref(cfg)))
+
+
+def route_workspace_size(cfg: MoEConfig, T: int) -> int:
+    return int(lib.moe_route_workspace_size(ctypes.byref(cfg), T))
 
 
 def grouped_swiglu_workspace_size(cfg: MoEConfig, rows: int) -> int:

@@ -82,9 +82,9 @@ ExpertWs carve_expert(Carve &cv, const MoEConfig &c) {
 }
 
 // ---- gate/up and down with dtype handling (offsets == null: single group)
-moe_status run_gate_up(const MoEConfig &c, int rows, const void *a, const int32_t *offsets,
-                       const void *wg, const void *wu, const void *sg, const void *su, void *h,
-                       const ExpertWs &ws, cudaStream_t s) {
+moe_status run_gate_up(const MoEConfig &c, int rows, const void *a, int a_rows, const int32_t *row_token,
+                       const int32_t *offsets, const void *wg, const void *wu, const void *sg, const void *su,
+                       void *h, const ExpertWs &ws, cudaStream_t s) {
   MoEConfig cc = c;
   if (c.expert_dtype == MOE_NVFP4) {
     const long n = (long)c.num_experts * c.intermediate_dim * c.hidden_dim;
@@ -97,8 +97,8 @@ moe_status run_gate_up(const MoEConfig &c, int rows, const void *a, const int32_
     cc.expert_dtype = MOE_BF16;
   }
   if (tc_shapes_ok(cc, c.intermediate_dim))
-    return launch_gate_up_tc(cc, rows, a, offsets, wg, wu, c.intermediate_dim, h, ws.status, s);
-  return launch_gate_up_simt(cc, rows, a, offsets, wg, wu, c.intermediate_dim, h, s);
+    return launch_gate_up_tc(cc, rows, a, a_rows, row_token, offsets, wg, wu, c.intermediate_dim, h, ws.status, s);
+  return launch_gate_up_simt(cc, rows, a, row_token, offsets, wg, wu, c.intermediate_dim, h, s);
 }
 
 moe_status run_down(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
@@ -126,10 +126,10 @@ bool fused_requested() {
 
 // Both expert projections: x_perm -> h -> y.  On the tensor-core path one
 // fused persistent launch; otherwise the CUDA-core kernels one after the other.
-moe_status run_experts(const MoEConfig &c, int rows, const void *a, const int32_t *offsets, const void *wg,
-                       const void *wu, const void *wd, const void *sg, const void *su, const void *sd,
-                       const float *row_weight, void *h, void *y, const ExpertWs &ws, int *sched,
-                       cudaStream_t s) {
+moe_status run_experts(const MoEConfig &c, int rows, const void *a, int a_rows, const int32_t *row_token,
+                       const int32_t *offsets, const void *wg, const void *wu, const void *wd, const void *sg,
+                       const void *su, const void *sd, const float *row_weight, void *h, void *y,
+                       const ExpertWs &ws, int *sched, cudaStream_t s) {
   MoEConfig cc = c;
   if (c.expert_dtype == MOE_NVFP4) {
     const long n = (long)c.num_experts * c.intermediate_dim * c.hidden_dim;
@@ -143,14 +143,15 @@ moe_status run_experts(const MoEConfig &c, int rows, const void *a, const int32_
     cc.expert_dtype = MOE_BF16;
   }
   if (tc_shapes_ok(cc, c.intermediate_dim)) {
-    if (fused_requested())
+    if (fused_requested() && !row_token)
       return launch_experts_fused_tc(cc, rows, a, offsets, wg, wu, wd, row_weight, h, (float *)y, ws.status,
                                      sched, s);
-    moe_status st = launch_gate_up_tc(cc, rows, a, offsets, wg, wu, c.intermediate_dim, h, ws.status, s);
+    moe_status st = launch_gate_up_tc(cc, rows, a, a_rows, row_token, offsets, wg, wu, c.intermediate_dim, h,
+                                      ws.status, s);
     if (st != MOE_OK) return st;
     return launch_down_tc(cc, rows, h, offsets, wd, c.intermediate_dim, row_weight, (float *)y, ws.status, s);
   }
-  moe_status st = launch_gate_up_simt(cc, rows, a, offsets, wg, wu, c.intermediate_dim, h, s);
+  moe_status st = launch_gate_up_simt(cc, rows, a, row_token, offsets, wg, wu, c.intermediate_dim, h, s);
   if (st != MOE_OK) return st;
   return launch_down_simt(cc, rows, h, offsets, wd, c.intermediate_dim, row_weight, y, s);
 }
@@ -287,8 +288,8 @@ moe_status moe_dispatch(const MoEConfig *cfg, int T, const int32_t *topk_idx, co
   if (st != MOE_OK) return st;
   if ((st = validate_tokens(cfg, T)) != MOE_OK) return st;
   if (!expert_counts || !expert_offsets || !ws) return MOE_ERR_INVALID_ARG;
-  if (T > 0 && (!topk_idx || !topk_w || !ok_ptr(x) || !slot_row || !row_token || !row_weight ||
-                !ok_ptr(x_perm)))
+  if (T > 0 && (!topk_idx || !topk_w || !slot_row || !row_token || !row_weight ||
+                (x_perm && (!ok_ptr(x) || !aligned16(x_perm)))))
     return MOE_ERR_INVALID_ARG;
   if (ws_bytes < moe_dispatch_workspace_size(cfg, T)) return MOE_ERR_WORKSPACE;
   Carve cv(ws);
@@ -319,21 +320,21 @@ static bool ok_matrix(const MoEConfig *cfg, const void *w, const void *scales) {
   return ok_ptr(w) && (cfg->expert_dtype != MOE_NVFP4 || scales != nullptr);
 }
 
-moe_status moe_expert_gate_up(const MoEConfig *cfg, int rows, const void *x_perm,
-                              const int32_t *expert_offsets, const void *w_gate, const void *w_up,
-                              const void *s_gate, const void *s_up, void *h, void *ws,
+moe_status moe_expert_gate_up(const MoEConfig *cfg, int rows, const void *a, int a_rows,
+                              const int32_t *row_token, const int32_t *expert_offsets, const void *w_gate,
+                              const void *w_up, const void *s_gate, const void *s_up, void *h, void *ws,
                               size_t ws_bytes, moe_stream_t stream) {
   moe_status st = validate_cfg(cfg);
   if (st != MOE_OK) return st;
-  if (rows < 0 || !ws) return MOE_ERR_INVALID_ARG;
+  if (rows < 0 || !ws || (row_token && a_rows <= 0)) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < moe_expert_workspace_size(cfg)) return MOE_ERR_WORKSPACE;
   if (rows == 0) return MOE_OK;
-  if (!ok_ptr(x_perm) || !ok_ptr(h)) return MOE_ERR_INVALID_ARG;
+  if (!ok_ptr(a) || !ok_ptr(h)) return MOE_ERR_INVALID_ARG;
   if (!ok_matrix(cfg, w_gate, s_gate) || !ok_matrix(cfg, w_up, s_up)) return MOE_ERR_INVALID_ARG;
   Carve cv(ws);
   ExpertWs ew = carve_expert(cv, *cfg);
-  return run_gate_up(*cfg, rows, x_perm, expert_offsets, w_gate, w_up, s_gate, s_up, h, ew,
-                     (cudaStream_t)stream);
+  return run_gate_up(*cfg, rows, a, row_token ? a_rows : rows, row_token, expert_offsets, w_gate, w_up, s_gate,
+                     s_up, h, ew, (cudaStream_t)stream);
 }
 
 moe_status moe_expert_down(const MoEConfig *cfg, int rows, const void *h,
@@ -370,8 +371,8 @@ moe_status moe_grouped_swiglu(const MoEConfig *cfg, int rows, const void *x_perm
   ExpertWs ew = carve_expert(cv, *cfg);
   void *h = cv.take<char>((size_t)rows * cfg->intermediate_dim * act_size(*cfg));
   int *sched = cv.take<int>(fused_sched_ints(*cfg, rows, true));
-  return run_experts(*cfg, rows, x_perm, expert_offsets, w->w_gate, w->w_up, w->w_down, w->s_gate, w->s_up,
-                     w->s_down, row_weight, h, y_perm, ew, sched, (cudaStream_t)stream);
+  return run_experts(*cfg, rows, x_perm, rows, nullptr, expert_offsets, w->w_gate, w->w_up, w->w_down, w->s_gate,
+                     w->s_up, w->s_down, row_weight, h, y_perm, ew, sched, (cudaStream_t)stream);
 }
 
 moe_status moe_combine(const MoEConfig *cfg, int T, const void *y_perm, const int32_t *slot_row,
@@ -422,13 +423,15 @@ moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeig
   if ((st = launch_dispatch(c, T, idx, f.topk_w, x, counts, f.offsets, f.slot_row, f.row_token,
                             f.row_weight, f.x_perm, f.chunk_cnt, s)) != MOE_OK)
     return st;
-  if ((st = run_experts(c, rows, f.x_perm, f.offsets, w->w_gate, w->w_up, w->w_down, w->s_gate, w->s_up,
-                        w->s_down, f.row_weight, f.h, f.y_perm, f.ex, f.sched, s)) != MOE_OK)
+  // x_perm from the dispatch gather: the in-GEMM gather (TMA gather4, 512 bytes
+  // per copy) cannot keep the tensor cores fed, a dense tile load can
+  if ((st = run_experts(c, rows, f.x_perm, rows, nullptr, f.offsets, w->w_gate, w->w_up, w->w_down, w->s_gate,
+                        w->s_up, w->s_down, f.row_weight, f.h, f.y_perm, f.ex, f.sched, s)) != MOE_OK)
     return st;
   if (c.shared_intermediate_dim) {
     const MoEConfig sc = shared_cfg(c);
-    if ((st = run_experts(sc, T, x, nullptr, w->sh_gate, w->sh_up, w->sh_down, nullptr, nullptr, nullptr, nullptr,
-                          f.h, f.sh_y, f.ex, f.sched, s)) != MOE_OK)
+    if ((st = run_experts(sc, T, x, T, nullptr, nullptr, w->sh_gate, w->sh_up, w->sh_down, nullptr, nullptr,
+                          nullptr, nullptr, f.h, f.sh_y, f.ex, f.sched, s)) != MOE_OK)
       return st;
   }
   return launch_combine(c, T, f.y_perm, f.slot_row, f.sh_y, out, s);

@@ -201,6 +201,7 @@ moe_status launch_dispatch(const MoEConfig &c, int T, const int32_t *topk_idx, c
   maps_kernel<<<nch, kThreads, maps_smem, s>>>(T, E, k, c.expert_capacity, topk_idx, topk_w, chunk_cnt,
                                                expert_offsets, slot_row, row_token, row_weight);
   MOE_LAUNCH_CHECK();
+  if (!x_perm) return MOE_OK;  // maps only: the GEMM gathers the rows itself
   int dev = 0, sms = 148;
   MOE_CUDA_TRY(cudaGetDevice(&dev));
   MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));

@@ -46,6 +46,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
+#include "tma_host.h"
 
 namespace moe {
 namespace {
@@ -83,7 +84,9 @@ struct Smem {
 };
 
 struct Params {
-  int rows;                  // rows of A and of the output
+  int rows;                  // rows of the output (and of A unless gathered)
+  const int32_t *row_token;  // gathered A: row r of A is src[row_token[r]]; null: A is dense
+  int src_rows;              // rows of the gather source
   int K;                     // reduction length
   int N;                     // output columns (F for gate/up, D for down)
   int E;                     // groups
@@ -244,7 +247,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ================================================= TMA producer (both CTAs)
-    if (lane == 0) {
+    // Dense A: lane 0 issues everything.  Gathered A: every lane issues the
+    // gather of its 4 rows of the 128-row tile; lane 0 waits for the stage,
+    // expects the bytes and loads B.
+    const bool gather = p.row_token != nullptr;
+    if (gather || lane == 0) {
       uint32_t last_parity[C::STAGES];
       bool used[C::STAGES];
 #pragma unroll
@@ -256,34 +263,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int t = unit; t < total_tiles && ok; t += n_units) {
         const Tile tl = decode_tile(p, sm, t, C::TILE_M);
+        int tok[4] = {0, 0, 0, 0};
+        if (gather) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = tl.m0 + (int)rank * BM + lane * 4 + i;
+            tok[i] = r < tl.end ? p.row_token[r] : p.src_rows;  // out of range: zero fill
+          }
+        }
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1u;
-          if (!wait_bar<PAIR>(&sm.empty[s], ph ^ 1u, sm, p.status, rank)) { ok = false; break; }
+          bool got = true;
+          if (lane == 0) got = wait_bar<PAIR>(&sm.empty[s], ph ^ 1u, sm, p.status, rank);
+          if (gather) {
+            got = __shfl_sync(0xffffffffu, got, 0);
+            __syncwarp();
+          }
+          if (!got) { ok = false; break; }
           const int k0 = kb * BK;
           uint8_t *a = stage_a + s * A_BYTES;
           uint8_t *b = stage_b + s * C::B_BYTES;
           if (PAIR) {
             const uint32_t bar = ptx::map_to_rank(&sm.full[s], 0);   // the leader's barrier
-            if (leader) ptx::mbar_arrive_expect_tx(&sm.full[s], C::TX_BYTES);
-            ptx::tma_load_2d_pair(a, &tmA, bar, k0, tl.m0 + (int)rank * BM);
-            if (GATED) {
-              ptx::tma_load_3d_pair(b, rank == 0 ? &tmB0 : &tmB1, bar, k0, tl.n_blk * (BN / 2), tl.e);
-            } else {
-              ptx::tma_load_3d_pair(b, &tmB0, bar, k0, tl.n_blk * BN + (int)rank * (BN / 2), tl.e);
+            if (lane == 0) {
+              if (leader) ptx::mbar_arrive_expect_tx(&sm.full[s], C::TX_BYTES);
+              if (!gather) ptx::tma_load_2d_pair(a, &tmA, bar, k0, tl.m0 + (int)rank * BM);
+              if (GATED) {
+                ptx::tma_load_3d_pair(b, rank == 0 ? &tmB0 : &tmB1, bar, k0, tl.n_blk * (BN / 2), tl.e);
+              } else {
+                ptx::tma_load_3d_pair(b, &tmB0, bar, k0, tl.n_blk * BN + (int)rank * (BN / 2), tl.e);
+              }
             }
+            if (gather) ptx::tma_gather4_pair(a + lane * 512, &tmA, bar, k0, tok[0], tok[1], tok[2], tok[3]);
           } else {
-            ptx::mbar_arrive_expect_tx(&sm.full[s], C::TX_BYTES);
-            ptx::tma_load_2d(a, &tmA, &sm.full[s], k0, tl.m0);
-            if (GATED) {
-              const int n0 = tl.n_blk * (BN / 2);
-              ptx::tma_load_3d(b, &tmB0, &sm.full[s], k0, n0, tl.e);
-              ptx::tma_load_3d(b + C::B_BYTES / 2, &tmB1, &sm.full[s], k0, n0, tl.e);
-            } else {
-              const int n0 = tl.n_blk * BN;
-              ptx::tma_load_3d(b, &tmB0, &sm.full[s], k0, n0, tl.e);
-              ptx::tma_load_3d(b + C::B_BYTES / 2, &tmB0, &sm.full[s], k0, n0 + BN / 2, tl.e);
+            if (lane == 0) {
+              ptx::mbar_arrive_expect_tx(&sm.full[s], C::TX_BYTES);
+              if (!gather) ptx::tma_load_2d(a, &tmA, &sm.full[s], k0, tl.m0);
+              if (GATED) {
+                const int n0 = tl.n_blk * (BN / 2);
+                ptx::tma_load_3d(b, &tmB0, &sm.full[s], k0, n0, tl.e);
+                ptx::tma_load_3d(b + C::B_BYTES / 2, &tmB1, &sm.full[s], k0, n0, tl.e);
+              } else {
+                const int n0 = tl.n_blk * BN;
+                ptx::tma_load_3d(b, &tmB0, &sm.full[s], k0, n0, tl.e);
+                ptx::tma_load_3d(b + C::B_BYTES / 2, &tmB0, &sm.full[s], k0, n0 + BN / 2, tl.e);
+              }
             }
+            if (gather) ptx::tma_gather4(a + lane * 512, &tmA, &sm.full[s], k0, tok[0], tok[1], tok[2], tok[3]);
           }
           used[s] = true;
           last_parity[s] = ph;
@@ -292,11 +319,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // drain: every issued copy has landed before shared memory is released.
       // The leader's barriers count both CTAs' bytes; a peer that stopped early
       // gives its last copies time to land.
-      if (leader) {
-        for (int s = 0; s < C::STAGES; ++s)
-          if (used[s]) drain_bar(&sm.full[s], last_parity[s], p.status);
-      } else if (!ok) {
-        spin_ns(1000000);
+      if (lane == 0) {
+        if (leader) {
+          for (int s = 0; s < C::STAGES; ++s)
+            if (used[s]) drain_bar(&sm.full[s], last_parity[s], p.status);
+        } else if (!ok) {
+          spin_ns(1000000);
+        }
       }
     }
   } else if (warp == 1) {
@@ -803,34 +832,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ host
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-    void *f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      f = nullptr;
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  }();
-  return fn;
-}
-
-// bf16 tensor of rank 2 ([d1][d0]) or 3 ([d2][d1][d0]), d0 contiguous, box
-// {64, 128(, 1)}, 128-byte swizzle, zero fill outside the tensor.
-bool make_map(CUtensorMap *m, const void *ptr, int rank, uint64_t d0, uint64_t d1, uint64_t d2) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
-  cuuint32_t box[3] = {BK, 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(ptr), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 struct DevInfo {
   int sms = 0;
   int pair_clusters = 0;  // co-resident CTA pairs of the pair kernels
@@ -845,10 +846,10 @@ template <bool GATED, bool PAIR>
 moe_status launch_tc(const Params &p, const void *a, const void *b0, const void *b1, int Nw, cudaStream_t s) {
   // A: [rows, K]; B: [E, Nw, K] (rank 3 even for one group)
   CUtensorMap ta, tb0, tb1;
-  if (!make_map(&ta, a, 2, (uint64_t)p.K, (uint64_t)p.rows, 1)) return MOE_ERR_CUDA;
-  if (!make_map(&tb0, b0, 3, (uint64_t)p.K, (uint64_t)Nw, (uint64_t)p.E)) return MOE_ERR_CUDA;
+  if (!tma_map_bf16(&ta, a, 2, (uint64_t)p.K, (uint64_t)(p.row_token ? p.src_rows : p.rows), 1, p.row_token ? 1 : 128)) return MOE_ERR_CUDA;
+  if (!tma_map_bf16(&tb0, b0, 3, (uint64_t)p.K, (uint64_t)Nw, (uint64_t)p.E)) return MOE_ERR_CUDA;
   if (GATED) {
-    if (!make_map(&tb1, b1, 3, (uint64_t)p.K, (uint64_t)Nw, (uint64_t)p.E)) return MOE_ERR_CUDA;
+    if (!tma_map_bf16(&tb1, b1, 3, (uint64_t)p.K, (uint64_t)Nw, (uint64_t)p.E)) return MOE_ERR_CUDA;
   } else {
     tb1 = tb0;
   }
@@ -908,11 +909,11 @@ moe_status launch_fused(const MoEConfig &c, int rows, const void *x_perm, const 
   p.status = status;
   p.sched = sched;
   CUtensorMap tx, twg, twu, th, twd;
-  if (!make_map(&tx, x_perm, 2, (uint64_t)p.D, (uint64_t)rows, 1)) return MOE_ERR_CUDA;
-  if (!make_map(&twg, w_gate, 3, (uint64_t)p.D, (uint64_t)p.F, (uint64_t)p.E)) return MOE_ERR_CUDA;
-  if (!make_map(&twu, w_up, 3, (uint64_t)p.D, (uint64_t)p.F, (uint64_t)p.E)) return MOE_ERR_CUDA;
-  if (!make_map(&th, h, 2, (uint64_t)p.F, (uint64_t)rows, 1)) return MOE_ERR_CUDA;
-  if (!make_map(&twd, w_down, 3, (uint64_t)p.F, (uint64_t)p.D, (uint64_t)p.E)) return MOE_ERR_CUDA;
+  if (!tma_map_bf16(&tx, x_perm, 2, (uint64_t)p.D, (uint64_t)rows, 1)) return MOE_ERR_CUDA;
+  if (!tma_map_bf16(&twg, w_gate, 3, (uint64_t)p.D, (uint64_t)p.F, (uint64_t)p.E)) return MOE_ERR_CUDA;
+  if (!tma_map_bf16(&twu, w_up, 3, (uint64_t)p.D, (uint64_t)p.F, (uint64_t)p.E)) return MOE_ERR_CUDA;
+  if (!tma_map_bf16(&th, h, 2, (uint64_t)p.F, (uint64_t)rows, 1)) return MOE_ERR_CUDA;
+  if (!tma_map_bf16(&twd, w_down, 3, (uint64_t)p.F, (uint64_t)p.D, (uint64_t)p.E)) return MOE_ERR_CUDA;
   const long mt_ub = (long)(rows + BM - 1) / BM + p.E;
   MOE_CUDA_TRY(cudaMemsetAsync(sched, 0, sizeof(int) * (size_t)(1 + mt_ub), s));
   int dev = 0, sms = 148;
@@ -945,15 +946,17 @@ bool use_pair(int rows, int E, bool gated) {
 
 bool tc_shapes_ok(const MoEConfig &c, int F) {
   return c.act_dtype == MOE_BF16 && c.hidden_dim % BN == 0 && F % 128 == 0 && c.hidden_dim % BK == 0 &&
-         encode_fn() != nullptr;
+         tma_encode_fn() != nullptr;
 }
 
-moe_status launch_gate_up_tc(const MoEConfig &c, int rows, const void *a, const int32_t *offsets,
-                             const void *w_gate, const void *w_up, int F, void *h, int *status,
-                             cudaStream_t s) {
+moe_status launch_gate_up_tc(const MoEConfig &c, int rows, const void *a, int a_rows, const int32_t *row_token,
+                             const int32_t *offsets, const void *w_gate, const void *w_up, int F, void *h,
+                             int *status, cudaStream_t s) {
   if (rows == 0) return MOE_OK;
   Params p;
   p.rows = rows;
+  p.row_token = row_token;
+  p.src_rows = a_rows;
   p.K = c.hidden_dim;
   p.N = F;
   p.E = offsets ? c.num_experts : 1;
@@ -974,6 +977,8 @@ moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int
   if (rows == 0) return MOE_OK;
   Params p;
   p.rows = rows;
+  p.row_token = nullptr;
+  p.src_rows = rows;
   p.K = F;
   p.N = c.hidden_dim;
   p.E = offsets ? c.num_experts : 1;

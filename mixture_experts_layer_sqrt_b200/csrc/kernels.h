@@ -26,7 +26,8 @@ moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void 
                            int *status, cudaStream_t s);
 
 // dispatch.cu ------------------------------------------------------------
-// chunk_cnt: [num_chunks(T), E] int32 scratch.
+// chunk_cnt: [num_chunks(T), E] int32 scratch.  x_perm may be null: the row
+// maps are built but no rows are copied.
 moe_status launch_dispatch(const MoEConfig &c, int T, const int32_t *topk_idx, const float *topk_w,
                            const void *x, int32_t *expert_counts, int32_t *expert_offsets,
                            int32_t *slot_row, int32_t *row_token, float *row_weight, void *x_perm,
@@ -35,7 +36,7 @@ moe_status launch_dispatch(const MoEConfig &c, int T, const int32_t *topk_idx, c
 // gemm_simt.cu -----------------------------------------------------------
 // Grouped GEMMs on CUDA cores (fp32 FMA), any shape.  act: F32 or BF16 for
 // activations and weights alike.
-moe_status launch_gate_up_simt(const MoEConfig &c, int rows, const void *a,
+moe_status launch_gate_up_simt(const MoEConfig &c, int rows, const void *a, const int32_t *row_token,
                                const int32_t *offsets, const void *w_gate, const void *w_up,
                                int F, void *h, cudaStream_t s);
 moe_status launch_down_simt(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
@@ -46,9 +47,11 @@ moe_status launch_down_simt(const MoEConfig &c, int rows, const void *h, const i
 // Grouped GEMMs on tcgen05 tensor cores (bf16 in, fp32 accumulate).  Usable
 // when tc_shapes_ok(): bf16 activations, D % 256 == 0, F % 128 == 0.
 bool tc_shapes_ok(const MoEConfig &c, int F);
-moe_status launch_gate_up_tc(const MoEConfig &c, int rows, const void *a, const int32_t *offsets,
-                             const void *w_gate, const void *w_up, int F, void *h, int *status,
-                             cudaStream_t s);
+// A is dense [rows, D] when row_token is null; otherwise row r of A is
+// a[row_token[r]] of a [a_rows, D] source (gathered by the GEMM's loads).
+moe_status launch_gate_up_tc(const MoEConfig &c, int rows, const void *a, int a_rows, const int32_t *row_token,
+                             const int32_t *offsets, const void *w_gate, const void *w_up, int F, void *h,
+                             int *status, cudaStream_t s);
 moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
                           const void *w_down, int F, const float *row_weight, float *y, int *status,
                           cudaStream_t s);

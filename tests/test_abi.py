@@ -115,16 +115,25 @@ def test_workspace_too_small_rejected(B):
     st = B.lib.moe_forward(ctypes.byref(c), 64, 16, ctypes.byref(w), None, 16, None, None, 16, need - 1, None)
     assert st == B.MOE_ERR_WORKSPACE
     e = B.lib.moe_expert_workspace_size(ctypes.byref(c))
-    st = B.lib.moe_expert_gate_up(ctypes.byref(c), 8, 16, None, 16, 16, None, None, 16, 16, e - 1, None)
+    st = B.lib.moe_expert_gate_up(ctypes.byref(c), 8, 16, 8, None, None, 16, 16, None, None, 16, 16, e - 1,
+                                  None)
     assert st == B.MOE_ERR_WORKSPACE
 
 
 def test_nvfp4_requires_scales(B):
     c = _cfg(B, expert="nvfp4")
     e = B.lib.moe_expert_workspace_size(ctypes.byref(c))
-    st = B.lib.moe_expert_gate_up(ctypes.byref(c), 8, 16, None, 16, 16, None, 16, 16, 16, e, None)
+    st = B.lib.moe_expert_gate_up(ctypes.byref(c), 8, 16, 8, None, None, 16, 16, None, 16, 16, 16, e, None)
     assert st == B.MOE_ERR_INVALID_ARG
     st = B.lib.moe_expert_down(ctypes.byref(c), 8, 16, None, 16, None, None, 16, 16, e, None)
+    assert st == B.MOE_ERR_INVALID_ARG
+
+
+def test_gather_needs_source_rows(B):
+    # a row map without the row count of the source matrix cannot be bounded
+    c = _cfg(B, act="bf16")
+    e = B.lib.moe_expert_workspace_size(ctypes.byref(c))
+    st = B.lib.moe_expert_gate_up(ctypes.byref(c), 8, 16, 0, 16, None, 16, 16, None, None, 16, 16, e, None)
     assert st == B.MOE_ERR_INVALID_ARG
 
 

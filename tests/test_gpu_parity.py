@@ -65,6 +65,9 @@ def _stages(B, c: Case):
     d = B.dispatch(c.cfg, c.x, idx, w)
     s = {k: c.wt.get(k) for k in ("s_gate", "s_up", "s_down")}
     h = B.expert_gate_up(c.cfg, d["x_perm"], d["expert_offsets"], c.wt["w_gate"], c.wt["w_up"], s["s_gate"], s["s_up"])
+    # the same projection with the rows gathered from x by the GEMM's own loads
+    hg = B.expert_gate_up(c.cfg, c.x, d["expert_offsets"], c.wt["w_gate"], c.wt["w_up"], s["s_gate"], s["s_up"],
+                          row_token=d["row_token"])
     y = B.expert_down(c.cfg, h, d["expert_offsets"], c.wt["w_down"], s["s_down"], d["row_weight"])
     sh = None
     if p.Fs:
@@ -73,7 +76,7 @@ def _stages(B, c: Case):
         sh = B.expert_down(sc, hs, None, c.wt["sh_down"])
     out = B.combine(c.cfg, y, d["slot_row"], p.T, shared_y=sh)
     torch.cuda.synchronize()
-    return dict(idx=idx, w=w, h=h, y=y, sh=sh, out=out, **d)
+    return dict(idx=idx, w=w, h=h, hg=hg, y=y, sh=sh, out=out, **d)
 
 
 @pytest.mark.parametrize("name", SMALL_NAMES)
@@ -115,6 +118,8 @@ def test_stages_small(B, W, name):
         # a7 down + weight epilogue, fed with the GPU's own h
         y_ref[r0:r1] = w_g[d["row_token"][r0:r1], d["row_slot"][r0:r1], None] * (h_g[r0:r1] @ wd.T)
     H.assert_close_h(p, h_g, h_ref)
+    # gathered A rows are the same tile bytes as x_perm's: the same bits
+    assert torch.equal(g["hg"][:R], g["h"][:R])
     y_g = H.to_np(g["y"][:R])
     H.assert_close_f32(y_g, y_ref, "y_perm")
 
@@ -352,14 +357,18 @@ def test_fused_expert_kernel_matches(B, W, name, monkeypatch):
     # their m-block of h) gives the two-launch result bit for bit
     p = H.small(name)
     c = Case(B, W, p)
-    ws = B.workspace(B.workspace_size(c.cfg, p.T))
-    ref = B.forward(c.cfg, c.x, c.w, ws, c.mask)
+    idx, w = B.route_topk(c.cfg, c.x, c.w, c.mask)
+    d = B.dispatch(c.cfg, c.x, idx, w)
+    rows = p.T * p.k
+    ws = B.workspace(B.grouped_swiglu_workspace_size(c.cfg, rows))
+    ref = B.grouped_swiglu(c.cfg, d["x_perm"], d["expert_offsets"], c.w, d["row_weight"], ws=ws)
     torch.cuda.synchronize()
     monkeypatch.setenv("MOE_EXPERTS_FUSED", "1")
-    got = B.forward(c.cfg, c.x, c.w, ws, c.mask)
+    got = B.grouped_swiglu(c.cfg, d["x_perm"], d["expert_offsets"], c.w, d["row_weight"], ws=ws)
     torch.cuda.synchronize()
     B.check_device_status(ws)
-    assert torch.equal(got, ref)
+    R = int(d["expert_offsets"][-1])
+    assert torch.equal(got[:R], ref[:R])
 
 
 def test_host_batches_overlapped_copies(B, W):
