@@ -68,16 +68,24 @@ moe_status validate_tokens(const MoEConfig *c, int T) {
 }
 
 // ---- expert-stage workspace: [status][bf16 expansion of NVFP4 weights]
+// NVFP4 projections whose reduction length fits the tensor-core FP4 path read
+// the packed weights directly; the others are expanded to bf16 first (gate and
+// up together, then down into the same space).
 struct ExpertWs {
   int *status;
   __nv_bfloat16 *wexp;
 };
+inline bool gate_up_direct(const MoEConfig &c) { return fp4_direct_ok(c, c.hidden_dim); }
+inline bool down_direct(const MoEConfig &c) { return fp4_direct_ok(c, c.intermediate_dim); }
 ExpertWs carve_expert(Carve &cv, const MoEConfig &c) {
   ExpertWs w;
   w.status = cv.take<int>(kStatusBytes / sizeof(int));
   w.wexp = nullptr;
-  if (c.expert_dtype == MOE_NVFP4)
-    w.wexp = cv.take<__nv_bfloat16>(3ull * c.num_experts * c.intermediate_dim * c.hidden_dim);
+  if (c.expert_dtype == MOE_NVFP4) {
+    const size_t n = (size_t)c.num_experts * c.intermediate_dim * c.hidden_dim;
+    const size_t need = gate_up_direct(c) ? (down_direct(c) ? 0 : n) : 2 * n;
+    if (need) w.wexp = cv.take<__nv_bfloat16>(need);
+  }
   return w;
 }
 
@@ -86,6 +94,8 @@ moe_status run_gate_up(const MoEConfig &c, int rows, const void *a, int a_rows, 
                        const int32_t *offsets, const void *wg, const void *wu, const void *sg, const void *su,
                        void *h, const ExpertWs &ws, cudaStream_t s) {
   MoEConfig cc = c;
+  if (gate_up_direct(c))
+    return launch_gate_up_fp4(c, rows, a, a_rows, row_token, offsets, wg, wu, sg, su, h, ws.status, s);
   if (c.expert_dtype == MOE_NVFP4) {
     const long n = (long)c.num_experts * c.intermediate_dim * c.hidden_dim;
     moe_status st = launch_dequant_nvfp4(wg, sg, n, ws.wexp, s);
@@ -105,6 +115,8 @@ moe_status run_down(const MoEConfig &c, int rows, const void *h, const int32_t *
                     const void *wd, const void *sd, const float *row_weight, void *y,
                     const ExpertWs &ws, cudaStream_t s) {
   MoEConfig cc = c;
+  if (down_direct(c))
+    return launch_down_fp4(c, rows, h, offsets, wd, sd, row_weight, (float *)y, ws.status, s);
   if (c.expert_dtype == MOE_NVFP4) {
     const long n = (long)c.num_experts * c.intermediate_dim * c.hidden_dim;
     moe_status st = launch_dequant_nvfp4(wd, sd, n, ws.wexp, s);
@@ -124,36 +136,20 @@ bool fused_requested() {
   return e && e[0] == '1';
 }
 
-// Both expert projections: x_perm -> h -> y.  On the tensor-core path one
-// fused persistent launch; otherwise the CUDA-core kernels one after the other.
+// Both expert projections: x_perm -> h -> y.  NVFP4 experts: the two
+// projections one after the other, each straight from the packed weights or
+// expanded first.  bf16 on the tensor-core path: two launches, or with
+// MOE_EXPERTS_FUSED=1 one persistent launch.  Otherwise the CUDA-core kernels.
 moe_status run_experts(const MoEConfig &c, int rows, const void *a, int a_rows, const int32_t *row_token,
                        const int32_t *offsets, const void *wg, const void *wu, const void *wd, const void *sg,
                        const void *su, const void *sd, const float *row_weight, void *h, void *y,
                        const ExpertWs &ws, int *sched, cudaStream_t s) {
-  MoEConfig cc = c;
-  if (c.expert_dtype == MOE_NVFP4) {
-    const long n = (long)c.num_experts * c.intermediate_dim * c.hidden_dim;
-    moe_status st;
-    if ((st = launch_dequant_nvfp4(wg, sg, n, ws.wexp, s)) != MOE_OK) return st;
-    if ((st = launch_dequant_nvfp4(wu, su, n, ws.wexp + n, s)) != MOE_OK) return st;
-    if ((st = launch_dequant_nvfp4(wd, sd, n, ws.wexp + 2 * n, s)) != MOE_OK) return st;
-    wg = ws.wexp;
-    wu = ws.wexp + n;
-    wd = ws.wexp + 2 * n;
-    cc.expert_dtype = MOE_BF16;
+  moe_status st;
+  if (c.expert_dtype == MOE_NVFP4 || !tc_shapes_ok(c, c.intermediate_dim) || !fused_requested() || row_token) {
+    if ((st = run_gate_up(c, rows, a, a_rows, row_token, offsets, wg, wu, sg, su, h, ws, s)) != MOE_OK) return st;
+    return run_down(c, rows, h, offsets, wd, sd, row_weight, y, ws, s);
   }
-  if (tc_shapes_ok(cc, c.intermediate_dim)) {
-    if (fused_requested() && !row_token)
-      return launch_experts_fused_tc(cc, rows, a, offsets, wg, wu, wd, row_weight, h, (float *)y, ws.status,
-                                     sched, s);
-    moe_status st = launch_gate_up_tc(cc, rows, a, a_rows, row_token, offsets, wg, wu, c.intermediate_dim, h,
-                                      ws.status, s);
-    if (st != MOE_OK) return st;
-    return launch_down_tc(cc, rows, h, offsets, wd, c.intermediate_dim, row_weight, (float *)y, ws.status, s);
-  }
-  moe_status st = launch_gate_up_simt(cc, rows, a, row_token, offsets, wg, wu, c.intermediate_dim, h, s);
-  if (st != MOE_OK) return st;
-  return launch_down_simt(cc, rows, h, offsets, wd, c.intermediate_dim, row_weight, y, s);
+  return launch_experts_fused_tc(c, rows, a, offsets, wg, wu, wd, row_weight, h, (float *)y, ws.status, sched, s);
 }
 
 // The shared expert viewed as a one-expert layer of width F_s in the act dtype.
@@ -315,9 +311,10 @@ size_t moe_grouped_swiglu_workspace_size(const MoEConfig *cfg, int rows) {
   return align_up(cv.off, 256);
 }
 
-// An expert weight matrix: 16-byte aligned data, plus its scales when NVFP4.
+// An expert weight matrix: 16-byte aligned data, plus its scales (also
+// 16-byte aligned: TMA reads them) when NVFP4.
 static bool ok_matrix(const MoEConfig *cfg, const void *w, const void *scales) {
-  return ok_ptr(w) && (cfg->expert_dtype != MOE_NVFP4 || scales != nullptr);
+  return ok_ptr(w) && (cfg->expert_dtype != MOE_NVFP4 || ok_ptr(scales));
 }
 
 moe_status moe_expert_gate_up(const MoEConfig *cfg, int rows, const void *a, int a_rows,

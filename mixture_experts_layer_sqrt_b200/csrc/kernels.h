@@ -56,6 +56,18 @@ moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int
                           const void *w_down, int F, const float *row_weight, float *y, int *status,
                           cudaStream_t s);
 
+// gemm_fp4.cu ------------------------------------------------------------
+// The same projections with NVFP4 weights read in their packed form (codes
+// and scales expanded to bf16 on chip).  Usable when fp4_direct_ok() for the
+// projection's reduction length K (D for gate/up, F for down).
+bool fp4_direct_ok(const MoEConfig &c, int K);
+moe_status launch_gate_up_fp4(const MoEConfig &c, int rows, const void *a, int a_rows, const int32_t *row_token,
+                              const int32_t *offsets, const void *w_gate, const void *w_up, const void *s_gate,
+                              const void *s_up, void *h, int *status, cudaStream_t s);
+moe_status launch_down_fp4(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
+                           const void *w_down, const void *s_down, const float *row_weight, float *y,
+                           int *status, cudaStream_t s);
+
 // Both projections in one persistent launch (gate/up tiles, then down tiles
 // that wait for their m-block of h).  sched: fused_sched_ints() ints of
 // scratch, zeroed by the launcher.

@@ -39,4 +39,20 @@ inline bool tma_map_bf16(CUtensorMap *m, const void *ptr, int rank, uint64_t d0,
   return r == CUDA_SUCCESS;
 }
 
+// uint8 tensor [d2][d1][d0] (d0 contiguous, in bytes); box {box0, box_rows, 1};
+// no swizzle (rows land box0 bytes apart); zero fill outside the tensor.
+inline bool tma_map_u8(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
+                       uint32_t box_rows) {
+  auto fn = tma_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0, d0 * d1};
+  cuuint32_t box[3] = {box0, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace moe

@@ -27,7 +27,8 @@ def small(name: str) -> synth.MoEProblem:
     if name == "mixtral_bf16_pair":
         return synth.PROBLEMS["mixtral_bf16"].with_(name=name, T=4200, D=512, F=384, E=4)
     if name == "sqrt_fp4_pair":
-        return synth.PROBLEMS["sqrt_fp4"].with_(name=name, T=2100, D=512, F=384, E=12, k=3, Fs=256)
+        # F % 256 == 0: both projections read the packed FP4 weights directly
+        return synth.PROBLEMS["sqrt_fp4"].with_(name=name, T=2100, D=512, F=512, E=12, k=3, Fs=256)
     p = synth.PROBLEMS[name]
     if name == "tiny_f32":
         return p

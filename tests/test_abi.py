@@ -127,6 +127,9 @@ def test_nvfp4_requires_scales(B):
     assert st == B.MOE_ERR_INVALID_ARG
     st = B.lib.moe_expert_down(ctypes.byref(c), 8, 16, None, 16, None, None, 16, 16, e, None)
     assert st == B.MOE_ERR_INVALID_ARG
+    # scales are read by TMA: 16-byte aligned like the codes
+    st = B.lib.moe_expert_down(ctypes.byref(c), 8, 16, None, 16, 24, None, 16, 16, e, None)
+    assert st == B.MOE_ERR_INVALID_ARG
 
 
 def test_gather_needs_source_rows(B):

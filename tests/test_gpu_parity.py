@@ -351,7 +351,7 @@ def test_binding_rejects_mismatched_out(B, W):
         B.forward(c.cfg, c.x, c.w, ws, out=torch.empty((p.T - 1, p.D), dtype=torch.float32, device="cuda"))
 
 
-@pytest.mark.parametrize("name", ["mixtral_bf16", "finegrained_bf16", "sqrt_fp4"])
+@pytest.mark.parametrize("name", ["mixtral_bf16", "finegrained_bf16", "capacity_bf16"])
 def test_fused_expert_kernel_matches(B, W, name, monkeypatch):
     # the single persistent launch (gate/up tiles, then down tiles waiting on
     # their m-block of h) gives the two-launch result bit for bit
@@ -369,6 +369,36 @@ def test_fused_expert_kernel_matches(B, W, name, monkeypatch):
     B.check_device_status(ws)
     R = int(d["expert_offsets"][-1])
     assert torch.equal(got[:R], ref[:R])
+
+
+@pytest.mark.parametrize("name", ["sqrt_fp4_pair", "sqrt_fp4"])
+def test_fp4_direct_matches_expanded_weights(B, W, name, monkeypatch):
+    # NVFP4 codes converted to bf16 in shared memory give the MMA the same
+    # operand bits as weights expanded beforehand (every e2m1 * e4m3 product is
+    # exact in bf16): bit for bit the bf16 GEMM (same 128-row tiles) on the
+    # expanded weights
+    p = H.small(name)
+    c = Case(B, W, p)
+    idx, w = B.route_topk(c.cfg, c.x, c.w, c.mask)
+    d = B.dispatch(c.cfg, c.x, idx, w)
+    wt = c.wt
+    h4 = B.expert_gate_up(c.cfg, d["x_perm"], d["expert_offsets"], wt["w_gate"], wt["w_up"], wt["s_gate"],
+                          wt["s_up"])
+    y4 = B.expert_down(c.cfg, h4, d["expert_offsets"], wt["w_down"], wt["s_down"], d["row_weight"])
+    torch.cuda.synchronize()
+    ex = {}
+    for k in ("w_gate", "w_up", "w_down"):
+        v = O.dequant_nvfp4(c.a[k], c.a[k + "_scale"])
+        assert np.array_equal(v.astype(np.float32).astype(np.float64), v)  # exact in fp32 (and bf16)
+        ex[k] = W.to_torch(synth.f32_to_bf16_bits(v.astype(np.float32)))
+    cfg16 = W.config_of(p.with_(wdtype="bf16"))
+    monkeypatch.setenv("MOE_TC_TILE", "128")
+    h16 = B.expert_gate_up(cfg16, d["x_perm"], d["expert_offsets"], ex["w_gate"], ex["w_up"])
+    y16 = B.expert_down(cfg16, h16, d["expert_offsets"], ex["w_down"], None, d["row_weight"])
+    torch.cuda.synchronize()
+    R = int(d["expert_offsets"][-1])
+    assert torch.equal(h4[:R], h16[:R])
+    assert torch.equal(y4[:R], y16[:R])
 
 
 def test_host_batches_overlapped_copies(B, W):
