@@ -69,7 +69,7 @@ def load_peaks():
 
 def gemm_sources_sha() -> str:
     h = hashlib.sha256()
-    for n in ("gemm_tc.cu", "gemm_simt.cu", "tc_ptx.cuh", "api.cu"):
+    for n in ("gemm_tc.cu", "tc_ptx.cuh", "tma_host.h", "common.cuh"):
         p = os.path.join(ROOT, "mixture_experts_layer_sqrt_b200", "csrc", n)
         if os.path.exists(p):
             h.update(open(p, "rb").read())

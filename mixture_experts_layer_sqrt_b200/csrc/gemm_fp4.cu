@@ -25,12 +25,12 @@
 // Roles (448 threads per CTA):
 //   warp 0       TMA producer: A rows (128 x 64 bf16), packed codes (256 B
 //                rows x 32 bytes) and scales (256 x 16 bytes: the 4-k-block
-//                group) per k-block into a 5-stage ring.
+//                group) per k-block into a 4-stage ring.
 //   warp 1       TMEM owner; one thread issues the MMAs (A from the TMA ring,
 //                B from the converted ring) and commits stages back.
 //   warps 2-5    epilogue: TMEM -> registers -> SwiGLU or routing weight ->
 //                global stores; two 256-column accumulators overlap tiles.
-//   warps 6-13   converters: codes + scales -> swizzled bf16 B tile (2-stage
+//   warps 6-13   converters: codes + scales -> swizzled bf16 B tile (3-stage
 //                ring), one arrival per warp.
 //
 // Tiles never straddle two experts; the tile list (expert-major, n-block,
@@ -55,8 +55,8 @@ constexpr int A_BYTES = TILE_M * BK * 2;        // 16 KB
 constexpr int B_BYTES = FN * BK * 2;            // 32 KB
 constexpr int RAW_BYTES = FN * BK / 2;          // 8 KB of e2m1 codes
 constexpr int SCL_BYTES = FN * 16;              // 4 KB of e4m3 scales (4 k-blocks)
-constexpr int STAGES = 5;
-constexpr int B_STAGES = 2;
+constexpr int STAGES = 4;
+constexpr int B_STAGES = 3;
 constexpr int kConv = 8;                        // converter warps
 constexpr int kThreads = 192 + 32 * kConv;
 constexpr uint32_t TMEM_COLS = 512;             // 2 accumulators x FN
