@@ -163,59 +163,27 @@ def run_ours(args, p, rank, world, local_rank):
     x = WL.to_torch(arrays["x"], dev)
     mask = WL.to_torch(arrays.get("image_mask"), dev)
     T, k, D = p.T, p.k, p.D
-    act = torch.float32 if p.act == "f32" else torch.bfloat16
-    # preallocated stage buffers
-    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
-    tw = torch.empty((T, k), dtype=torch.float32, device=dev)
-    disp = dict(expert_counts=torch.empty(p.E, dtype=torch.int32, device=dev),
-                expert_offsets=torch.empty(p.E + 1, dtype=torch.int32, device=dev),
-                slot_row=torch.empty((T, k), dtype=torch.int32, device=dev),
-                row_token=torch.empty(T * k, dtype=torch.int32, device=dev),
-                row_weight=torch.empty(T * k, dtype=torch.float32, device=dev),
-                x_perm=torch.empty((T * k, D), dtype=act, device=dev))
-    h = torch.empty((max(T * k * p.F, T * p.Fs),), dtype=act, device=dev)
-    y = torch.empty((T * k, D), dtype=torch.float32, device=dev)
-    shy = torch.empty((T, D), dtype=torch.float32, device=dev) if p.Fs else None
     out = torch.empty((T, D), dtype=torch.float32, device=dev)
-    ws_r = B.workspace(B.route_workspace_size(cfg, T), dev)
-    ws_d = B.workspace(B.dispatch_workspace_size(cfg, T), dev)
-    ws_e = B.workspace(B.expert_workspace_size(cfg), dev)
-    scfg = B.make_config(E=1, k=1, D=D, F=max(p.Fs, 1), clamp=p.clamp, act=p.act, expert=p.act) if p.Fs else None
-    ws_s = B.workspace(B.expert_workspace_size(scfg), dev) if p.Fs else None
+    ws_f = B.workspace(B.workspace_size(cfg, T), dev)
     stream = torch.cuda.current_stream(dev)
-    hF = h[:T * k * p.F].view(T * k, p.F)
 
-    def mark(ev, i):
-        if ev is not None:
-            ev[i].record(stream)
-
-    # the kernels moe_forward launches, one stage per call so each can be timed:
-    # events: 0 | route | 1 | dispatch | 2 | gate/up | 3 | down | 4 | shared | 5 | combine | 6
+    # one step = one moe_forward call (the product's own entry point); with
+    # events it records them on the stream at the stage boundaries:
+    # 0 | route | 1 | dispatch | 2 | gate/up | 3 | down | 4 | shared | 5 | combine | 6
     def step(ev=None):
-        mark(ev, 0)
-        B.route_topk(cfg, x, w, mask, idx, tw, ws_r)
-        mark(ev, 1)
-        B.dispatch(cfg, x, idx, tw, disp, ws_d)
-        mark(ev, 2)
-        B.expert_gate_up(cfg, disp["x_perm"], disp["expert_offsets"], wt["w_gate"], wt["w_up"],
-                         wt.get("s_gate"), wt.get("s_up"), hF, ws_e)
-        mark(ev, 3)
-        B.expert_down(cfg, hF, disp["expert_offsets"], wt["w_down"], wt.get("s_down"), disp["row_weight"], y, ws_e)
-        mark(ev, 4)
-        if p.Fs:
-            hs = h[:T * p.Fs].view(T, p.Fs)
-            B.expert_gate_up(scfg, x, None, wt["sh_gate"], wt["sh_up"], None, None, hs, ws_s)
-            B.expert_down(scfg, hs, None, wt["sh_down"], None, None, shy, ws_s)
-        mark(ev, 5)
-        B.combine(cfg, y, disp["slot_row"], T, shy, out)
-        mark(ev, 6)
+        if ev is None:
+            B.forward(cfg, x, w, ws_f, mask, out)
+        else:
+            B.forward_profiled(cfg, x, w, ws_f, ev, mask, out)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    B.check_device_status(ws_e)
-    B.check_device_status(ws_r)
-    rows = int(disp["expert_offsets"][-1].item())
+    B.check_device_status(ws_f)
+    counts = torch.empty(p.E, dtype=torch.int32, device=dev)
+    B.forward(cfg, x, w, ws_f, mask, out, expert_counts_out=counts)
+    cap = cfg.expert_capacity
+    rows = int((counts.clamp(max=cap) if cap else counts).sum().item())
 
     dist = None
     if world > 1:
@@ -227,7 +195,10 @@ def run_ours(args, p, rank, world, local_rank):
     torch.cuda.synchronize()
     n0 = B.launch_count()
     step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    g_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    g_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(B.STAGE_EVENTS)] for _ in range(args.steps)]
+    for e in step_ev + [ev for evs in g_ev for ev in evs]:  # create every CUDA event before timing
+        e.record(stream)
+    torch.cuda.synchronize()
     step_ev[0].record(stream)
     for i in range(args.steps):
         step(g_ev[i])
@@ -242,7 +213,7 @@ def run_ours(args, p, rank, world, local_rank):
     names = ["route", "dispatch", "gate_up", "down", "shared", "combine"]
     stage_ms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in g_ev) / args.steps for i, n in enumerate(names)}
     gemm_ms = stage_ms["gate_up"]
-    B.check_device_status(ws_e)
+    B.check_device_status(ws_f)
     t_max = total_ms
     if dist:
         tt = torch.tensor([total_ms], device=dev)

@@ -73,6 +73,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_combine": (I, [cfgp, I, P, P, P, P, P]),
         "moe_workspace_size": (S, [cfgp, I]),
         "moe_forward": (I, [cfgp, I, P, wp, P, P, P, P, P, S, P]),
+        "moe_forward_profiled": (I, [cfgp, I, P, wp, P, P, P, P, P, S, P, P, I]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -88,7 +89,7 @@ EXPORTS = ("moe_status_string", "moe_version", "moe_expert_capacity", "moe_launc
            "moe_check_device_status", "moe_route_workspace_size", "moe_route_topk", "moe_dispatch_workspace_size",
            "moe_dispatch", "moe_dispatch_noalloc", "moe_grouped_swiglu_workspace_size", "moe_expert_workspace_size",
            "moe_expert_gate_up", "moe_expert_down", "moe_grouped_swiglu", "moe_combine",
-           "moe_workspace_size", "moe_forward")
+           "moe_workspace_size", "moe_forward", "moe_forward_profiled")
 
 
 def status_string(s: int) -> str:
@@ -293,6 +294,41 @@ def forward(cfg: MoEConfig, x: torch.Tensor, w: MoEWeights, ws: torch.Tensor, im
     _check(lib.moe_forward(ctypes.byref(cfg), T, _p(x), ctypes.byref(w), _p(image_mask), _p(out),
                            _p(topk_idx_out), _p(expert_counts_out), _p(ws), ws.numel(), _stream(stream)),
            "moe_forward")
+    return out
+
+
+STAGES = ("route", "dispatch", "gate_up", "down", "shared", "combine")
+STAGE_EVENTS = 7
+
+
+def _event_handles(events):
+    hs = []
+    for ev in events:
+        if ev is None:
+            hs.append(None)
+            continue
+        if not ev.cuda_event:  # torch creates the CUDA event lazily
+            ev.record()
+        hs.append(ctypes.c_void_p(ev.cuda_event))
+    return (ctypes.c_void_p * len(hs))(*hs)
+
+
+def forward_profiled(cfg: MoEConfig, x: torch.Tensor, w: MoEWeights, ws: torch.Tensor, events, image_mask=None,
+                     out=None, topk_idx_out=None, expert_counts_out=None, stream=None) -> torch.Tensor:
+    """moe_forward_profiled: `events` are 7 torch.cuda.Event (or None), recorded at the stage
+    boundaries: before route, then after route, dispatch, gate/up, down, shared, combine."""
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, cfg.hidden_dim), dtype=out_torch_dtype(cfg), device=x.device)
+    _expect(out, (T, cfg.hidden_dim), out_torch_dtype(cfg), "out")
+    _expect(topk_idx_out, (T, cfg.top_k), torch.int32, "topk_idx_out")
+    _expect(expert_counts_out, (cfg.num_experts,), torch.int32, "expert_counts_out")
+    if len(events) != STAGE_EVENTS:
+        raise ValueError(f"forward_profiled needs {STAGE_EVENTS} events")
+    _check(lib.moe_forward_profiled(ctypes.byref(cfg), T, _p(x), ctypes.byref(w), _p(image_mask), _p(out),
+                                    _p(topk_idx_out), _p(expert_counts_out), _p(ws), ws.numel(), _stream(stream),
+                                    ctypes.cast(_event_handles(events), ctypes.c_void_p), STAGE_EVENTS),
+           "moe_forward_profiled")
     return out
 
 

@@ -77,9 +77,9 @@ struct ExpertWs {
 };
 inline bool gate_up_direct(const MoEConfig &c) { return fp4_direct_ok(c, c.hidden_dim); }
 inline bool down_direct(const MoEConfig &c) { return fp4_direct_ok(c, c.intermediate_dim); }
-ExpertWs carve_expert(Carve &cv, const MoEConfig &c) {
+ExpertWs carve_expert(Carve &cv, const MoEConfig &c, bool with_status = true) {
   ExpertWs w;
-  w.status = cv.take<int>(kStatusBytes / sizeof(int));
+  w.status = with_status ? cv.take<int>(kStatusBytes / sizeof(int)) : nullptr;
   w.wexp = nullptr;
   if (c.expert_dtype == MOE_NVFP4) {
     const size_t n = (size_t)c.num_experts * c.intermediate_dim * c.hidden_dim;
@@ -95,7 +95,7 @@ moe_status run_gate_up(const MoEConfig &c, int rows, const void *a, int a_rows, 
                        void *h, const ExpertWs &ws, cudaStream_t s) {
   MoEConfig cc = c;
   if (gate_up_direct(c))
-    return launch_gate_up_fp4(c, rows, a, a_rows, row_token, offsets, wg, wu, sg, su, h, ws.status, s);
+    return launch_gate_up_fp4(c, rows, a, a_rows, row_token, offsets, wg, wu, sg, su, nullptr, h, ws.status, s);
   if (c.expert_dtype == MOE_NVFP4) {
     const long n = (long)c.num_experts * c.intermediate_dim * c.hidden_dim;
     moe_status st = launch_dequant_nvfp4(wg, sg, n, ws.wexp, s);
@@ -167,7 +167,7 @@ struct ForwardWs {
   int *status;
   int *sched;
   int32_t *topk_idx, *counts, *offsets, *slot_row, *row_token, *chunk_cnt;
-  float *topk_w, *row_weight;
+  float *topk_w, *row_weight, *row_scale;
   void *x_perm, *h, *y_perm, *sh_y;
   ExpertWs ex;
 };
@@ -189,6 +189,7 @@ ForwardWs carve_forward(Carve &cv, const MoEConfig &c, int T) {
   w.slot_row = cv.take<int32_t>(Tk);
   w.row_token = cv.take<int32_t>(Tk);
   w.row_weight = cv.take<float>(Tk);
+  w.row_scale = gate_up_direct(c) ? cv.take<float>(Tk) : nullptr;
   w.chunk_cnt = cv.take<int32_t>((size_t)num_chunks(T) * E);
   w.x_perm = cv.take<char>(Tk * D * as);
   size_t hrows = Tk * c.intermediate_dim;
@@ -197,9 +198,7 @@ ForwardWs carve_forward(Carve &cv, const MoEConfig &c, int T) {
   w.y_perm = cv.take<float>(Tk * D);
   w.sh_y = c.shared_intermediate_dim ? cv.take<float>((size_t)T * D) : nullptr;
   w.ex.status = w.status;
-  w.ex.wexp = nullptr;
-  if (c.expert_dtype == MOE_NVFP4)
-    w.ex.wexp = cv.take<__nv_bfloat16>(3ull * c.num_experts * c.intermediate_dim * D);
+  w.ex.wexp = carve_expert(cv, c, false).wexp;  // NVFP4 expansion space, if any projection needs it
   return w;
 }
 
@@ -390,15 +389,21 @@ size_t moe_workspace_size(const MoEConfig *cfg, int T) {
   return align_up(cv.off, 256);
 }
 
-moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
-                       const uint8_t *image_mask, void *out, int32_t *topk_idx_out,
-                       int32_t *expert_counts_out, void *ws, size_t ws_bytes, moe_stream_t stream) {
+static moe_status forward_impl(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
+                               const uint8_t *image_mask, void *out, int32_t *topk_idx_out,
+                               int32_t *expert_counts_out, void *ws, size_t ws_bytes, moe_stream_t stream,
+                               void *const *events) {
   moe_status st = validate_cfg(cfg);
   if (st != MOE_OK) return st;
   if ((st = validate_tokens(cfg, T)) != MOE_OK) return st;
   if (!w || !ws) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < moe_workspace_size(cfg, T)) return MOE_ERR_WORKSPACE;
-  if (T == 0) return MOE_OK;
+  if (T == 0) {  // nothing to compute; the stage boundaries still get their events
+    for (int e = 0; events && e < MOE_STAGE_EVENTS; ++e)
+      if (events[e] && cudaEventRecord((cudaEvent_t)events[e], (cudaStream_t)stream) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
   if (!ok_ptr(x) || !ok_ptr(out) || !ok_ptr(w->w_router)) return MOE_ERR_INVALID_ARG;
   if (!ok_matrix(cfg, w->w_gate, w->s_gate) || !ok_matrix(cfg, w->w_up, w->s_up) ||
       !ok_matrix(cfg, w->w_down, w->s_down))
@@ -413,25 +418,69 @@ moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeig
   int32_t *idx = topk_idx_out ? topk_idx_out : f.topk_idx;
   int32_t *counts = expert_counts_out ? expert_counts_out : f.counts;
   const int rows = T * c.top_k;
+  // stage boundary i: record events[i] when the caller asked for it
+  auto mark = [&](int i) -> moe_status {
+    if (events && events[i] && cudaEventRecord((cudaEvent_t)events[i], s) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  };
 
+  if ((st = mark(0)) != MOE_OK) return st;
   if ((st = launch_route(c, T, x, w->w_router, w->bias, w->bias_vl, image_mask, idx, f.topk_w, f.status, s)) !=
       MOE_OK)
     return st;
+  if ((st = mark(1)) != MOE_OK) return st;
+  // NVFP4 experts on the direct path: x_perm is gathered in f16 with a
+  // power-of-two scale per row and the gate/up GEMM multiplies in f16
+  const bool fp4_f16 = f.row_scale != nullptr;
   if ((st = launch_dispatch(c, T, idx, f.topk_w, x, counts, f.offsets, f.slot_row, f.row_token,
-                            f.row_weight, f.x_perm, f.chunk_cnt, s)) != MOE_OK)
+                            f.row_weight, fp4_f16 ? nullptr : f.x_perm, f.chunk_cnt, s)) != MOE_OK)
     return st;
-  // x_perm from the dispatch gather: the in-GEMM gather (TMA gather4, 512 bytes
-  // per copy) cannot keep the tensor cores fed, a dense tile load can
-  if ((st = run_experts(c, rows, f.x_perm, rows, nullptr, f.offsets, w->w_gate, w->w_up, w->w_down, w->s_gate,
-                        w->s_up, w->s_down, f.row_weight, f.h, f.y_perm, f.ex, f.sched, s)) != MOE_OK)
+  if (fp4_f16 && (st = launch_gather_f16(c, T, f.offsets, f.row_token, x, f.x_perm, f.row_scale, s)) != MOE_OK)
     return st;
+  if ((st = mark(2)) != MOE_OK) return st;
+  if (fp4_f16 || events) {
+    // the two projections as separate launches (the stage boundary between them is observable)
+    if (fp4_f16) {
+      st = launch_gate_up_fp4(c, rows, f.x_perm, rows, nullptr, f.offsets, w->w_gate, w->w_up, w->s_gate, w->s_up,
+                              f.row_scale, f.h, f.ex.status, s);
+    } else {
+      st = run_gate_up(c, rows, f.x_perm, rows, nullptr, f.offsets, w->w_gate, w->w_up, w->s_gate, w->s_up, f.h,
+                       f.ex, s);
+    }
+    if (st != MOE_OK) return st;
+    if ((st = mark(3)) != MOE_OK) return st;
+    if ((st = run_down(c, rows, f.h, f.offsets, w->w_down, w->s_down, f.row_weight, f.y_perm, f.ex, s)) != MOE_OK)
+      return st;
+  } else if ((st = run_experts(c, rows, f.x_perm, rows, nullptr, f.offsets, w->w_gate, w->w_up, w->w_down, w->s_gate,
+                        w->s_up, w->s_down, f.row_weight, f.h, f.y_perm, f.ex, f.sched, s)) != MOE_OK) {
+    return st;
+  }
+  if ((st = mark(4)) != MOE_OK) return st;
   if (c.shared_intermediate_dim) {
     const MoEConfig sc = shared_cfg(c);
     if ((st = run_experts(sc, T, x, T, nullptr, nullptr, w->sh_gate, w->sh_up, w->sh_down, nullptr, nullptr,
                           nullptr, nullptr, f.h, f.sh_y, f.ex, f.sched, s)) != MOE_OK)
       return st;
   }
-  return launch_combine(c, T, f.y_perm, f.slot_row, f.sh_y, out, s);
+  if ((st = mark(5)) != MOE_OK) return st;
+  if ((st = launch_combine(c, T, f.y_perm, f.slot_row, f.sh_y, out, s)) != MOE_OK) return st;
+  return mark(6);
+}
+
+moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
+                       const uint8_t *image_mask, void *out, int32_t *topk_idx_out,
+                       int32_t *expert_counts_out, void *ws, size_t ws_bytes, moe_stream_t stream) {
+  return forward_impl(cfg, T, x, w, image_mask, out, topk_idx_out, expert_counts_out, ws, ws_bytes, stream,
+                      nullptr);
+}
+
+moe_status moe_forward_profiled(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
+                                const uint8_t *image_mask, void *out, int32_t *topk_idx_out,
+                                int32_t *expert_counts_out, void *ws, size_t ws_bytes, moe_stream_t stream,
+                                void *const *events, int n_events) {
+  if (n_events != 0 && (n_events != MOE_STAGE_EVENTS || !events)) return MOE_ERR_INVALID_ARG;
+  return forward_impl(cfg, T, x, w, image_mask, out, topk_idx_out, expert_counts_out, ws, ws_bytes, stream,
+                      n_events ? events : nullptr);
 }
 
 }  // extern "C"

@@ -178,7 +178,70 @@ __global__ void __launch_bounds__(256) gather_kernel(int max_rows, int D,
   }
 }
 
+// x_perm in f16 with one power-of-two scale per row, for the FP4 gate/up GEMM
+// that multiplies in f16: row r holds x[row_token[r]] * 2^s_r, with s_r chosen
+// so that the row's largest magnitude lands in [2^14, 2^15), and
+// row_scale[r] = 2^-s_r.  Scaling by a power of two is exact; a bf16 value v
+// (8 significant bits) is then exact in f16 whenever |v| >= max|row| * 2^-31
+// or v = 0, so the GEMM's products equal those of the bf16 operands.
+__global__ void __launch_bounds__(256) gather_f16_kernel(int max_rows, int D,
+                                                         const int32_t *__restrict__ expert_offsets, int E,
+                                                         const int32_t *__restrict__ row_token,
+                                                         const __nv_bfloat16 *__restrict__ x,
+                                                         __half *__restrict__ x_perm, float *__restrict__ row_scale) {
+  constexpr int V = 8;
+  const int R = min(expert_offsets[E], max_rows);
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += warps) {
+    const __nv_bfloat16 *src = x + (long)row_token[r] * D;
+    float m = 0.0f;
+#pragma unroll 8
+    for (int c = lane * V; c < D; c += 32 * V) {
+      const Vec16<__nv_bfloat16> v = load16(src + c);
+#pragma unroll
+      for (int j = 0; j < V; ++j) m = fmaxf(m, fabsf(v.get(j)));
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    // s = 14 - floor(log2 m), from m's exponent field; zero, subnormal or
+    // non-finite rows keep s in [-100, 100] so 2^s and 2^-s stay normal floats
+    int s = 0;
+    if (m > 0.0f) {
+      s = 14 - ((int)((__float_as_uint(m) >> 23) & 255u) - 127);
+      s = max(-100, min(100, s));
+    }
+    const float mul = __uint_as_float((uint32_t)(s + 127) << 23);
+    __half *dst = x_perm + (long)r * D;
+#pragma unroll 8
+    for (int c = lane * V; c < D; c += 32 * V) {
+      const Vec16<__nv_bfloat16> v = load16(src + c);
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        __half2 h2 = __floats2half2_rn(v.get(2 * j) * mul, v.get(2 * j + 1) * mul);
+        o[j] = *reinterpret_cast<uint32_t *>(&h2);
+      }
+      *reinterpret_cast<uint4 *>(dst + c) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    if (lane == 0) row_scale[r] = __uint_as_float((uint32_t)(127 - s) << 23);
+  }
+}
+
 }  // namespace
+
+moe_status launch_gather_f16(const MoEConfig &c, int T, const int32_t *expert_offsets, const int32_t *row_token,
+                             const void *x, void *x_perm, float *row_scale, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  if (c.act_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  int dev = 0, sms = 148;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  gather_f16_kernel<<<sms * 8, 256, 0, s>>>(T * c.top_k, c.hidden_dim, expert_offsets, c.num_experts, row_token,
+                                            (const __nv_bfloat16 *)x, (__half *)x_perm, row_scale);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
 
 moe_status launch_dispatch(const MoEConfig &c, int T, const int32_t *topk_idx, const float *topk_w,
                            const void *x, int32_t *expert_counts, int32_t *expert_offsets,

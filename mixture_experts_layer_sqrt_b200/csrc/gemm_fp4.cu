@@ -33,6 +33,13 @@
 //   warps 6-13   converters: codes + scales -> swizzled bf16 B tile (3-stage
 //                ring), one arrival per warp.
 //
+// F16 (gate/up inside moe_forward): A arrives as f16 rows pre-scaled by a
+// power of two per row (launch_gather_f16), the codes are expanded to f16
+// (e2m1 -> f16 needs no re-bias, so one conversion and one f16 multiply per
+// pair of weights), the MMAs run f16 x f16 -> fp32, and the epilogue undoes
+// the row scale.  All three steps are exact, so the result equals the bf16
+// path's bit for bit whenever the scaled activations are exact in f16.
+//
 // Tiles never straddle two experts; the tile list (expert-major, n-block,
 // m-block) comes from expert_offsets on the device.  Every wait is bounded
 // (2 s, then MOE_ERR_DEVICE_TIMEOUT in the status word and an orderly wind
@@ -90,6 +97,7 @@ struct Params {
   int clamp_mode;
   int *status;
   uint32_t hi_mul;           // 2^29, passed at run time so the multiply-add stays one
+  const float *row_scale;    // F16: 2^-s_r of each A row
 };
 
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Smem &sm, int *status) {
@@ -194,7 +202,33 @@ __device__ __forceinline__ uint4 expand_e2m1x8(uint32_t q, uint32_t scale2, uint
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-template <bool GATED>
+// e4m3 scale byte -> f16x2 of the scale, both halves (exact: e4m3 values are
+// normal f16 numbers).
+__device__ __forceinline__ uint32_t scale_f16x2(uint32_t b) {
+  const uint32_t E = (b >> 3) & 15u, m = b & 7u;
+  float v;
+  if (E == 15u && m == 7u) v = __uint_as_float(0x7fc00000u);          // the NaN code
+  else if (E) v = __uint_as_float(((E + 120u) << 23) | (m << 20));     // 2^(E-7) (1 + m/8)
+  else v = (float)m * __uint_as_float(118u << 23);                     // m 2^-9
+  if (b & 0x80u) v = -v;
+  const uint32_t h = __half_as_ushort(__float2half_rn(v));
+  return h | (h << 16);
+}
+
+// Eight e2m1 codes times one scale (from scale_f16x2) -> eight f16; each
+// product has at most 6 significant bits and lies in [2^-10, 2688]: exact.
+__device__ __forceinline__ uint4 expand_e2m1x8_f16(uint32_t q, uint32_t scale2) {
+  uint32_t h[4], o[4];
+  ptx::e2m1x8_to_f16x2(q, h);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    __half2 r = __hmul2(*reinterpret_cast<const __half2 *>(&h[j]), *reinterpret_cast<const __half2 *>(&scale2));
+    o[j] = *reinterpret_cast<uint32_t *>(&r);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <bool GATED, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_fp4_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                 const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmS0,
@@ -264,7 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) sm.tile_start[p.E] = carry;
   }
   if (warp >= 6) {
-    for (int b = (int)threadIdx.x - 192; b < 256; b += 32 * kConv) lut[b] = scale_bf16x2((uint32_t)b);
+    for (int b = (int)threadIdx.x - 192; b < 256; b += 32 * kConv)
+      lut[b] = F16 ? scale_f16x2((uint32_t)b) : scale_bf16x2((uint32_t)b);
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -335,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ================================================= MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = ptx::idesc_bf16_f32(TILE_M, FN);
+      constexpr uint32_t idesc = F16 ? ptx::idesc_f16_f32(TILE_M, FN) : ptx::idesc_bf16_f32(TILE_M, FN);
       uint32_t it = 0;
       int i = 0;
       bool ok = true;
@@ -386,6 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tl.m0 + q * 32 < tl.end) {  // warp-uniform: some row of this quarter is live
         if (GATED) {
           __nv_bfloat16 *hrow = (__nv_bfloat16 *)p.out + (long)row * p.N + tl.n_blk * (FN / 2);
+          const float rs = (F16 && live) ? p.row_scale[row] : 1.0f;
 #pragma unroll 1
           for (int c = 0; c < FN / 2; c += 32) {
             uint32_t g[32], u[32];
@@ -396,10 +432,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               uint32_t pk[16];
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
-                const float h0 =
-                    swiglu_h(__uint_as_float(g[2 * j]), __uint_as_float(u[2 * j]), p.clamp, p.clamp_mode);
-                const float h1 =
-                    swiglu_h(__uint_as_float(g[2 * j + 1]), __uint_as_float(u[2 * j + 1]), p.clamp, p.clamp_mode);
+                float g0 = __uint_as_float(g[2 * j]), u0 = __uint_as_float(u[2 * j]);
+                float g1 = __uint_as_float(g[2 * j + 1]), u1 = __uint_as_float(u[2 * j + 1]);
+                if (F16) {
+                  g0 *= rs;
+                  u0 *= rs;
+                  g1 *= rs;
+                  u1 *= rs;
+                }
+                const float h0 = swiglu_h(g0, u0, p.clamp, p.clamp_mode);
+                const float h1 = swiglu_h(g1, u1, p.clamp, p.clamp_mode);
                 __nv_bfloat162 b2 = __floats2bfloat162_rn(h0, h1);
                 pk[j] = *reinterpret_cast<uint32_t *>(&b2);
               }
@@ -473,7 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < JOBS; ++j) sc[j] = lut[sc[j]];
 #pragma unroll
         for (int j = 0; j < JOBS; ++j)
-          *reinterpret_cast<uint4 *>(dst + j * ROW_STEP * (BK * 2)) = expand_e2m1x8(qv[j], sc[j], p.hi_mul);
+          *reinterpret_cast<uint4 *>(dst + j * ROW_STEP * (BK * 2)) =
+              F16 ? expand_e2m1x8_f16(qv[j], sc[j]) : expand_e2m1x8(qv[j], sc[j], p.hi_mul);
         ptx::fence_proxy_async_smem();  // the MMA reads these stores through the async proxy
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&sm.b_full[sb]);
@@ -497,7 +540,7 @@ static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 // A: [rows, K] bf16 (or the gather source); codes [E, Nw, K/2] bytes and
 // scales [E, Nw, K/16] bytes for b0/s0 (and b1/s1 when gated).
-template <bool GATED>
+template <bool GATED, bool F16>
 moe_status launch_fp4(const Params &p, const void *a, const void *b0, const void *b1, const void *s0,
                       const void *s1, int Nw, cudaStream_t s) {
   CUtensorMap ta, tb0, tb1, ts0, ts1;
@@ -516,7 +559,7 @@ moe_status launch_fp4(const Params &p, const void *a, const void *b0, const void
   int dev = 0, sms = 148;
   MOE_CUDA_TRY(cudaGetDevice(&dev));
   MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  auto kern = tc_fp4_gemm<GATED>;
+  auto kern = tc_fp4_gemm<GATED, F16>;
   MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes));
   const long ub = ((long)(p.rows + TILE_M - 1) / TILE_M + (p.offsets ? p.E : 0)) * p.n_tiles;  // tile bound
   if (ub <= 0) return MOE_OK;
@@ -537,7 +580,7 @@ bool fp4_direct_ok(const MoEConfig &c, int K) {
 
 moe_status launch_gate_up_fp4(const MoEConfig &c, int rows, const void *a, int a_rows, const int32_t *row_token,
                               const int32_t *offsets, const void *w_gate, const void *w_up, const void *s_gate,
-                              const void *s_up, void *h, int *status, cudaStream_t s) {
+                              const void *s_up, const float *row_scale, void *h, int *status, cudaStream_t s) {
   if (rows == 0) return MOE_OK;
   Params p;
   p.rows = rows;
@@ -554,7 +597,9 @@ moe_status launch_gate_up_fp4(const MoEConfig &c, int rows, const void *a, int a
   p.clamp_mode = c.clamp_mode;
   p.status = status;
   p.hi_mul = 1u << 29;
-  return launch_fp4<true>(p, a, w_gate, w_up, s_gate, s_up, c.intermediate_dim, s);
+  p.row_scale = row_scale;
+  if (row_scale) return launch_fp4<true, true>(p, a, w_gate, w_up, s_gate, s_up, c.intermediate_dim, s);
+  return launch_fp4<true, false>(p, a, w_gate, w_up, s_gate, s_up, c.intermediate_dim, s);
 }
 
 moe_status launch_down_fp4(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
@@ -576,7 +621,8 @@ moe_status launch_down_fp4(const MoEConfig &c, int rows, const void *h, const in
   p.clamp_mode = 0;
   p.status = status;
   p.hi_mul = 1u << 29;
-  return launch_fp4<false>(p, h, w_down, nullptr, s_down, nullptr, c.hidden_dim, s);
+  p.row_scale = nullptr;
+  return launch_fp4<false, false>(p, h, w_down, nullptr, s_down, nullptr, c.hidden_dim, s);
 }
 
 }  // namespace moe

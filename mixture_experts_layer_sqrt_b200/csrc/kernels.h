@@ -33,6 +33,11 @@ moe_status launch_dispatch(const MoEConfig &c, int T, const int32_t *topk_idx, c
                            int32_t *slot_row, int32_t *row_token, float *row_weight, void *x_perm,
                            int32_t *chunk_cnt, cudaStream_t s);
 
+// x_perm rows in f16, each scaled by a power of two (row_scale[r] = 2^-s_r),
+// for the FP4 gate/up GEMM in f16 (bf16 activations only).
+moe_status launch_gather_f16(const MoEConfig &c, int T, const int32_t *expert_offsets, const int32_t *row_token,
+                             const void *x, void *x_perm, float *row_scale, cudaStream_t s);
+
 // gemm_simt.cu -----------------------------------------------------------
 // Grouped GEMMs on CUDA cores (fp32 FMA), any shape.  act: F32 or BF16 for
 // activations and weights alike.
@@ -61,9 +66,11 @@ moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int
 // and scales expanded to bf16 on chip).  Usable when fp4_direct_ok() for the
 // projection's reduction length K (D for gate/up, F for down).
 bool fp4_direct_ok(const MoEConfig &c, int K);
+// row_scale non-null: `a` holds f16 rows scaled by 2^s_r (launch_gather_f16)
+// and the MMAs run in f16; the epilogue multiplies g and u by row_scale[r].
 moe_status launch_gate_up_fp4(const MoEConfig &c, int rows, const void *a, int a_rows, const int32_t *row_token,
                               const int32_t *offsets, const void *w_gate, const void *w_up, const void *s_gate,
-                              const void *s_up, void *h, int *status, cudaStream_t s);
+                              const void *s_up, const float *row_scale, void *h, int *status, cudaStream_t s);
 moe_status launch_down_fp4(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
                            const void *w_down, const void *s_down, const float *row_weight, float *y,
                            int *status, cudaStream_t s);

@@ -140,5 +140,20 @@ def test_gather_needs_source_rows(B):
     assert st == B.MOE_ERR_INVALID_ARG
 
 
+def test_profiled_forward_event_count(B):
+    # 0 events (plain forward) or exactly MOE_STAGE_EVENTS; checked before any CUDA work
+    c = _cfg(B)
+    w = B.MoEWeights(w_router=16, w_gate=16, w_up=16, w_down=16)
+    need = B.lib.moe_workspace_size(ctypes.byref(c), 64)
+    ev = (ctypes.c_void_p * 7)()
+    for n in (1, 6, 8, -1):
+        st = B.lib.moe_forward_profiled(ctypes.byref(c), 64, 16, ctypes.byref(w), None, 16, None, None, 16, need,
+                                        None, ctypes.cast(ev, ctypes.c_void_p), n)
+        assert st == B.MOE_ERR_INVALID_ARG
+    st = B.lib.moe_forward_profiled(ctypes.byref(c), 64, 16, ctypes.byref(w), None, 16, None, None, 16, need,
+                                    None, None, 7)
+    assert st == B.MOE_ERR_INVALID_ARG
+
+
 def test_launch_count_starts_at_zero_without_gpu(B):
     assert B.launch_count() >= 0

@@ -401,6 +401,43 @@ def test_fp4_direct_matches_expanded_weights(B, W, name, monkeypatch):
     assert torch.equal(y4[:R], y16[:R])
 
 
+@pytest.mark.parametrize("name", ["mixtral_bf16", "sqrt_fp4"])
+def test_profiled_forward_matches(B, W, name):
+    # the stage events change nothing in the result; they bracket the stages in order
+    p = H.small(name)
+    c = Case(B, W, p)
+    ws = B.workspace(B.workspace_size(c.cfg, p.T))
+    ref = B.forward(c.cfg, c.x, c.w, ws, c.mask)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(B.STAGE_EVENTS)]
+    got = B.forward_profiled(c.cfg, c.x, c.w, ws, ev, c.mask)
+    torch.cuda.synchronize()
+    B.check_device_status(ws)
+    assert torch.equal(got, ref)
+    stage = [ev[i].elapsed_time(ev[i + 1]) for i in range(B.STAGE_EVENTS - 1)]
+    assert all(t >= 0.0 for t in stage)
+    assert abs(sum(stage) - ev[0].elapsed_time(ev[-1])) < 1e-2
+
+
+def test_fp4_forward_f16_rows_exact(B, W):
+    # moe_forward gathers NVFP4 gate/up rows in f16 under a power-of-two scale
+    # per row: rows of any magnitude (zero, tiny, large) keep the bf16 path's
+    # products, so the layer equals the staged bf16-operand result bit for bit
+    p = H.small("sqrt_fp4")
+    c = Case(B, W, p)
+    x = c.x.float()
+    x[0] = 0.0
+    x[1] *= 1.0e4
+    x[2] *= 1.0e-6
+    x[3] *= 3.0e-30
+    c.x = x.to(torch.bfloat16)
+    g = _stages(B, c)
+    ws = B.workspace(B.workspace_size(c.cfg, p.T))
+    out_f = B.forward(c.cfg, c.x, c.w, ws, c.mask)
+    torch.cuda.synchronize()
+    B.check_device_status(ws)
+    assert torch.equal(out_f, g["out"])
+
+
 def test_host_batches_overlapped_copies(B, W):
     # pinned host batches through the overlapped-copy path give the same
     # outputs as one forward per device batch
