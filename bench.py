@@ -147,6 +147,42 @@ def oracle_sample(p, arrays, n_tokens: int, seed: int):
     return time.perf_counter() - t0
 
 
+# ------------------------------------------------------------ ranks (host)
+
+def rank_problem(p, rank: int):
+    """The token batch of one data-parallel rank: same weights, its own tokens
+    (rank 0 keeps the workload's seed; rank r draws x from seed + 1000 r)."""
+    return p if rank == 0 else p.with_(seed=p.seed + 1000 * rank)
+
+
+def rank_arrays(p, rank: int, synth):
+    arrays = synth.generate(p)
+    if rank > 0:
+        arrays["x"] = synth.generate(rank_problem(p, rank), experts=False)["x"]
+    return arrays
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The job's time is the slowest rank's (an all-reduce MAX; identity on one rank)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Tokens per second of the whole job: every rank processes its own batch each step."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
+def emit(res, rank: int):
+    """Rank 0 prints the one JSON line; the other ranks print nothing."""
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+
+
 # --------------------------------------------------------------------- ours
 
 def run_ours(args, p, rank, world, local_rank):
@@ -154,9 +190,7 @@ def run_ours(args, p, rank, world, local_rank):
     from mixture_experts_layer_sqrt_b200 import binding as B, synth, workload as WL
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    arrays = synth.generate(p)
-    if rank > 0:  # each rank its own tokens, same weights
-        arrays["x"] = synth.generate(p.with_(seed=p.seed + 1000 * rank), experts=False)["x"]
+    arrays = rank_arrays(p, rank, synth)  # each rank its own tokens, same weights
     cfg = WL.config_of(p)
     wt = WL.device_weights(p, arrays, dev)
     w = B.make_weights(wt)
@@ -214,13 +248,8 @@ def run_ours(args, p, rank, world, local_rank):
     stage_ms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in g_ev) / args.steps for i, n in enumerate(names)}
     gemm_ms = stage_ms["gate_up"]
     B.check_device_status(ws_f)
-    t_max = total_ms
-    if dist:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
-    ms = t_max / args.steps
-    value = world * T / (ms / 1e3)
+    ms = max_over_ranks(total_ms, dist, dev) / args.steps
+    value = whole_job_value(world, T, ms)
 
     e2e = None
     if not args.no_e2e:
@@ -256,13 +285,9 @@ def run_e2e(args, B, WL, cfg, wt, arrays, T, D, dev, stream, dist):
     layer.forward_host_batches(xs, outs, masks)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
     B.check_device_status(layer.ws)
-    return {"value": world * T / (e2e_ms / args.steps / 1e3), "unit": "tokens/s",
+    return {"value": whole_job_value(world, T, e2e_ms / args.steps), "unit": "tokens/s",
             "h2d_bytes_per_step": int(x_h.numel() * x_h.element_size() + (m_h.numel() if m_h is not None else 0)),
             "d2h_bytes_per_step": int(out_h[0].numel() * out_h[0].element_size()),
             "copies": "overlapped with compute on separate streams (forward_host_batches)"}
@@ -363,9 +388,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
-    if args.impl == "reference":
+    if args.impl == "reference":  # the oracle on the host cores: rank 0 only
         if rank == 0:
-            print(json.dumps(run_reference(args, p)), flush=True)
+            emit(run_reference(args, p), rank)
         return
 
     from mixture_experts_layer_sqrt_b200 import build
@@ -379,10 +404,9 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     try:
         res = run_ours(args, p, rank, world, local_rank)
-        if rank == 0:
-            if world == 1 and not args.no_cpu_baseline:
-                res["cpu_baseline"] = cpu_baseline_leg(p)
-            print(json.dumps(res), flush=True)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline_leg(p)
+        emit(res, rank)
     finally:
         if world > 1:
             import torch.distributed as dist
