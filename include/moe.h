@@ -130,6 +130,14 @@ uint64_t moe_launch_count(void);
  * MOE_ERR_DEVICE_TIMEOUT; MOE_ERR_CUDA if the stream reports an error. */
 moe_status moe_check_device_status(void *ws, moe_stream_t stream);
 
+/* Exercises the timeout path of the kernels' bounded waits: launches one
+ * block that waits, with the same bounded wait the GEMM pipelines use, on an
+ * mbarrier that nothing arrives on.  After the limit (2 s) it records
+ * MOE_ERR_DEVICE_TIMEOUT in the status word of `ws` and returns normally, so
+ * the context stays usable.  ws: >= 256 bytes.  For tests of the failure
+ * path; nothing else calls it. */
+moe_status moe_selftest_wait_timeout(void *ws, size_t ws_bytes, moe_stream_t stream);
+
 /* ------------------------------------------------------------ stage 1: route */
 
 /* Bytes of workspace moe_route_topk needs (its device status word). */

@@ -74,6 +74,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_workspace_size": (S, [cfgp, I]),
         "moe_forward": (I, [cfgp, I, P, wp, P, P, P, P, P, S, P]),
         "moe_forward_profiled": (I, [cfgp, I, P, wp, P, P, P, P, P, S, P, P, I]),
+        "moe_selftest_wait_timeout": (I, [P, S, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -89,7 +90,7 @@ EXPORTS = ("moe_status_string", "moe_version", "moe_expert_capacity", "moe_launc
            "moe_check_device_status", "moe_route_workspace_size", "moe_route_topk", "moe_dispatch_workspace_size",
            "moe_dispatch", "moe_dispatch_noalloc", "moe_grouped_swiglu_workspace_size", "moe_expert_workspace_size",
            "moe_expert_gate_up", "moe_expert_down", "moe_grouped_swiglu", "moe_combine",
-           "moe_workspace_size", "moe_forward", "moe_forward_profiled")
+           "moe_workspace_size", "moe_forward", "moe_forward_profiled", "moe_selftest_wait_timeout")
 
 
 def status_string(s: int) -> str:
@@ -330,6 +331,11 @@ def forward_profiled(cfg: MoEConfig, x: torch.Tensor, w: MoEWeights, ws: torch.T
                                     ctypes.cast(_event_handles(events), ctypes.c_void_p), STAGE_EVENTS),
            "moe_forward_profiled")
     return out
+
+
+def selftest_wait_timeout(ws: torch.Tensor, stream=None):
+    """Launch the never-satisfied bounded wait (about 2 s); the status word of ws then reads timeout."""
+    _check(lib.moe_selftest_wait_timeout(_p(ws), ws.numel(), _stream(stream)), "moe_selftest_wait_timeout")
 
 
 def check_device_status(ws: torch.Tensor, stream=None):

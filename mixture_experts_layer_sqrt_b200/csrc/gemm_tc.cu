@@ -942,7 +942,25 @@ bool use_pair(int rows, int E, bool gated) {
   return rows >= (gated ? 2048L : 768L) * E;
 }
 
+// One thread waits on an mbarrier that nothing arrives on, with the bounded
+// wait of the pipelines above: it gives up after kWaitLimitNs and records the
+// timeout in the status word.
+__global__ void wait_selftest_kernel(int *status) {
+  __shared__ Smem sm;
+  if (threadIdx.x != 0) return;
+  sm.abort = 0;
+  ptx::mbar_init(&sm.full[0], 1);
+  ptx::fence_mbar_init();
+  wait_bar<false>(&sm.full[0], 0, sm, status, 0);
+}
+
 }  // namespace
+
+moe_status launch_wait_selftest(int *status, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(status);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
 
 bool tc_shapes_ok(const MoEConfig &c, int F) {
   return c.act_dtype == MOE_BF16 && c.hidden_dim % BN == 0 && F % 128 == 0 && c.hidden_dim % BK == 0 &&

@@ -19,6 +19,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "route_select.cuh"
 
 namespace moe {
 namespace {
@@ -39,52 +40,6 @@ __device__ __forceinline__ float transpose_reduce32(float (&a)[32], int lane) {
     }
   }
   return a[0];
-}
-
-// Top-k of one token's logits (in shared memory) and its weights, by one warp:
-// k rounds of a warp argmax (larger key first, equal keys to the lower expert).
-__device__ __forceinline__ void select_topk(const float *lg, long t, int E, int k, int gate,
-                                            const float *__restrict__ bias, const float *__restrict__ bias_vl,
-                                            const uint8_t *__restrict__ image_mask, int32_t *__restrict__ topk_idx,
-                                            float *__restrict__ topk_w, int lane) {
-  const float *sel_bias = nullptr;
-  if (gate == MOE_GATE_SQRT_SOFTPLUS_RAW) sel_bias = (bias_vl && image_mask && image_mask[t]) ? bias_vl : bias;
-  uint32_t removed = 0;  // bit j: expert lane + 32 j already selected
-  int my_e = 0;
-  float my_l = 0.0f;
-  for (int r = 0; r < k; ++r) {
-    float bk = -INFINITY;
-    int be = E;
-    for (int j = 0, e = lane; e < E; ++j, e += 32) {
-      if (removed >> j & 1u) continue;
-      float key = lg[e] + (sel_bias ? sel_bias[e] : 0.0f);
-      if (key != key) key = -INFINITY;
-      if (key > bk || (key == bk && e < be)) { bk = key; be = e; }
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-      int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      if (ok > bk || (ok == bk && oe < be)) { bk = ok; be = oe; }
-    }
-    if ((be & 31) == lane) removed |= 1u << (be >> 5);
-    if (lane == r) { my_e = be; my_l = lg[be]; }
-  }
-  float w;
-  if (gate == MOE_GATE_SOFTMAX_TOPK_RENORM) {
-    float m = __shfl_sync(0xffffffffu, my_l, 0);  // the largest selected logit
-    float ex = lane < k ? expf(my_l - m) : 0.0f;
-    float sum = ex;
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    w = ex / sum;
-  } else {
-    w = sqrtf(softplus_f32(my_l));
-  }
-  if (lane < k) {
-    topk_idx[t * k + lane] = my_e;
-    topk_w[t * k + lane] = w;
-  }
 }
 
 // Few experts: one token per warp.  The warp first issues every 16-byte load
@@ -232,10 +187,10 @@ moe_status launch_route_t(const MoEConfig &c, int T, const void *x, const void *
 
 moe_status launch_route(const MoEConfig &c, int T, const void *x, const void *w_router,
                         const float *bias, const float *bias_vl, const uint8_t *image_mask,
-                        int32_t *topk_idx, float *topk_w, int *status, cudaStream_t s) {
+                        int32_t *topk_idx, float *topk_w, int *status, float *scratch, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   if (route_tc_ok(c))
-    return launch_route_tc(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, status, s);
+    return launch_route_tc(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, status, scratch, s);
   const int E = c.num_experts;
   if (E <= 32) {  // one token per warp, x row slice in registers
     const size_t smem = (size_t)kFewWarps * E * sizeof(float);

@@ -3,8 +3,9 @@
 // logits r = W_r x ("FFN、SwiGLU 与 MoE" sec. 3; ops-transformer MoE walkthrough,
 // 优化一) with fp32 accumulation (坑三), then the gate and a partial top-k
 // selection (优化二) -- here without a heap and without writing the logits to
-// HBM: they stay in TMEM and each epilogue thread streams its token's row out
-// in 32-column chunks into a sorted register list.  Softmax mode: weights
+// HBM: the tensor-core kernel leaves them in an L2-resident scratch row per
+// token and a second kernel selects each token's top-k with one warp (k rounds
+// of a warp argmax) on every SM.  Softmax mode: weights
 // are the renormalised softmax of the selected (optionally logit-biased)
 // logits.  Sqrt mode: selection on s + bias / bias_vl, weights
 // sqrt(softplus(s)) of the raw score ("5A · MoE fine-grained" sec. 1, 3).
@@ -14,10 +15,14 @@
 // tcgen05.mma (M=128, N <= 256 per instruction, two instructions when
 // E_pad > 256) into fp32 TMEM accumulators of E_pad columns -- up to four,
 // fed by interleaved k-blocks and summed in a fixed order afterwards, which
-// keeps each fp32 sum short; warps 2-5 own one token (TMEM lane) per thread
-// for the selection.  All waits bounded.
+// keeps each fp32 sum short.  Warps 2-5 then sum the accumulators of their
+// tokens (TMEM lanes) and store the logit rows.  Selecting in this kernel
+// left 4 warps per 128 tokens doing a serial search on 64 SMs at T = 8192
+// (~130 us of 175); the separate selection kernel spreads it over the GPU.
+// All waits bounded.
 #include "common.cuh"
 #include "kernels.h"
+#include "route_select.cuh"
 #include "tc_ptx.cuh"
 #include "tma_host.h"
 
@@ -34,13 +39,11 @@ constexpr uint64_t kRDrainNs = 200000000ull;
 
 struct RParams {
   int T, D, E, E_pad, k, gate, stages, b_rows;
+  float *logits;  // [T, ld] fp32 out (router logit bias included in softmax mode)
+  int ld;         // logit row stride: E_pad rounded up to whole 32-column chunks
   int n_acc;  // independent accumulators over interleaved k-blocks (shorter fp32 sums)
   uint32_t tmem_cols;
   const float *bias;
-  const float *bias_vl;
-  const uint8_t *image_mask;
-  int32_t *topk_idx;
-  float *topk_w;
   int *status;
 };
 
@@ -52,7 +55,6 @@ struct RSmem {
   uint32_t tmem_base;
   int abort;
   float bias[kMaxEPad];
-  float bias_vl[kMaxEPad];
 };
 
 __device__ __forceinline__ bool rwait(uint64_t *bar, uint32_t parity, RSmem &sm, int *status) {
@@ -79,28 +81,6 @@ __device__ __forceinline__ void rdrain(uint64_t *bar, uint32_t parity, int *stat
   }
 }
 
-// Insert (v, e, l) into a list sorted by descending key, equal keys ordered by
-// lower expert index; the smallest entry falls off the end.
-template <int KMAX>
-__device__ __forceinline__ void topk_insert(float (&kv)[KMAX], int (&ke)[KMAX], float (&kl)[KMAX], float v, int e,
-                                            float l) {
-#pragma unroll
-  for (int j = 0; j < KMAX; ++j) {
-    const bool better = v > kv[j] || (v == kv[j] && e < ke[j]);
-    if (better) {
-      const float tv = kv[j], tl = kl[j];
-      const int te = ke[j];
-      kv[j] = v;
-      ke[j] = e;
-      kl[j] = l;
-      v = tv;
-      e = te;
-      l = tl;
-    }
-  }
-}
-
-template <int KMAX>
 __global__ void __launch_bounds__(kRThreads, 1)
     tc_route_topk(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, const RParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -131,11 +111,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
     ptx::tmem_alloc(&sm.tmem_base, p.tmem_cols);
     ptx::tmem_relinquish();
   }
-  if (warp >= 2) {
-    for (int e = threadIdx.x - 64; e < p.E; e += kRThreads - 64) {
-      sm.bias[e] = p.bias ? p.bias[e] : 0.0f;
-      sm.bias_vl[e] = p.bias_vl ? p.bias_vl[e] : 0.0f;
-    }
+  if (warp >= 2) {  // router logit bias (softmax mode), added before the logits are stored
+    for (int e = threadIdx.x - 64; e < p.E; e += kRThreads - 64)
+      sm.bias[e] = (p.bias && p.gate == MOE_GATE_SOFTMAX_TOPK_RENORM) ? p.bias[e] : 0.0f;
   }
   ptx::tc_fence_before();
   __syncwarp();
@@ -194,7 +172,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
       rdrain(&sm.drain, 0, p.status);
     }
   } else {
-    // ---- selection: one token (TMEM lane) per thread
+    // ---- logit rows: one token (TMEM lane) per thread
     const int q = warp & 3;
     const int row = m0 + q * 32 + lane;
     bool ok = true;
@@ -202,16 +180,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
     if (__shfl_sync(0xffffffffu, ok, 0)) {
       ptx::tc_fence_after();
       const bool live = row < p.T;
-      const bool sqrt_gate = p.gate == MOE_GATE_SQRT_SOFTPLUS_RAW;
-      const float *sel = (sqrt_gate && live && p.bias_vl && p.image_mask && p.image_mask[row]) ? sm.bias_vl : sm.bias;
-      float kv[KMAX], kl[KMAX];
-      int ke[KMAX];
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        kv[j] = -INFINITY;
-        kl[j] = 0.0f;
-        ke[j] = 0x7fffffff;
-      }
+      float *dst = p.logits + (long)row * p.ld;  // chunk c writes columns [c, c + 32) < ld
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16);
       for (int c = 0; c < p.E_pad; c += 32) {
         uint32_t v[32];
@@ -226,39 +195,15 @@ __global__ void __launch_bounds__(kRThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) lsum[j] += __uint_as_float(v[j]);
         }
+        if (live) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int e = c + j;
-          if (e < p.E) {
-            float l = lsum[j];
-            if (!sqrt_gate) l += sm.bias[e];  // router logit bias: selection and weight
-            float key = sqrt_gate ? l + sel[e] : l;
-            if (key != key) key = -INFINITY;
-            const bool cand = key > kv[KMAX - 1] || (key == kv[KMAX - 1] && e < ke[KMAX - 1]);
-            if (cand) topk_insert<KMAX>(kv, ke, kl, key, e, l);
-          }
-        }
-      }
-      if (live) {
-        float w[KMAX];
-        if (!sqrt_gate) {
-          float sum = 0.0f;
-#pragma unroll
-          for (int j = 0; j < KMAX; ++j) {
-            w[j] = j < p.k ? expf(kl[j] - kl[0]) : 0.0f;
-            sum += w[j];
-          }
-#pragma unroll
-          for (int j = 0; j < KMAX; ++j) w[j] = w[j] / sum;
-        } else {
-#pragma unroll
-          for (int j = 0; j < KMAX; ++j) w[j] = sqrtf(softplus_f32(kl[j]));
-        }
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-          if (j < p.k) {
-            p.topk_idx[(long)row * p.k + j] = ke[j];
-            p.topk_w[(long)row * p.k + j] = w[j];
+          for (int j = 0; j < 32; j += 4) {
+            float4 o;
+            o.x = c + j < p.E ? lsum[j] + sm.bias[c + j] : -INFINITY;
+            o.y = c + j + 1 < p.E ? lsum[j + 1] + sm.bias[c + j + 1] : -INFINITY;
+            o.z = c + j + 2 < p.E ? lsum[j + 2] + sm.bias[c + j + 2] : -INFINITY;
+            o.w = c + j + 3 < p.E ? lsum[j + 3] + sm.bias[c + j + 3] : -INFINITY;
+            *reinterpret_cast<float4 *>(dst + c + j) = o;
           }
         }
       }
@@ -275,7 +220,36 @@ __global__ void __launch_bounds__(kRThreads, 1)
   }
 }
 
+// One warp per token: copy its logit row to shared memory, then select.
+constexpr int kSelWarps = 8;
+__global__ void __launch_bounds__(32 * kSelWarps) route_select_kernel(int T, int E, int ld, int k, int gate,
+                                                                     const float *__restrict__ logits,
+                                                                     const float *__restrict__ bias,
+                                                                     const float *__restrict__ bias_vl,
+                                                                     const uint8_t *__restrict__ image_mask,
+                                                                     int32_t *__restrict__ topk_idx,
+                                                                     float *__restrict__ topk_w) {
+  extern __shared__ float rows[];  // [kSelWarps][ld]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float *lg = rows + warp * ld;
+  for (long t = (long)blockIdx.x * kSelWarps + warp; t < T; t += (long)gridDim.x * kSelWarps) {
+    const float *src = logits + t * ld;
+    for (int e = lane; e < E; e += 32) lg[e] = src[e];
+    __syncwarp();
+    select_topk(lg, t, E, k, gate, bias, bias_vl, image_mask, topk_idx, topk_w, lane);
+    __syncwarp();
+  }
+}
+
 }  // namespace
+
+// Logit row stride of the tensor-core router: E padded to 16 (the MMA's N
+// granularity), then to whole 32-column TMEM load chunks.
+static int route_ld(int E) { return ((E + 15) / 16 * 16 + 31) / 32 * 32; }
+
+size_t route_scratch_floats(const MoEConfig &c, int T) {
+  return route_tc_ok(c) ? (size_t)T * route_ld(c.num_experts) : 0;
+}
 
 // Few experts: one CTA per 128 tokens leaves most SMs idle while it streams x,
 // and the CUDA-core router (all SMs) is faster (measured 52 vs 84 us at E=8).
@@ -286,7 +260,7 @@ bool route_tc_ok(const MoEConfig &c) {
 
 moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void *w_router, const float *bias,
                            const float *bias_vl, const uint8_t *image_mask, int32_t *topk_idx, float *topk_w,
-                           int *status, cudaStream_t s) {
+                           int *status, float *scratch, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   RParams p;
   p.T = T;
@@ -304,10 +278,8 @@ moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void 
   while (cols < need) cols <<= 1;
   p.tmem_cols = cols;
   p.bias = bias;
-  p.bias_vl = bias_vl;
-  p.image_mask = image_mask;
-  p.topk_idx = topk_idx;
-  p.topk_w = topk_w;
+  p.logits = scratch;
+  p.ld = route_ld(c.num_experts);
   p.status = status;
   const int stage_bytes = RBM * RBK * 2 + p.b_rows * RBK * 2;
   int stages = (192 * 1024) / stage_bytes;
@@ -317,13 +289,18 @@ moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void 
   if (!tma_map_bf16(&tw, w_router, 2, (uint64_t)p.D, (uint64_t)p.E, 1)) return MOE_ERR_CUDA;
   const size_t smem = 1024 + (size_t)p.stages * stage_bytes + sizeof(RSmem);
   const dim3 grid((T + RBM - 1) / RBM);
-  if (c.top_k <= 8) {
-    MOE_CUDA_TRY(cudaFuncSetAttribute(tc_route_topk<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    tc_route_topk<8><<<grid, kRThreads, smem, s>>>(tx, tw, p);
-  } else {
-    MOE_CUDA_TRY(cudaFuncSetAttribute(tc_route_topk<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    tc_route_topk<16><<<grid, kRThreads, smem, s>>>(tx, tw, p);
-  }
+  MOE_CUDA_TRY(cudaFuncSetAttribute(tc_route_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  tc_route_topk<<<grid, kRThreads, smem, s>>>(tx, tw, p);
+  MOE_LAUNCH_CHECK();
+  int dev = 0, sms = 148;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  long sel_blocks = ((long)T + kSelWarps - 1) / kSelWarps;
+  if (sel_blocks > (long)sms * 8) sel_blocks = (long)sms * 8;
+  const float *sel_bias = c.gate == MOE_GATE_SQRT_SOFTPLUS_RAW ? bias : nullptr;  // softmax: already in the logits
+  route_select_kernel<<<(unsigned)sel_blocks, 32 * kSelWarps, (size_t)kSelWarps * p.ld * sizeof(float), s>>>(
+      T, p.E, p.ld, p.k, p.gate, scratch, sel_bias, c.gate == MOE_GATE_SQRT_SOFTPLUS_RAW ? bias_vl : nullptr,
+      image_mask, topk_idx, topk_w);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }

@@ -155,5 +155,10 @@ def test_profiled_forward_event_count(B):
     assert st == B.MOE_ERR_INVALID_ARG
 
 
+def test_selftest_needs_a_status_word(B):
+    assert B.lib.moe_selftest_wait_timeout(None, 256, None) == B.MOE_ERR_INVALID_ARG
+    assert B.lib.moe_selftest_wait_timeout(16, 8, None) == B.MOE_ERR_INVALID_ARG
+
+
 def test_launch_count_starts_at_zero_without_gpu(B):
     assert B.launch_count() >= 0

@@ -438,6 +438,22 @@ def test_fp4_forward_f16_rows_exact(B, W):
     assert torch.equal(out_f, g["out"])
 
 
+def test_bounded_wait_times_out_and_context_survives(B, W):
+    # a wait that nothing satisfies gives up after its limit, records the
+    # timeout in the status word and returns; the GPU keeps working
+    ws = B.workspace(256)
+    B.selftest_wait_timeout(ws)
+    assert B.lib.moe_check_device_status(B._p(ws), None) == B.MOE_ERR_DEVICE_TIMEOUT
+    assert B.lib.moe_check_device_status(B._p(ws), None) == B.MOE_OK  # read and cleared
+    p = H.small("mixtral_bf16")
+    c = Case(B, W, p)
+    wsf = B.workspace(B.workspace_size(c.cfg, p.T))
+    out = B.forward(c.cfg, c.x, c.w, wsf, c.mask)
+    torch.cuda.synchronize()
+    B.check_device_status(wsf)
+    assert torch.isfinite(out).all()
+
+
 def test_host_batches_overlapped_copies(B, W):
     # pinned host batches through the overlapped-copy path give the same
     # outputs as one forward per device batch
