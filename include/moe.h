@@ -269,7 +269,13 @@ size_t moe_workspace_size(const MoEConfig *cfg, int T);
  *   topk_idx_out [T, k] int32 or NULL: copy of the routing decision
  *   expert_counts_out [E] int32 or NULL: assignments per expert before capacity
  *   ws: workspace of at least moe_workspace_size(cfg, T) bytes
- * No host synchronisation; per-expert counts never leave the device. */
+ * No host synchronisation; per-expert counts never leave the device.
+ * Same kernels and results as the stage entry points called in order, with
+ * one difference in operand format: for NVFP4 experts whose gate/up reduction
+ * length D is a multiple of 256, the gate/up GEMM multiplies f16 operands
+ * (x rows scaled by a power of two each, expanded FP4 weights) instead of
+ * bf16 ones.  Both are exact, so the results are identical whenever every
+ * element of a token row satisfies |x| >= max|row| * 2^-31 or x = 0. */
 moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
                        const uint8_t *image_mask, void *out, int32_t *topk_idx_out,
                        int32_t *expert_counts_out, void *ws, size_t ws_bytes, moe_stream_t stream);
