@@ -140,7 +140,9 @@ moe_status moe_selftest_wait_timeout(void *ws, size_t ws_bytes, moe_stream_t str
 
 /* ------------------------------------------------------------ stage 1: route */
 
-/* Bytes of workspace moe_route_topk needs (its device status word). */
+/* Bytes of workspace moe_route_topk needs: its device status word, plus for
+ * E > 32 with bf16 activations (the tensor-core router) the fp32 logit rows
+ * [T, E rounded up to 32] it hands to its selection kernel. */
 size_t moe_route_workspace_size(const MoEConfig *cfg, int T);
 
 /* Router GEMM + gate + top-k for T tokens (a1-a2).
