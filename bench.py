@@ -293,6 +293,20 @@ def run_e2e(args, B, WL, cfg, wt, arrays, T, D, dev, stream, dist):
             "copies": "overlapped with compute on separate streams (forward_host_batches)"}
 
 
+# fp32 layers run on the CUDA cores: 148 SMs x 128 fp32 lanes x 2 FLOP per FMA at the 1965 MHz maximum clock
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def gate_up_kernel(p, peaks):
+    """The gate/up launch the roofline object describes: (name, bound, peak, sustained peak, peak note)."""
+    if p.act == "f32":
+        return ("grouped_gemm_simt<gate/up> (fp32 CUDA-core FMA)", "alu", FP32_ALU_TFLOPS, FP32_ALU_TFLOPS,
+                "fp32 FMA: 148 SMs x 128 lanes x 2 FLOP x 1965 MHz (nominal unit counts and clock)")
+    name = ("tc_fp4_gemm<gate/up> (packed NVFP4 weights expanded on chip, f16 MMA)" if p.wdtype == "nvfp4"
+            else "tc_grouped_gemm<gate/up> (grouped gate/up GEMM + SwiGLU epilogue)")
+    return (name, "tensor", peaks["bf16"], peaks["bf16_sustained"], f"bf16_tflops (burst) of {peaks['src']}")
+
+
 def report(args, p, world, rows, value, ms, per_step, gemm_ms, e2e, n_launch, clocks):
     peaks = load_peaks()
     flops = layer_flops(p, rows)
@@ -301,6 +315,7 @@ def report(args, p, world, rows, value, ms, per_step, gemm_ms, e2e, n_launch, cl
     # reported beside it for a GPU that settles under its power cap
     peak_t = peaks["bf16"]
     achieved = gemm1_flops / (gemm_ms / 1e3) / 1e12
+    kernel, bound, peak_k, peak_sus, peak_kind = gate_up_kernel(p, peaks)
     ideal_ms = max(flops / (peak_t * 1e12), layer_bytes(p) / (peaks["hbm"] * 1e9)) * 1e3
     ideal_sus_ms = max(flops / (peaks["bf16_sustained"] * 1e12), layer_bytes(p) / (peaks["hbm"] * 1e9)) * 1e3
     res = {
@@ -317,11 +332,11 @@ def report(args, p, world, rows, value, ms, per_step, gemm_ms, e2e, n_launch, cl
                            "flops": flops, "bytes": layer_bytes(p),
                            "peak": f"bf16 {peak_t} TFLOP/s burst ({peaks['bf16_sustained']} sustained), "
                                    f"HBM {peaks['hbm']} GB/s, of {peaks['src']}"},
-        "roofline": {"kernel": "tc_grouped_gemm<gate/up> (grouped gate/up GEMM + SwiGLU epilogue)",
-                     "bound": "tensor",
-                     "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s", "frac": achieved / peak_t,
-                     "frac_vs_sustained": achieved / peaks["bf16_sustained"],
-                     "peak_kind": f"bf16_tflops (burst) of {peaks['src']}",
+        "roofline": {"kernel": kernel,
+                     "bound": bound,
+                     "achieved": achieved, "peak": peak_k, "unit": "TFLOP/s", "frac": achieved / peak_k,
+                     "frac_vs_sustained": achieved / peak_sus,
+                     "peak_kind": peak_kind,
                      "flops_per_launch": gemm1_flops, "ms_per_launch": gemm_ms,
                      "traffic": profiled_traffic("gate_up_" + p.name)},
         "e2e": e2e,

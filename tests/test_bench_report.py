@@ -1,0 +1,41 @@
+"""bench.py's JSON line: every key the measurement contract names, and the
+roofline arithmetic (achieved = gate/up FLOP / launch time, frac = achieved /
+peak) for each kind of gate/up launch.  Pure host code: no GPU."""
+import argparse
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from mixture_experts_layer_sqrt_b200 import synth  # noqa: E402
+
+KEYS = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+        "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks")
+
+
+@pytest.mark.parametrize("name,kind,bound", [("mixtral_bf16", "tc_grouped_gemm", "tensor"),
+                                             ("sqrt_fp4", "tc_fp4_gemm", "tensor"),
+                                             ("tiny_f32", "grouped_gemm_simt", "alu")])
+def test_report_keys_and_roofline(name, kind, bound):
+    p = synth.PROBLEMS[name]
+    args = argparse.Namespace(steps=10, warmup=3)
+    rows = p.T * p.k
+    gemm_ms, ms = 1.5, 2.5
+    value = bench.whole_job_value(2, p.T, ms)
+    e2e = {"value": 1.0, "unit": "tokens/s", "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 1}
+    res = bench.report(args, p, 2, rows, value, ms, [ms] * 10, gemm_ms, e2e, 80, None)
+    for k in KEYS:
+        assert k in res, k
+    r = res["roofline"]
+    assert r["kernel"].startswith(kind) and r["bound"] == bound and r["unit"] == "TFLOP/s"
+    flops = 4.0 * rows * p.D * p.F
+    assert r["achieved"] == pytest.approx(flops / (gemm_ms / 1e3) / 1e12)
+    assert r["frac"] == pytest.approx(r["achieved"] / r["peak"])
+    assert res["value"] == pytest.approx(2 * p.T / (ms / 1e3))
+    assert res["n_gpus"] == 2 and res["scaling"] == "weak" and res["vs_baseline"] is None
+    assert res["gpu_launches"] == 80 and res["gpu_launches_per_step"] == 8
+    assert res["dtype"] == ("f32" if p.act == "f32" else "bf16")
