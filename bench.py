@@ -67,9 +67,16 @@ def load_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
 
 
-def gemm_sources_sha() -> str:
+# the sources each recorded traffic figure depends on (a change to any of them voids the record)
+TRAFFIC_SOURCES = {
+    "gate_up_mixtral_bf16": ("gemm_tc.cu", "tc_ptx.cuh", "tma_host.h", "common.cuh"),
+    "gate_up_sqrt_fp4": ("gemm_fp4.cu", "tc_ptx.cuh", "tma_host.h", "common.cuh"),
+}
+
+
+def gemm_sources_sha(files=TRAFFIC_SOURCES["gate_up_mixtral_bf16"]) -> str:
     h = hashlib.sha256()
-    for n in ("gemm_tc.cu", "tc_ptx.cuh", "tma_host.h", "common.cuh"):
+    for n in files:
         p = os.path.join(ROOT, "mixture_experts_layer_sqrt_b200", "csrc", n)
         if os.path.exists(p):
             h.update(open(p, "rb").read())
@@ -77,11 +84,11 @@ def gemm_sources_sha() -> str:
 
 
 def profiled_traffic(kernel_key: str):
-    """DRAM bytes per launch recorded from an ncu capture, if the kernel sources are unchanged since."""
+    """DRAM bytes per launch recorded from an ncu capture, if the kernel's sources are unchanged since."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
-    if not os.path.exists(path):
+    if not os.path.exists(path) or kernel_key not in TRAFFIC_SOURCES:
         return None
-    want = gemm_sources_sha()
+    want = gemm_sources_sha(TRAFFIC_SOURCES[kernel_key])
     for line in open(path):
         parts = line.split()
         if len(parts) >= 3 and parts[0] == kernel_key and parts[1] == want:

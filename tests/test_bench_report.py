@@ -39,3 +39,14 @@ def test_report_keys_and_roofline(name, kind, bound):
     assert res["n_gpus"] == 2 and res["scaling"] == "weak" and res["vs_baseline"] is None
     assert res["gpu_launches"] == 80 and res["gpu_launches_per_step"] == 8
     assert res["dtype"] == ("f32" if p.act == "f32" else "bf16")
+
+
+def test_traffic_records_follow_their_kernel_sources(monkeypatch):
+    # each recorded DRAM figure is keyed to a hash of its kernel's sources;
+    # the record is void as soon as one of them differs
+    assert bench.profiled_traffic("gate_up_mixtral_bf16") > 0
+    assert bench.profiled_traffic("gate_up_sqrt_fp4") > 0
+    assert bench.profiled_traffic("gate_up_tiny_f32") is None
+    changed = dict(bench.TRAFFIC_SOURCES, gate_up_sqrt_fp4=("gemm_fp4.cu", "api.cu"))
+    monkeypatch.setattr(bench, "TRAFFIC_SOURCES", changed)
+    assert bench.profiled_traffic("gate_up_sqrt_fp4") is None
