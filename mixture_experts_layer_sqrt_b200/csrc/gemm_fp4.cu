@@ -125,7 +125,7 @@ __device__ __forceinline__ void drain_bar(uint64_t *bar, uint32_t parity, int *s
   }
 }
 
-// Warp-uniform wait: lane 0 polls, the verdict is broadcast.
+// Warp-uniform wait: lane 0 polls, the outcome is broadcast to the warp.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, Smem &sm, int *status, int lane) {
   bool ok = true;
   if (lane == 0) ok = wait_bar(bar, parity, sm, status);
