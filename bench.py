@@ -422,7 +422,9 @@ def main():
         import datetime
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+        # short enough to end a job whose ranks wait on one another for good; long
+        # enough for every rank to generate its inputs (GBs of weights) on a shared host
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
         res = run_ours(args, p, rank, world, local_rank)
