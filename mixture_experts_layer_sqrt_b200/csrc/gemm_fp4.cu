@@ -15,8 +15,9 @@
 //
 // The expansion runs on the CUDA cores (hardware e2m1 -> f16 conversion, an
 // exponent re-bias to bf16, one bf16 multiply by the scale) and is balanced
-// between the integer-logic and the multiply-add pipes, so that converting
-// a 256-row B tile takes less time than the MMAs that consume it.  N = 256
+// between the integer-logic and the multiply-add pipes; it still sets the
+// pace (the MMAs wait on converted tiles), so every instruction per weight
+// counts.  N = 256
 // keeps the MMAs' shared-memory operand traffic low; pairs of CTAs are not
 // used because handing a converted half-tile to the peer CTA needs a
 // cluster-scope release per k-block, which costs more than converting the
