@@ -3,7 +3,8 @@
 Small shrunken copies of the five workloads (several tiles, ragged tails) are
 checked element by element; the full-size workloads on sampled tokens (routing
 and dispatch on every token).  Tolerances: indices, counts, rows and copies
-bit-exact (near-ties excepted and reported); routing weights 1e-5 relative;
+bit-exact (a selection may differ only on a k-th near-tie, and only within
+1e-4 of a valid top-k; see harness.check_selection); routing weights 1e-5 relative;
 fp32 layer 1e-5 relative; bf16/FP4 layer max|err| <= 2e-2 * rms(oracle).
 """
 import math
@@ -88,8 +89,8 @@ def test_stages_small(B, W, name):
 
     # a1-a2 route
     logits, idx_o, w_o, keys = H.oracle_route(p, c.L, c.a)
-    flips, ties = H.check_route(p, idx_g, w_g, logits, idx_o, keys, c.a.get("bias"))
-    print(f"{p.name}: near-ties {ties}, flipped {flips}")
+    rc = H.check_route(p, idx_g, w_g, logits, idx_o, keys, c.a.get("bias"))
+    print(f"{p.name}: {H.route_report(rc)}")
 
     # a3-a5 dispatch, conditioned on the GPU's selection: bit-exact
     d = O.dispatch(idx_g.astype(np.int64), p.E, c.C)
@@ -194,7 +195,7 @@ def _full_forward_check(B, W, name, n_sample):
     assert np.array_equal(idx_g, H.to_np(idx_t))
 
     logits, idx_o, w_o, keys = H.oracle_route(p, c.L, c.a)
-    flips, ties = H.check_route(p, idx_g, w_g, logits, idx_o, keys, c.a.get("bias"))
+    rc = H.check_route(p, idx_g, w_g, logits, idx_o, keys, c.a.get("bias"))
     d = O.dispatch(idx_g.astype(np.int64), p.E, c.C)
     R = int(d["offsets"][-1])
     np.testing.assert_array_equal(H.to_np(cnt_t), d["counts"])
@@ -215,7 +216,7 @@ def _full_forward_check(B, W, name, n_sample):
                       c.L.shared(), tokens=toks)
     got = H.to_np(out[torch.from_numpy(toks).cuda()])
     rel = H.assert_close_layer(p, got, o["out"], "out")
-    print(f"{name}: near-ties {ties}, flipped {flips}, sampled {len(toks)} tokens, max|err|/rms {rel:.3g}")
+    print(f"{name}: {H.route_report(rc)}, sampled {len(toks)} tokens, max|err|/rms {rel:.3g}")
 
 
 @pytest.mark.parametrize("name,n_sample", [("tiny_f32", 64), ("mixtral_bf16", 48), ("capacity_bf16", 48),
@@ -242,8 +243,8 @@ def test_route_many_experts(B, W, E, k, gate, bias):
     torch.cuda.synchronize()
     L = H.oracle_layer(p, a)
     logits, idx_o, w_o, keys = H.oracle_route(p, L, a)
-    flips, ties = H.check_route(p, H.to_np(idx), H.to_np(w), logits, idx_o, keys, a.get("bias"))
-    print(f"route E={E} k={k} {gate}: near-ties {ties}, flipped {flips}")
+    rc = H.check_route(p, H.to_np(idx), H.to_np(w), logits, idx_o, keys, a.get("bias"))
+    print(f"route E={E} k={k} {gate}: {H.route_report(rc)}")
 
 
 # ---------------------------------------------------------------- edge cases
