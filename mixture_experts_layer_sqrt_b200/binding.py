@@ -190,8 +190,10 @@ def dispatch(cfg: MoEConfig, x: torch.Tensor, topk_idx: torch.Tensor, topk_w: to
 
 
 def dispatch_noalloc(cfg: MoEConfig, x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,
-                     out: Optional[Dict[str, torch.Tensor]] = None, stream=None) -> Dict[str, torch.Tensor]:
-    """moe_dispatch_noalloc: dispatch with the library's own fixed scratch, no workspace."""
+                     out: Optional[Dict[str, torch.Tensor]] = None, stream=None,
+                     gather: bool = True) -> Dict[str, torch.Tensor]:
+    """moe_dispatch_noalloc: dispatch with the library's own fixed scratch, no
+    workspace.  gather=False builds the row maps only (x_perm None)."""
     T, D, E, k = x.shape[0], cfg.hidden_dim, cfg.num_experts, cfg.top_k
     dev = x.device
     o = out or dict(
@@ -200,7 +202,7 @@ def dispatch_noalloc(cfg: MoEConfig, x: torch.Tensor, topk_idx: torch.Tensor, to
         slot_row=torch.empty((T, k), dtype=torch.int32, device=dev),
         row_token=torch.empty(T * k, dtype=torch.int32, device=dev),
         row_weight=torch.empty(T * k, dtype=torch.float32, device=dev),
-        x_perm=torch.empty((T * k, D), dtype=x.dtype, device=dev))
+        x_perm=torch.empty((T * k, D), dtype=x.dtype, device=dev) if gather else None)
     _check(lib.moe_dispatch_noalloc(ctypes.byref(cfg), T, _p(topk_idx), _p(topk_w), _p(x),
                                     _p(o["expert_counts"]), _p(o["expert_offsets"]), _p(o["slot_row"]),
                                     _p(o["row_token"]), _p(o["row_weight"]), _p(o["x_perm"]),

@@ -58,8 +58,9 @@ extern "C" moe_status moe_dispatch_noalloc(const MoEConfig *cfg, int T, const in
   if (need == 0) return MOE_ERR_INVALID_ARG;
   if ((long long)T * cfg->top_k > INT_MAX / 2) return MOE_ERR_UNSUPPORTED;
   if (!expert_counts || !expert_offsets) return MOE_ERR_INVALID_ARG;
-  if (T > 0 && (!topk_idx || !topk_w || !x || !slot_row || !row_token || !row_weight || !x_perm ||
-                ((uintptr_t)x & 15u) || ((uintptr_t)x_perm & 15u)))
+  // x_perm == NULL builds the row maps only, and x may then be NULL too
+  if (T > 0 && (!topk_idx || !topk_w || !slot_row || !row_token || !row_weight ||
+                (x_perm && (!x || ((uintptr_t)x & 15u) || ((uintptr_t)x_perm & 15u)))))
     return MOE_ERR_INVALID_ARG;
   if ((long long)num_chunks(T) * cfg->num_experts > kNoAllocScratchInts) return MOE_ERR_UNSUPPORTED;
   int32_t *scratch = scratch_on_current_device();

@@ -47,13 +47,31 @@ def test_noalloc_dispatch_matches_workspace_dispatch_twice():
             if k in ("row_token", "row_weight", "x_perm"):
                 a, b = a[:R], b[:R]
             assert torch.equal(a, b), k
+        # the maps-only form (no x_perm), as with the workspace entry point
+        maps = B.dispatch_noalloc(cfg, x, idx, w, gather=False)
+        torch.cuda.synchronize()
+        assert maps["x_perm"] is None
+        for k in KEYS[:-1]:
+            a, b = ref[k], maps[k]
+            if k in ("row_token", "row_weight"):
+                a, b = a[:R], b[:R]
+            assert torch.equal(a, b), k
+
+
+def _host_library():
+    # the size check runs on the host: no GPU needed, only the built library
+    try:
+        from mixture_experts_layer_sqrt_b200 import build
+        build.build()
+        from mixture_experts_layer_sqrt_b200 import binding
+    except (RuntimeError, OSError) as e:
+        pytest.skip(f"native library unavailable here: {e}")
+    return binding
 
 
 def test_noalloc_dispatch_rejects_oversize():
     # rejected on the host before any CUDA call: 257 chunks x 1024 experts > 262144 ints
-    from mixture_experts_layer_sqrt_b200 import build
-    build.build()
-    from mixture_experts_layer_sqrt_b200 import binding as B
+    B = _host_library()
     cfg = B.make_config(E=1024, k=2, D=512, F=384)
     T = 256 * 257
     st = B.lib.moe_dispatch_noalloc(ctypes.byref(cfg), T, 16, 16, 16, 16, 16, 16, 16, 16, 16, None)
