@@ -140,18 +140,66 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def oracle_sample(p, arrays, n_tokens: int, seed: int):
-    """The float64 oracle on a bounded sample: routing and dispatch of every
-    token (capacity needs them), the expert FFN and combine for n_tokens."""
+def oracle_pass(p, arrays, n_tokens: int, seed: int):
+    """One bounded pass of the float64 oracle, in two timed parts:
+    route + dispatch of every token (capacity needs them all), then the expert
+    FFN + combine of n_tokens sampled tokens (each touched expert's weights
+    decoded once, then its rows multiplied).  Returns (route_dispatch_s, ffn_s,
+    rows kept after capacity)."""
     import oracle.moe_oracle as O
     L = O.StoredLayer(arrays, p.act, p.wdtype)
     t0 = time.perf_counter()
-    logits = O.router_logits(L.x(), L.w_router())
+    x = L.x()
+    logits = O.router_logits(x, L.w_router())
     idx, w, _ = O.route(logits, p.k, p.gate, arrays.get("bias"), arrays.get("bias_vl"), arrays.get("image_mask"))
     C = O.expert_capacity(p.T, p.k, p.E, p.capacity_factor)
-    toks = np.random.default_rng(seed).choice(p.T, size=n_tokens, replace=False)
-    O.moe_forward(L.x(), logits, idx, w, L.expert, p.E, C, p.clamp, "preact", L.shared(), tokens=toks)
-    return time.perf_counter() - t0
+    d = O.dispatch(idx, p.E, C)
+    t1 = time.perf_counter()
+    toks = np.random.default_rng(seed).choice(p.T, size=min(n_tokens, p.T), replace=False)
+    O.moe_forward(x, logits, idx, w, L.expert, p.E, C, p.clamp, "preact", L.shared(), tokens=toks)
+    t2 = time.perf_counter()
+    return t1 - t0, t2 - t1, int(d["offsets"][-1])
+
+
+def extrapolate_ffn(samples):
+    """Fit ffn_s = fixed + per_token * n over (n, ffn_s) samples of two or more
+    sizes (least squares).  The fixed part is the weight decoding, paid once
+    per touched expert whatever the sample size; per_token is the marginal
+    matmul cost.  Falls back to a line through the origin (the largest
+    sample's rate) when the fit is not increasing."""
+    n = np.array([s[0] for s in samples], dtype=np.float64)
+    t = np.array([s[1] for s in samples], dtype=np.float64)
+    if len(set(n.tolist())) >= 2:
+        b, a = np.polyfit(n, t, 1)
+        if b > 0 and a >= 0:
+            return float(a), float(b)
+    i = int(np.argmax(n))
+    return 0.0, float(t[i] / n[i])
+
+
+def cpu_core_counts():
+    """(nproc: the host's usable cores, threads: the BLAS threads the oracle's matmuls use)."""
+    try:
+        nproc = len(os.sched_getaffinity(0))
+    except AttributeError:
+        nproc = os.cpu_count() or 1
+    return nproc, blas_threads()
+
+
+def oracle_summary(p, rd_s: float, samples, kind_note: str):
+    """The oracle's whole-layer rate for all T tokens, extrapolated from the
+    timed samples: T / (route_dispatch_s + fixed + per_token * T)."""
+    fixed, per_tok = extrapolate_ffn(samples)
+    layer_s = rd_s + fixed + per_tok * p.T
+    nproc, threads = cpu_core_counts()
+    sizes = sorted({int(n) for n, _ in samples})
+    return {"value": p.T / layer_s, "unit": "tokens/s", "cores": threads, "nproc": nproc, "threads": threads,
+            "kind": "oracle", "extrapolated": True, "route_dispatch_s": rd_s,
+            "ffn_s_per_token": per_tok, "ffn_fixed_s": fixed, "layer_s": layer_s,
+            "ffn_samples": [[int(n), float(t)] for n, t in samples],
+            "sample": (f"float64 numpy oracle ({kind_note}): route + dispatch of all {p.T} tokens timed alone; "
+                       f"expert FFN + combine timed on seeded samples of {sizes} tokens, fitted as fixed "
+                       f"(weight decoding) + per-token cost and extrapolated to {p.T} tokens")}
 
 
 # ------------------------------------------------------------ ranks (host)
@@ -314,6 +362,13 @@ def gate_up_kernel(p, peaks):
     return (name, "tensor", peaks["bf16"], peaks["bf16_sustained"], f"bf16_tflops (burst) of {peaks['src']}")
 
 
+def workload_config(p, world: int, rows: int):
+    """The `config` object of both arms' JSON lines."""
+    return {"workload": describe(p), "tokens_per_gpu": p.T, "rows_after_capacity": rows, "out_dtype": "f32",
+            "parallelism": f"dp{world} (independent token batches, replicated weights)",
+            "l2": "inputs larger than L2: expert weights %.2f GB streamed every step" % (layer_bytes(p) / 1e9)}
+
+
 def report(args, p, world, rows, value, ms, per_step, gemm_ms, e2e, n_launch, clocks):
     peaks = load_peaks()
     flops = layer_flops(p, rows)
@@ -329,10 +384,7 @@ def report(args, p, world, rows, value, ms, per_step, gemm_ms, e2e, n_launch, cl
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32" if p.act == "f32" else "bf16", "data": "synthetic",
-        "config": {"workload": describe(p), "tokens_per_gpu": p.T, "rows_after_capacity": rows,
-                   "out_dtype": "f32",
-                   "parallelism": f"dp{world} (independent token batches, replicated weights)",
-                   "l2": "inputs larger than L2: expert weights %.2f GB streamed every step" % (layer_bytes(p) / 1e9)},
+        "config": workload_config(p, world, rows),
         "latency_ms": {"p50": float(np.percentile(per_step, 50)), "p95": float(np.percentile(per_step, 95)),
                        "p99": float(np.percentile(per_step, 99))},
         "layer_roofline": {"ideal_ms": ideal_ms, "frac": ideal_ms / ms, "frac_vs_sustained": ideal_sus_ms / ms,
@@ -354,32 +406,46 @@ def report(args, p, world, rows, value, ms, per_step, gemm_ms, e2e, n_launch, cl
     return res
 
 
-def cpu_baseline_leg(p, n_tokens=8):
+def cpu_baseline_leg(p, sizes=(64, 256)):
+    """The oracle as it stands on a bounded sample of the bench workload
+    (about 10-30 s of CPU work), reported beside the GPU number."""
     from mixture_experts_layer_sqrt_b200 import synth
     arrays = synth.generate(p)
-    el = oracle_sample(p, arrays, n_tokens, seed=1)
-    return {"value": n_tokens / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"float64 numpy oracle: route + dispatch of all {p.T} tokens, expert FFN + combine "
-                      f"for {n_tokens} sampled tokens, {el:.1f} s"}
+    samples, rd = [], []
+    for i, n in enumerate(sizes):
+        r, f, _ = oracle_pass(p, arrays, n, seed=1 + i)
+        rd.append(r)
+        samples.append((n, f))
+    return oracle_summary(p, float(np.mean(rd)), samples, "cpu_baseline")
 
 
 def run_reference(args, p):
+    """The reference arm: the float64 oracle on the host cores, each step a
+    bounded sample of the workload (route + dispatch of all T tokens, FFN +
+    combine of a few sampled tokens; steps alternate two sample sizes).  The
+    line's value is the oracle's whole-layer rate for all T tokens,
+    extrapolated from those steps."""
     from mixture_experts_layer_sqrt_b200 import synth
     arrays = synth.generate(p)
-    n_tok = 4
+    sizes = (16, 96)
     for i in range(args.warmup):
-        oracle_sample(p, arrays, n_tok, seed=100 + i)
-    times = [oracle_sample(p, arrays, n_tok, seed=i) for i in range(args.steps)]
-    ms = 1e3 * sum(times) / len(times)
-    value = n_tok / (ms / 1e3)
-    sample = (f"float64 numpy oracle per step: route + dispatch of all {p.T} tokens, expert FFN + combine "
-              f"for {n_tok} sampled tokens")
+        oracle_pass(p, arrays, sizes[0], seed=100 + i)
+    samples, rd, step_s, rows = [], [], [], 0
+    for i in range(args.steps):
+        n = sizes[i % 2]
+        t0 = time.perf_counter()
+        r, f, rows = oracle_pass(p, arrays, n, seed=i)
+        step_s.append(time.perf_counter() - t0)
+        rd.append(r)
+        samples.append((n, f))
+    cb = oracle_summary(p, float(np.mean(rd)), samples, "--impl reference")
+    value = cb["value"]
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": describe(p), "tokens_per_step": n_tok},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                             "sample": sample},
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["layer_s"] * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(p, 1, rows),
+            "sample_ms_per_step": 1e3 * float(np.mean(step_s)),
+            "cpu_baseline": cb,
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 

@@ -50,3 +50,41 @@ def test_traffic_records_follow_their_kernel_sources(monkeypatch):
     changed = dict(bench.TRAFFIC_SOURCES, gate_up_sqrt_fp4=("gemm_fp4.cu", "api.cu"))
     monkeypatch.setattr(bench, "TRAFFIC_SOURCES", changed)
     assert bench.profiled_traffic("gate_up_sqrt_fp4") is None
+
+
+def test_extrapolation_arithmetic():
+    # ffn_s = 2 + 0.01 n exactly: the fit recovers both parts
+    a, b = bench.extrapolate_ffn([(64, 2.64), (256, 4.56), (64, 2.64)])
+    assert a == pytest.approx(2.0) and b == pytest.approx(0.01)
+    # a decreasing fit falls back to the largest sample's rate through the origin
+    a, b = bench.extrapolate_ffn([(64, 3.0), (256, 2.0)])
+    assert a == 0.0 and b == pytest.approx(2.0 / 256)
+    # one size only: linear through the origin
+    a, b = bench.extrapolate_ffn([(32, 1.6)])
+    assert a == 0.0 and b == pytest.approx(0.05)
+
+
+def test_cpu_baseline_fields_small_workload():
+    p = synth.PROBLEMS["mixtral_bf16"].with_(name="cb", T=96, D=128, F=64, E=4)
+    cb = bench.cpu_baseline_leg(p, sizes=(8, 32))
+    for k in ("value", "unit", "cores", "nproc", "threads", "kind", "extrapolated", "route_dispatch_s",
+              "ffn_s_per_token", "ffn_fixed_s", "sample"):
+        assert k in cb, k
+    assert cb["kind"] == "oracle" and cb["extrapolated"] is True and cb["unit"] == "tokens/s"
+    assert cb["nproc"] >= 1 and cb["threads"] >= 1 and cb["cores"] == cb["threads"]
+    layer_s = cb["route_dispatch_s"] + cb["ffn_fixed_s"] + cb["ffn_s_per_token"] * p.T
+    assert cb["value"] == pytest.approx(p.T / layer_s)
+
+
+def test_reference_arm_line_small_workload():
+    p = synth.PROBLEMS["capacity_bf16"].with_(name="ref", T=128, D=128, F=64, E=4)
+    args = argparse.Namespace(steps=4, warmup=3)
+    res = bench.run_reference(args, p)
+    for k in KEYS:
+        if k not in ("roofline", "gpu_launches", "clocks"):
+            assert k in res, k
+    assert res["impl"] == "reference" and res["dtype"] == "f64"
+    assert res["cpu_baseline"]["value"] == res["value"]
+    assert res["e2e"]["value"] == res["value"] and res["e2e"]["h2d_bytes_per_step"] == 0
+    assert res["config"] == bench.workload_config(p, 1, res["config"]["rows_after_capacity"])
+    assert 0 < res["config"]["rows_after_capacity"] <= p.T * p.k
