@@ -83,9 +83,8 @@ def gemm_sources_sha(files=TRAFFIC_SOURCES["gate_up_mixtral_bf16"]) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel_key: str):
+def profiled_traffic(kernel_key: str, path: str = os.path.join(ROOT, "profiles", "traffic.txt")):
     """DRAM bytes per launch recorded from an ncu capture, if the kernel's sources are unchanged since."""
-    path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path) or kernel_key not in TRAFFIC_SOURCES:
         return None
     want = gemm_sources_sha(TRAFFIC_SOURCES[kernel_key])
@@ -258,7 +257,7 @@ def run_ours(args, p, rank, world, local_rank):
 
     # one step = one moe_forward call (the product's own entry point); with
     # events it records them on the stream at the stage boundaries:
-    # 0 | route | 1 | dispatch | 2 | gate/up | 3 | down | 4 | shared | 5 | combine | 6
+    # 0 | route | 1 | dispatch maps | 2 | gather | 3 | gate/up | 4 | down | 5 | shared | 6 | combine | 7
     def step(ev=None):
         if ev is None:
             B.forward(cfg, x, w, ws_f, mask, out)
@@ -299,7 +298,7 @@ def run_ours(args, p, rank, world, local_rank):
     clocks = sampler.stop() if sampler else None
     total_ms = step_ev[0].elapsed_time(step_ev[-1])
     per_step = [step_ev[i].elapsed_time(step_ev[i + 1]) for i in range(args.steps)]
-    names = ["route", "dispatch", "gate_up", "down", "shared", "combine"]
+    names = STAGES
     stage_ms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in g_ev) / args.steps for i, n in enumerate(names)}
     gemm_ms = stage_ms["gate_up"]
     B.check_device_status(ws_f)
@@ -313,6 +312,7 @@ def run_ours(args, p, rank, world, local_rank):
         return None
     res = report(args, p, world, rows, value, ms, per_step, gemm_ms, e2e, n_launch, clocks)
     res["stage_ms"] = stage_ms
+    res["permute_combine"] = permute_combine(p, rows, stage_ms, load_peaks())
     return res
 
 
@@ -346,6 +346,30 @@ def run_e2e(args, B, WL, cfg, wt, arrays, T, D, dev, stream, dist):
             "h2d_bytes_per_step": int(x_h.numel() * x_h.element_size() + (m_h.numel() if m_h is not None else 0)),
             "d2h_bytes_per_step": int(out_h[0].numel() * out_h[0].element_size()),
             "copies": "overlapped with compute on separate streams (forward_host_batches)"}
+
+
+# the stage intervals moe_forward_profiled brackets with its events
+STAGES = ["route", "dispatch_maps", "gather", "gate_up", "down", "shared", "combine"]
+
+
+def permute_combine(p, rows: int, stage_ms, peaks):
+    """Achieved HBM bandwidth of the two data-movement stages, from their
+    algorithmic bytes and their stage event times:
+      gather   reads each kept row's x row and writes it to x_perm: 2 rows D a
+               (+ a 4-byte row scale per row for the f16 rows of NVFP4 layers)
+      combine  reads every kept row of fp32 y_perm (and the fp32 shared-expert
+               row of every token) and writes the fp32 output row of every token"""
+    a = 4 if p.act == "f32" else 2
+    g_bytes = 2.0 * rows * p.D * a + (4.0 * rows if p.wdtype == "nvfp4" else 0.0)
+    c_bytes = 4.0 * rows * p.D + 4.0 * p.T * p.D * (2 if p.Fs else 1)
+    out = {}
+    for name, b in (("gather", g_bytes), ("combine", c_bytes)):
+        ms = stage_ms[name]
+        gbs = b / (ms / 1e3) / 1e9 if ms > 0 else None
+        out[name] = {"bytes": b, "ms": ms, "gbs": gbs, "frac": gbs / peaks["hbm"] if gbs else None}
+    out["peak_gbs"] = peaks["hbm"]
+    out["peak_kind"] = f"hbm_gbs of {peaks['src']}"
+    return out
 
 
 # fp32 layers run on the CUDA cores: 148 SMs x 128 fp32 lanes x 2 FLOP per FMA at the 1965 MHz maximum clock

@@ -287,13 +287,16 @@ moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeig
 /* moe_forward with stage timing hooks (for profilers and benchmarks).
  * events: n_events CUDA event handles (cudaEvent_t, created by the caller;
  * NULL entries are skipped), recorded on `stream` at the stage boundaries:
- *   [0] before routing, [1] after routing (a1-a2), [2] after dispatch (a3-a5),
- *   [3] after the expert gate/up GEMM (a6), [4] after the down GEMM (a7),
- *   [5] after the shared expert (a8), [6] after combine (a9).
+ *   [0] before routing, [1] after routing (a1-a2), [2] after the dispatch
+ *   maps (histogram, scan, row positions: a3-a4), [3] after the row gather
+ *   into x_perm (a5), [4] after the expert gate/up GEMM (a6), [5] after the
+ *   down GEMM (a7), [6] after the shared expert (a8), [7] after combine (a9).
+ * Each interval brackets exactly the kernels of its stage, so the elapsed
+ * time between events i and i+1 is that stage's device time.
  * n_events is 0 (then events may be NULL and this is moe_forward) or
  * MOE_STAGE_EVENTS; anything else is MOE_ERR_INVALID_ARG.  A failed event
  * record returns MOE_ERR_CUDA. */
-#define MOE_STAGE_EVENTS 7
+#define MOE_STAGE_EVENTS 8
 moe_status moe_forward_profiled(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
                                 const uint8_t *image_mask, void *out, int32_t *topk_idx_out,
                                 int32_t *expert_counts_out, void *ws, size_t ws_bytes, moe_stream_t stream,

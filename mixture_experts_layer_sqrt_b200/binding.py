@@ -301,7 +301,7 @@ def forward(cfg: MoEConfig, x: torch.Tensor, w: MoEWeights, ws: torch.Tensor, im
 
 
 STAGES = ("route", "dispatch", "gate_up", "down", "shared", "combine")
-STAGE_EVENTS = 7
+STAGE_EVENTS = 8
 
 
 def _event_handles(events):

@@ -129,27 +129,14 @@ moe_status run_down(const MoEConfig &c, int rows, const void *h, const int32_t *
   return launch_down_simt(cc, rows, h, offsets, wd, c.intermediate_dim, row_weight, y, s);
 }
 
-// The expert projections run as two tensor-core launches; MOE_EXPERTS_FUSED=1
-// selects the single persistent launch instead (same results, bit for bit).
-bool fused_requested() {
-  const char *e = getenv("MOE_EXPERTS_FUSED");
-  return e && e[0] == '1';
-}
-
-// Both expert projections: x_perm -> h -> y.  NVFP4 experts: the two
-// projections one after the other, each straight from the packed weights or
-// expanded first.  bf16 on the tensor-core path: two launches, or with
-// MOE_EXPERTS_FUSED=1 one persistent launch.  Otherwise the CUDA-core kernels.
+// Both expert projections: x_perm -> h -> y, as two launches (gate/up, then down).
 moe_status run_experts(const MoEConfig &c, int rows, const void *a, int a_rows, const int32_t *row_token,
                        const int32_t *offsets, const void *wg, const void *wu, const void *wd, const void *sg,
                        const void *su, const void *sd, const float *row_weight, void *h, void *y,
-                       const ExpertWs &ws, int *sched, cudaStream_t s) {
-  moe_status st;
-  if (c.expert_dtype == MOE_NVFP4 || !tc_shapes_ok(c, c.intermediate_dim) || !fused_requested() || row_token) {
-    if ((st = run_gate_up(c, rows, a, a_rows, row_token, offsets, wg, wu, sg, su, h, ws, s)) != MOE_OK) return st;
-    return run_down(c, rows, h, offsets, wd, sd, row_weight, y, ws, s);
-  }
-  return launch_experts_fused_tc(c, rows, a, offsets, wg, wu, wd, row_weight, h, (float *)y, ws.status, sched, s);
+                       const ExpertWs &ws, cudaStream_t s) {
+  moe_status st = run_gate_up(c, rows, a, a_rows, row_token, offsets, wg, wu, sg, su, h, ws, s);
+  if (st != MOE_OK) return st;
+  return run_down(c, rows, h, offsets, wd, sd, row_weight, y, ws, s);
 }
 
 // The shared expert viewed as a one-expert layer of width F_s in the act dtype.
@@ -165,7 +152,6 @@ MoEConfig shared_cfg(const MoEConfig &c) {
 // ---- whole-layer workspace
 struct ForwardWs {
   int *status;
-  int *sched;
   int32_t *topk_idx, *counts, *offsets, *slot_row, *row_token, *chunk_cnt;
   float *topk_w, *row_weight, *row_scale, *route_logits;
   void *x_perm, *h, *y_perm, *sh_y;
@@ -176,12 +162,6 @@ ForwardWs carve_forward(Carve &cv, const MoEConfig &c, int T) {
   const size_t Tk = (size_t)T * c.top_k, E = c.num_experts, D = c.hidden_dim;
   const size_t as = act_size(c);
   w.status = cv.take<int>(kStatusBytes / sizeof(int));
-  size_t ns = fused_sched_ints(c, (int)Tk, true);
-  if (c.shared_intermediate_dim) {
-    const size_t ns2 = fused_sched_ints(c, T, false);
-    if (ns2 > ns) ns = ns2;
-  }
-  w.sched = cv.take<int>(ns);
   w.topk_idx = cv.take<int32_t>(Tk);
   w.topk_w = cv.take<float>(Tk);
   w.counts = cv.take<int32_t>(E);
@@ -318,7 +298,6 @@ size_t moe_grouped_swiglu_workspace_size(const MoEConfig *cfg, int rows) {
   Carve cv(nullptr);
   carve_expert(cv, *cfg);
   cv.take<char>((size_t)rows * cfg->intermediate_dim * act_size(*cfg));
-  cv.take<int>(fused_sched_ints(*cfg, rows, true));
   return align_up(cv.off, 256);
 }
 
@@ -378,9 +357,8 @@ moe_status moe_grouped_swiglu(const MoEConfig *cfg, int rows, const void *x_perm
   Carve cv(ws);
   ExpertWs ew = carve_expert(cv, *cfg);
   void *h = cv.take<char>((size_t)rows * cfg->intermediate_dim * act_size(*cfg));
-  int *sched = cv.take<int>(fused_sched_ints(*cfg, rows, true));
   return run_experts(*cfg, rows, x_perm, rows, nullptr, expert_offsets, w->w_gate, w->w_up, w->w_down, w->s_gate,
-                     w->s_up, w->s_down, row_weight, h, y_perm, ew, sched, (cudaStream_t)stream);
+                     w->s_up, w->s_down, row_weight, h, y_perm, ew, (cudaStream_t)stream);
 }
 
 moe_status moe_combine(const MoEConfig *cfg, int T, const void *y_perm, const int32_t *slot_row,
@@ -441,42 +419,39 @@ static moe_status forward_impl(const MoEConfig *cfg, int T, const void *x, const
                          f.route_logits, s)) != MOE_OK)
     return st;
   if ((st = mark(1)) != MOE_OK) return st;
+  // the row maps (histogram, scan, positions), then the row gather
+  if ((st = launch_dispatch(c, T, idx, f.topk_w, x, counts, f.offsets, f.slot_row, f.row_token, f.row_weight,
+                            nullptr, f.chunk_cnt, s)) != MOE_OK)
+    return st;
+  if ((st = mark(2)) != MOE_OK) return st;
   // NVFP4 experts on the direct path: x_perm is gathered in f16 with a
   // power-of-two scale per row and the gate/up GEMM multiplies in f16
   const bool fp4_f16 = f.row_scale != nullptr;
-  if ((st = launch_dispatch(c, T, idx, f.topk_w, x, counts, f.offsets, f.slot_row, f.row_token,
-                            f.row_weight, fp4_f16 ? nullptr : f.x_perm, f.chunk_cnt, s)) != MOE_OK)
-    return st;
-  if (fp4_f16 && (st = launch_gather_f16(c, T, f.offsets, f.row_token, x, f.x_perm, f.row_scale, s)) != MOE_OK)
-    return st;
-  if ((st = mark(2)) != MOE_OK) return st;
-  if (fp4_f16 || events) {
-    // the two projections as separate launches (the stage boundary between them is observable)
-    if (fp4_f16) {
-      st = launch_gate_up_fp4(c, rows, f.x_perm, rows, nullptr, f.offsets, w->w_gate, w->w_up, w->s_gate, w->s_up,
-                              f.row_scale, f.h, f.ex.status, s);
-    } else {
-      st = run_gate_up(c, rows, f.x_perm, rows, nullptr, f.offsets, w->w_gate, w->w_up, w->s_gate, w->s_up, f.h,
-                       f.ex, s);
-    }
-    if (st != MOE_OK) return st;
-    if ((st = mark(3)) != MOE_OK) return st;
-    if ((st = run_down(c, rows, f.h, f.offsets, w->w_down, w->s_down, f.row_weight, f.y_perm, f.ex, s)) != MOE_OK)
-      return st;
-  } else if ((st = run_experts(c, rows, f.x_perm, rows, nullptr, f.offsets, w->w_gate, w->w_up, w->w_down, w->s_gate,
-                        w->s_up, w->s_down, f.row_weight, f.h, f.y_perm, f.ex, f.sched, s)) != MOE_OK) {
-    return st;
+  if (fp4_f16) st = launch_gather_f16(c, T, f.offsets, f.row_token, x, f.x_perm, f.row_scale, s);
+  else st = launch_gather(c, T, f.offsets, f.row_token, x, f.x_perm, s);
+  if (st != MOE_OK) return st;
+  if ((st = mark(3)) != MOE_OK) return st;
+  if (fp4_f16) {
+    st = launch_gate_up_fp4(c, rows, f.x_perm, rows, nullptr, f.offsets, w->w_gate, w->w_up, w->s_gate, w->s_up,
+                            f.row_scale, f.h, f.ex.status, s);
+  } else {
+    st = run_gate_up(c, rows, f.x_perm, rows, nullptr, f.offsets, w->w_gate, w->w_up, w->s_gate, w->s_up, f.h,
+                     f.ex, s);
   }
+  if (st != MOE_OK) return st;
   if ((st = mark(4)) != MOE_OK) return st;
+  if ((st = run_down(c, rows, f.h, f.offsets, w->w_down, w->s_down, f.row_weight, f.y_perm, f.ex, s)) != MOE_OK)
+    return st;
+  if ((st = mark(5)) != MOE_OK) return st;
   if (c.shared_intermediate_dim) {
     const MoEConfig sc = shared_cfg(c);
     if ((st = run_experts(sc, T, x, T, nullptr, nullptr, w->sh_gate, w->sh_up, w->sh_down, nullptr, nullptr,
-                          nullptr, nullptr, f.h, f.sh_y, f.ex, f.sched, s)) != MOE_OK)
+                          nullptr, nullptr, f.h, f.sh_y, f.ex, s)) != MOE_OK)
       return st;
   }
-  if ((st = mark(5)) != MOE_OK) return st;
+  if ((st = mark(6)) != MOE_OK) return st;
   if ((st = launch_combine(c, T, f.y_perm, f.slot_row, f.sh_y, out, s)) != MOE_OK) return st;
-  return mark(6);
+  return mark(7);
 }
 
 moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,

@@ -6,57 +6,81 @@
 //   out[t] = sum_{j=0..k-1, slot kept} y_perm[slot_row[t, j]]  (+ shared_y[t])
 // summed in fp32 in that fixed order: deterministic, no atomics.
 //
-// One warp per token row, 16-byte vector loads of the fp32 expert outputs: a
-// pure HBM stream of k (+1 shared) rows read and one row written per token.
+// One warp per token row, 16-byte streaming loads of the fp32 expert outputs:
+// a pure HBM stream of k (+1 shared) rows read and one row written per token.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace moe {
 namespace {
 
-template <typename TOut>
-__global__ void __launch_bounds__(256) combine_kernel(int T, int D, int k,
-                                                      const float *__restrict__ y_perm,
-                                                      const int32_t *__restrict__ slot_row,
-                                                      const float *__restrict__ shared_y,
-                                                      TOut *__restrict__ out) {
+constexpr int kCombineThreads = 128;  // small blocks: every SM holds 16, so the last wave is even
+
+// Streaming (evict-first) 16-byte load and store: y_perm and out are touched once.
+__device__ __forceinline__ float4 ld_stream(const float *p) { return __ldcs(reinterpret_cast<const float4 *>(p)); }
+__device__ __forceinline__ void st_stream(float *p, float4 v) { __stcs(reinterpret_cast<float4 *>(p), v); }
+
+// kK > 0: the layer's top-k fixed at compile time (rows held in registers, the
+// column loop unrolled with every row's load in flight); kK == 0: any k <= 16.
+template <typename TOut, int kK>
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(int T, int D, int k_rt,
+                                                                  const float *__restrict__ y_perm,
+                                                                  const int32_t *__restrict__ slot_row,
+                                                                  const float *__restrict__ shared_y,
+                                                                  TOut *__restrict__ out) {
   constexpr int V = 4;  // four fp32 per 16-byte load
+  constexpr int kMaxK = kK > 0 ? kK : 16;
+  const int k = kK > 0 ? kK : k_rt;
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (blockDim.x >> 5);
   for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
-    int rows[16];
+    // the token's k rows: lane j < k loads slot j, then every lane gets all of them
+    const int my_row = lane < k ? slot_row[(long)t * k + lane] : -1;
+    int rows[kMaxK];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) rows[j] = j < k ? slot_row[(long)t * k + j] : -1;
-#pragma unroll 4
+    for (int j = 0; j < kMaxK; ++j) rows[j] = __shfl_sync(0xffffffffu, my_row, j);
+#pragma unroll(kK > 0 && kK <= 4 ? 4 : 1)
     for (int c = lane * V; c < D; c += 32 * V) {
-      float acc[V];
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
-      for (int v = 0; v < V; ++v) acc[v] = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
+      for (int j = 0; j < kMaxK; ++j) {
         if (j < k && rows[j] >= 0) {
-          Vec16<float> y = load16(y_perm + (long)rows[j] * D + c);
-#pragma unroll
-          for (int v = 0; v < V; ++v) acc[v] += y.get(v);
+          const float4 y = ld_stream(y_perm + (long)rows[j] * D + c);
+          acc.x += y.x;
+          acc.y += y.y;
+          acc.z += y.z;
+          acc.w += y.w;
         }
       }
       if (shared_y) {
-        Vec16<float> y = load16(shared_y + (long)t * D + c);
-#pragma unroll
-        for (int v = 0; v < V; ++v) acc[v] += y.get(v);
+        const float4 y = ld_stream(shared_y + (long)t * D + c);
+        acc.x += y.x;
+        acc.y += y.y;
+        acc.z += y.z;
+        acc.w += y.w;
       }
       if constexpr (sizeof(TOut) == 4) {
-        Vec16<float> o;
-#pragma unroll
-        for (int v = 0; v < V; ++v) o.set(v, acc[v]);
-        store16((float *)out + (long)t * D + c, o);
+        st_stream((float *)out + (long)t * D + c, acc);
       } else {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
         uint2 o = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
         *reinterpret_cast<uint2 *>((__nv_bfloat16 *)out + (long)t * D + c) = o;
       }
     }
+  }
+}
+
+template <typename TOut>
+void launch_combine_k(int k, int blocks, int T, int D, const float *y, const int32_t *slot_row, const float *sh,
+                      TOut *out, cudaStream_t s) {
+  switch (k) {
+    case 1: combine_kernel<TOut, 1><<<blocks, kCombineThreads, 0, s>>>(T, D, k, y, slot_row, sh, out); break;
+    case 2: combine_kernel<TOut, 2><<<blocks, kCombineThreads, 0, s>>>(T, D, k, y, slot_row, sh, out); break;
+    case 4: combine_kernel<TOut, 4><<<blocks, kCombineThreads, 0, s>>>(T, D, k, y, slot_row, sh, out); break;
+    case 6: combine_kernel<TOut, 6><<<blocks, kCombineThreads, 0, s>>>(T, D, k, y, slot_row, sh, out); break;
+    case 8: combine_kernel<TOut, 8><<<blocks, kCombineThreads, 0, s>>>(T, D, k, y, slot_row, sh, out); break;
+    default: combine_kernel<TOut, 0><<<blocks, kCombineThreads, 0, s>>>(T, D, k, y, slot_row, sh, out); break;
   }
 }
 
@@ -68,16 +92,15 @@ moe_status launch_combine(const MoEConfig &c, int T, const void *y_perm, const i
   int dev = 0, sms = 148;
   MOE_CUDA_TRY(cudaGetDevice(&dev));
   MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  int blocks = (T + 7) / 8;
+  constexpr int kWarpsPerBlock = kCombineThreads / 32;
+  int blocks = (T + kWarpsPerBlock - 1) / kWarpsPerBlock;
   if (blocks > sms * 16) blocks = sms * 16;
   if (c.out_dtype == MOE_F32)
-    combine_kernel<float><<<blocks, 256, 0, s>>>(T, c.hidden_dim, c.top_k, (const float *)y_perm,
-                                                 slot_row, (const float *)shared_y, (float *)out);
+    launch_combine_k<float>(c.top_k, blocks, T, c.hidden_dim, (const float *)y_perm, slot_row,
+                            (const float *)shared_y, (float *)out, s);
   else
-    combine_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(T, c.hidden_dim, c.top_k,
-                                                         (const float *)y_perm, slot_row,
-                                                         (const float *)shared_y,
-                                                         (__nv_bfloat16 *)out);
+    launch_combine_k<__nv_bfloat16>(c.top_k, blocks, T, c.hidden_dim, (const float *)y_perm, slot_row,
+                                    (const float *)shared_y, (__nv_bfloat16 *)out, s);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }

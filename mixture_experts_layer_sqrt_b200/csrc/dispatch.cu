@@ -5,11 +5,13 @@
 // to expert e; Gather") and 坑一 (tokens beyond the expert capacity are
 // dropped); Echo MoE quick reference, "Dispatch".
 //
-// Four kernels, no global atomics:
+// Four kernels, no atomics:
 //   hist    one block per chunk of kChunkTokens tokens: per-chunk expert counts
-//           (shared-memory counters) -> chunk_cnt[c][e]
-//   scan    one block: per expert, exclusive scan of chunk_cnt over chunks
-//           (in place), total count, kept = min(count, C), offsets = prefix of kept
+//           (warp match groups into per-warp counter rows, then summed over
+//           the warps) -> chunk_cnt[c][e]
+//   scan    one block: per expert (a warp each), exclusive scan of chunk_cnt
+//           over chunks (in place), total count, kept = min(count, C);
+//           offsets = prefix of kept
 //   maps    one block per chunk: the rank of each assignment among its
 //           expert's assignments in token order (warp match + per-warp
 //           running counters), -> slot_row, row_token, row_weight
@@ -24,20 +26,39 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 static_assert(kChunkTokens == kWarps * 32, "one warp per 32 tokens of a chunk");
 
+// Per-warp expert counts of the warp's 32 tokens (32 * k assignments): each
+// round the lanes holding the same expert form a peer group
+// (__match_any_sync) and the group's lowest lane adds the group's size to the
+// warp's own counter row.  A row belongs to one warp and each round's leaders
+// hold distinct experts, so no two lanes ever update one counter at once.
+__device__ __forceinline__ void warp_expert_counts(long a0, long a_end, int E, int k,
+                                                   const int32_t *__restrict__ topk_idx, int32_t *my, int lane) {
+  for (long a = a0; a < a0 + 32L * k; a += 32) {
+    long ai = a + lane;
+    int e = ai < a_end ? topk_idx[ai] : -1;
+    if (e >= E) e = -1;
+    unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && (__ffs(peers) - 1) == lane) my[e] += __popc(peers);
+    __syncwarp();
+  }
+}
+
 __global__ void __launch_bounds__(kThreads) hist_kernel(int T, int E, int k,
                                                         const int32_t *__restrict__ topk_idx,
                                                         int32_t *__restrict__ chunk_cnt) {
-  extern __shared__ int32_t cnt[];  // [E]
-  for (int e = threadIdx.x; e < E; e += kThreads) cnt[e] = 0;
+  extern __shared__ int32_t cnt[];  // [kWarps][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kWarps * E; i += kThreads) cnt[i] = 0;
   __syncthreads();
-  const long a0 = (long)blockIdx.x * kChunkTokens * k;
-  const long a1 = min((long)T * k, a0 + (long)kChunkTokens * k);
-  for (long a = a0 + threadIdx.x; a < a1; a += kThreads) {
-    int e = topk_idx[a];
-    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+  const long a0 = ((long)blockIdx.x * kChunkTokens + warp * 32) * k;
+  warp_expert_counts(a0, min((long)T * k, a0 + 32L * k), E, k, topk_idx, cnt + warp * E, lane);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kThreads) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) c += cnt[w * E + e];
+    chunk_cnt[(long)blockIdx.x * E + e] = c;
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += kThreads) chunk_cnt[(long)blockIdx.x * E + e] = cnt[e];
 }
 
 // Block-wide exclusive scan of one int per thread (1024 threads).
@@ -69,25 +90,42 @@ __device__ int block_exclusive_scan(int v, int *warp_sums, int &total) {
   return r;
 }
 
+// Per expert: exclusive scan of its chunk counts over the chunks (in place:
+// chunk c's entry becomes the number of e's assignments in chunks < c), the
+// total count, kept = min(count, C); then offsets = exclusive prefix of kept.
+// One warp per expert walks the chunks 32 at a time (independent loads, a
+// warp scan each); one block of 1024 threads.
 __global__ void __launch_bounds__(1024) scan_kernel(int n_chunks, int E, int capacity,
                                                     int32_t *__restrict__ chunk_cnt,
                                                     int32_t *__restrict__ expert_counts,
                                                     int32_t *__restrict__ expert_offsets) {
   __shared__ int warp_sums[33];
+  extern __shared__ int kept_s[];  // [E]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int e = warp; e < E; e += 32) {
+    int run = 0;
+    for (int c0 = 0; c0 < n_chunks; c0 += 32) {
+      const int c = c0 + lane;
+      const int v = c < n_chunks ? chunk_cnt[(long)c * E + e] : 0;
+      int incl = v;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        int n = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += n;
+      }
+      if (c < n_chunks) chunk_cnt[(long)c * E + e] = run + incl - v;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      expert_counts[e] = run;
+      kept_s[e] = (capacity > 0 && run > capacity) ? capacity : run;
+    }
+  }
+  __syncthreads();
   int carry = 0;
   for (int e0 = 0; e0 < E; e0 += 1024) {
     const int e = e0 + threadIdx.x;
-    int kept = 0;
-    if (e < E) {
-      int run = 0;
-      for (int c = 0; c < n_chunks; ++c) {
-        int v = chunk_cnt[(long)c * E + e];
-        chunk_cnt[(long)c * E + e] = run;  // exclusive base of chunk c within expert e
-        run += v;
-      }
-      expert_counts[e] = run;
-      kept = (capacity > 0 && run > capacity) ? capacity : run;
-    }
+    const int kept = e < E ? kept_s[e] : 0;
     int total;
     int off = block_exclusive_scan(kept, warp_sums, total);
     if (e < E) expert_offsets[e] = carry + off;
@@ -115,14 +153,7 @@ __global__ void __launch_bounds__(kThreads) maps_kernel(int T, int E, int k, int
   const long a0 = tw * k;
   const long a_end = min((long)T * k, a0 + 32L * k);
   // pass 1: per-warp counts per expert
-  for (long a = a0; a < a0 + 32L * k; a += 32) {
-    long ai = a + lane;
-    int e = ai < a_end ? topk_idx[ai] : -1;
-    if (e >= E) e = -1;
-    unsigned peers = __match_any_sync(0xffffffffu, e);
-    if (e >= 0 && (__ffs(peers) - 1) == lane) my[e] += __popc(peers);
-    __syncwarp();
-  }
+  warp_expert_counts(a0, a_end, E, k, topk_idx, my, lane);
   __syncthreads();
   // warps' bases: chunk base + counts of the lower warps of this chunk
   for (int e = threadIdx.x; e < E; e += kThreads) {
@@ -255,20 +286,27 @@ moe_status launch_dispatch(const MoEConfig &c, int T, const int32_t *topk_idx, c
     MOE_CUDA_TRY(cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), s));
     return MOE_OK;
   }
-  hist_kernel<<<nch, kThreads, E * sizeof(int32_t), s>>>(T, E, k, topk_idx, chunk_cnt);
+  const size_t warp_rows_smem = (size_t)kWarps * E * sizeof(int32_t);  // <= 32 KB (E <= 1024)
+  hist_kernel<<<nch, kThreads, warp_rows_smem, s>>>(T, E, k, topk_idx, chunk_cnt);
   MOE_LAUNCH_CHECK();
-  scan_kernel<<<1, 1024, 0, s>>>(nch, E, c.expert_capacity, chunk_cnt, expert_counts, expert_offsets);
+  scan_kernel<<<1, 1024, E * sizeof(int32_t), s>>>(nch, E, c.expert_capacity, chunk_cnt, expert_counts,
+                                                   expert_offsets);
   MOE_LAUNCH_CHECK();
-  size_t maps_smem = (size_t)kWarps * E * sizeof(int32_t);
-  MOE_CUDA_TRY(cudaFuncSetAttribute(maps_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)maps_smem));
+  const size_t maps_smem = warp_rows_smem;
   maps_kernel<<<nch, kThreads, maps_smem, s>>>(T, E, k, c.expert_capacity, topk_idx, topk_w, chunk_cnt,
                                                expert_offsets, slot_row, row_token, row_weight);
   MOE_LAUNCH_CHECK();
   if (!x_perm) return MOE_OK;  // maps only: the GEMM gathers the rows itself
+  return launch_gather(c, T, expert_offsets, row_token, x, x_perm, s);
+}
+
+moe_status launch_gather(const MoEConfig &c, int T, const int32_t *expert_offsets, const int32_t *row_token,
+                         const void *x, void *x_perm, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
   int dev = 0, sms = 148;
   MOE_CUDA_TRY(cudaGetDevice(&dev));
   MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  const int max_rows = T * k;
+  const int max_rows = T * c.top_k, E = c.num_experts;
   if (c.act_dtype == MOE_F32) {
     gather_kernel<float><<<sms * 8, 256, 0, s>>>(max_rows, c.hidden_dim, expert_offsets, E, row_token,
                                                  (const float *)x, (float *)x_perm);

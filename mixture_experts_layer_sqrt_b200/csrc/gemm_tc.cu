@@ -41,7 +41,6 @@
 // CTAs of a pair) and every role winds down (copies and MMAs drained, TMEM
 // freed) instead of hanging.
 #include <cudaTypedefs.h>
-#include <stdlib.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -450,393 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 
-// ==========================================================================
-// Fused gate/up + down: one persistent launch for both expert projections
-// (opt-in: MOE_EXPERTS_FUSED=1).  Measured on the Mixtral-shaped layer under
-// the power cap it is ~2% slower than two separate launches: the wave tail it
-// removes from the down pass is smaller than its per-tile overheads.
-//
-// Tiles are claimed dynamically from a global counter: first every gate/up
-// tile (expert-major, n-block, m-block), then every down tile.  A down tile of
-// (expert e, m-block i) reads the rows of h written by the F/128 gate/up tiles
-// of (e, i); their epilogues bump a per-m-block counter after the h stores
-// (proxy fence + release), and the producer of the down tile waits (bounded)
-// for the count before its TMA loads.  Claims are ordered, so every tile that
-// is waited on is already owned by a running CTA: no deadlock, whatever the
-// residency.  The tail of the gate/up pass overlaps the start of the down pass
-// and the down pass has no wave boundary of its own.
-// ==========================================================================
-constexpr int kRing = 4;
-
-struct SmemF {
-  uint64_t full[4];
-  uint64_t empty[4];
-  uint64_t tmem_full[2];
-  uint64_t tmem_empty[2];
-  uint64_t h_done[2];
-  uint64_t drain;
-  uint64_t ring_full[kRing];
-  uint64_t ring_empty[kRing];
-  int ring_tile[kRing];
-  uint32_t tmem_base;
-  int abort;
-  int m_prefix[MAX_E + 1];   // per-expert prefix of 128-row m-tiles
-};
-
-struct FusedParams {
-  int rows, D, F, E;
-  int n1, n2;                // n-tiles of gate/up (F / 128) and of down (D / 256)
-  const int32_t *offsets;    // [E+1] or null: one group of `rows` rows
-  __nv_bfloat16 *h;          // [rows, F]
-  float *y;                  // [rows, D]
-  const float *row_weight;   // nullable
-  float clamp;
-  int clamp_mode;
-  int *status;
-  int *sched;                // [0] next tile; [1 + m-tile] finished gate/up tiles (zeroed per launch)
-};
-
-struct FTile {
-  int phase, e, gm, m0, end, n_blk;
-};
-
-__device__ __forceinline__ int fseg_begin(const FusedParams &p, int e) { return p.offsets ? p.offsets[e] : 0; }
-__device__ __forceinline__ int fseg_end(const FusedParams &p, int e) {
-  int v = p.offsets ? p.offsets[e + 1] : p.rows;
-  return v < p.rows ? v : p.rows;
-}
-
-__device__ __forceinline__ FTile decode_fused(const FusedParams &p, const SmemF &sm, int t) {
-  const int total1 = sm.m_prefix[p.E] * p.n1;
-  FTile r;
-  r.phase = t < total1 ? 1 : 2;
-  const int n = r.phase == 1 ? p.n1 : p.n2;
-  if (r.phase == 2) t -= total1;
-  int lo = 0, hi = p.E - 1;
-  while (lo < hi) {
-    int mid = (lo + hi + 1) >> 1;
-    if (sm.m_prefix[mid] * n <= t) lo = mid;
-    else hi = mid - 1;
-  }
-  const int e = lo;
-  const int local = t - sm.m_prefix[e] * n;
-  const int m_tiles = sm.m_prefix[e + 1] - sm.m_prefix[e];
-  r.e = e;
-  r.n_blk = local / m_tiles;
-  const int m_blk = local - r.n_blk * m_tiles;
-  r.gm = sm.m_prefix[e] + m_blk;
-  r.m0 = fseg_begin(p, e) + m_blk * BM;
-  r.end = fseg_end(p, e);
-  return r;
-}
-
-__device__ __forceinline__ bool fwait(uint64_t *bar, uint32_t parity, SmemF &sm, int *status) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = ptx::globaltimer_ns();
-  while (true) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    if (*(volatile int *)&sm.abort) return false;
-    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
-      *(volatile int *)&sm.abort = 1;
-      atomicExch(status, kDevTimeout);
-      return false;
-    }
-  }
-}
-
-// Bounded wait for a gate/up m-block to be complete (all n1 tiles stored).
-__device__ __forceinline__ bool wait_count(const int *ctr, int want, SmemF &sm, int *status) {
-  if ((int)ptx::ld_acquire_gpu(ctr) >= want) return true;
-  const uint64_t t0 = ptx::globaltimer_ns();
-  while (true) {
-    __nanosleep(128);
-    if ((int)ptx::ld_acquire_gpu(ctr) >= want) return true;
-    if (*(volatile int *)&sm.abort) return false;
-    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
-      *(volatile int *)&sm.abort = 1;
-      atomicExch(status, kDevTimeout);
-      return false;
-    }
-  }
-}
-
-__global__ void __launch_bounds__(kThreads, 1)
-    tc_experts_fused(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmWg,
-                     const __grid_constant__ CUtensorMap tmWu, const __grid_constant__ CUtensorMap tmH,
-                     const __grid_constant__ CUtensorMap tmWd, const FusedParams p) {
-  using C = Cfg<false>;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t *stage_a = base;
-  uint8_t *stage_b = base + C::STAGES * A_BYTES;
-  SmemF &sm = *reinterpret_cast<SmemF *>(base + C::STAGES * C::STAGE_BYTES);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      ptx::mbar_init(&sm.full[s], 1);
-      ptx::mbar_init(&sm.empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      ptx::mbar_init(&sm.tmem_full[a], 1);
-      ptx::mbar_init(&sm.tmem_empty[a], 4);
-      ptx::mbar_init(&sm.h_done[a], 4);
-    }
-    for (int r = 0; r < kRing; ++r) {
-      ptx::mbar_init(&sm.ring_full[r], 1);
-      ptx::mbar_init(&sm.ring_empty[r], 5);  // the MMA thread + 4 epilogue warps
-    }
-    ptx::mbar_init(&sm.drain, 1);
-    sm.abort = 0;
-    ptx::fence_mbar_init();
-    ptx::fence_proxy_async_smem();
-  }
-  if (warp == 0 && lane == 0) {
-    ptx::prefetch_tmap(&tmX);
-    ptx::prefetch_tmap(&tmWg);
-    ptx::prefetch_tmap(&tmWu);
-    ptx::prefetch_tmap(&tmH);
-    ptx::prefetch_tmap(&tmWd);
-  }
-  if (warp == 1) {
-    ptx::tmem_alloc(&sm.tmem_base, TMEM_COLS);
-    ptx::tmem_relinquish();
-  }
-  if (warp == 2) {
-    int carry = 0;
-    for (int e0 = 0; e0 < p.E; e0 += 32) {
-      const int e = e0 + lane;
-      int v = 0;
-      if (e < p.E) {
-        int n = fseg_end(p, e) - fseg_begin(p, e);
-        v = n > 0 ? (n + BM - 1) / BM : 0;
-      }
-      int incl = v;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        int o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
-      }
-      if (e < p.E) sm.m_prefix[e] = carry + incl - v;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    if (lane == 0) sm.m_prefix[p.E] = carry;
-  }
-  ptx::tc_fence_before();
-  __syncwarp();
-  __syncthreads();
-  ptx::tc_fence_after();
-  const uint32_t tmem_base = sm.tmem_base;
-  const int total = sm.m_prefix[p.E] * (p.n1 + p.n2);
-  const int kb1 = p.D / BK, kb2 = p.F / BK;
-
-  if (warp == 0) {
-    // ================================================= producer: claims tiles, loads
-    if (lane == 0) {
-      uint32_t last_parity[4];
-      bool used[4];
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        used[s] = false;
-        last_parity[s] = 0;
-      }
-      uint32_t it = 0, ti = 0;
-      bool ok = true;
-      while (ok) {
-        int t = atomicAdd(&p.sched[0], 1);
-        if (t >= total) t = -1;
-        const int r = ti % kRing;
-        if (!fwait(&sm.ring_empty[r], ((ti / kRing) & 1u) ^ 1u, sm, p.status)) break;
-        sm.ring_tile[r] = t;
-        ptx::mbar_arrive(&sm.ring_full[r]);
-        ++ti;
-        if (t < 0) break;
-        const FTile tl = decode_fused(p, sm, t);
-        const int kbs = tl.phase == 1 ? kb1 : kb2;
-        if (tl.phase == 2) {
-          if (!wait_count(&p.sched[1 + tl.gm], p.n1, sm, p.status)) break;
-          ptx::fence_proxy_async_global();  // h written by other CTAs' generic stores, read by TMA
-        }
-        for (int kb = 0; kb < kbs; ++kb, ++it) {
-          const int s = it % C::STAGES;
-          const uint32_t ph = (it / C::STAGES) & 1u;
-          if (!fwait(&sm.empty[s], ph ^ 1u, sm, p.status)) { ok = false; break; }
-          ptx::mbar_arrive_expect_tx(&sm.full[s], C::TX_BYTES);
-          const int k0 = kb * BK;
-          uint8_t *a = stage_a + s * A_BYTES;
-          uint8_t *b = stage_b + s * C::B_BYTES;
-          if (tl.phase == 1) {
-            const int n0 = tl.n_blk * (BN / 2);
-            ptx::tma_load_2d(a, &tmX, &sm.full[s], k0, tl.m0);
-            ptx::tma_load_3d(b, &tmWg, &sm.full[s], k0, n0, tl.e);
-            ptx::tma_load_3d(b + C::B_BYTES / 2, &tmWu, &sm.full[s], k0, n0, tl.e);
-          } else {
-            const int n0 = tl.n_blk * BN;
-            ptx::tma_load_2d(a, &tmH, &sm.full[s], k0, tl.m0);
-            ptx::tma_load_3d(b, &tmWd, &sm.full[s], k0, n0, tl.e);
-            ptx::tma_load_3d(b + C::B_BYTES / 2, &tmWd, &sm.full[s], k0, n0 + BN / 2, tl.e);
-          }
-          used[s] = true;
-          last_parity[s] = ph;
-        }
-      }
-      if (!ok || *(volatile int *)&sm.abort) {
-        // make sure the consumers see an end marker if they are still reading the ring
-        const int r = ti % kRing;
-        if (fwait(&sm.ring_empty[r], ((ti / kRing) & 1u) ^ 1u, sm, p.status)) {
-          sm.ring_tile[r] = -1;
-          ptx::mbar_arrive(&sm.ring_full[r]);
-        }
-      }
-      for (int s = 0; s < 4; ++s)
-        if (used[s]) drain_bar(&sm.full[s], last_parity[s], p.status);
-    }
-  } else if (warp == 1) {
-    // ================================================= MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, BN);
-      uint32_t it = 0, ti = 0;
-      int i = 0;
-      while (true) {
-        const int r = ti % kRing;
-        if (!fwait(&sm.ring_full[r], (ti / kRing) & 1u, sm, p.status)) break;
-        const int t = sm.ring_tile[r];
-        ptx::mbar_arrive(&sm.ring_empty[r]);
-        ++ti;
-        if (t < 0) break;
-        const FTile tl = decode_fused(p, sm, t);
-        const int kbs = tl.phase == 1 ? kb1 : kb2;
-        const int acc = i & 1;
-        const uint32_t aph = (i >> 1) & 1u;
-        ++i;
-        if (!fwait(&sm.tmem_empty[acc], aph ^ 1u, sm, p.status)) break;
-        ptx::tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
-        bool ok = true;
-        for (int kb = 0; kb < kbs; ++kb, ++it) {
-          const int s = it % C::STAGES;
-          const uint32_t ph = (it / C::STAGES) & 1u;
-          if (!fwait(&sm.full[s], ph, sm, p.status)) { ok = false; break; }
-          ptx::tc_fence_after();
-          const uint32_t a_addr = ptx::smem_addr(stage_a + s * A_BYTES);
-          const uint32_t b_addr = ptx::smem_addr(stage_b + s * C::B_BYTES);
-#pragma unroll
-          for (int k = 0; k < BK / UMMA_K; ++k) {
-            const uint64_t ad = ptx::desc_kmajor_sw128(a_addr + k * UMMA_K * 2);
-            const uint64_t bd = ptx::desc_kmajor_sw128(b_addr + k * UMMA_K * 2);
-            ptx::mma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0);
-          }
-          ptx::mma_commit(&sm.empty[s]);
-        }
-        if (!ok) break;
-        ptx::mma_commit(&sm.tmem_full[acc]);
-      }
-      ptx::mma_commit(&sm.drain);
-      drain_bar(&sm.drain, 0, p.status);
-    }
-  } else {
-    // ================================================= epilogue (warps 2..5)
-    const int q = warp & 3;
-    const int row_in_tile = q * 32 + lane;
-    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
-    uint32_t ti = 0;
-    int i = 0;
-    while (true) {
-      const int r = ti % kRing;
-      // one lane waits; decisions are warp-uniform (tcgen05.ld needs the whole warp)
-      bool ok = true;
-      if (lane == 0) ok = fwait(&sm.ring_full[r], (ti / kRing) & 1u, sm, p.status);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      const int t = sm.ring_tile[r];
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&sm.ring_empty[r]);
-      ++ti;
-      if (t < 0) break;
-      const FTile tl = decode_fused(p, sm, t);
-      const int acc = i & 1;
-      const uint32_t aph = (i >> 1) & 1u;
-      ++i;
-      if (lane == 0) ok = fwait(&sm.tmem_full[acc], aph, sm, p.status);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      ptx::tc_fence_after();
-      const uint32_t tbase = tmem_base + lane_addr + acc * BN;
-      const int row = tl.m0 + row_in_tile;
-      const bool live = row < tl.end;
-      if (tl.phase == 1) {
-        const int ncol0 = tl.n_blk * (BN / 2);
-        __nv_bfloat16 *hrow = p.h + (long)row * p.F + ncol0;
-#pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
-          uint32_t g[32], u[32];
-          ptx::tmem_ld32(tbase + c, g);
-          ptx::tmem_ld32(tbase + BN / 2 + c, u);
-          ptx::tmem_ld_wait();
-          if (live) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              float h0 = swiglu_h(__uint_as_float(g[2 * j]), __uint_as_float(u[2 * j]), p.clamp, p.clamp_mode);
-              float h1 = swiglu_h(__uint_as_float(g[2 * j + 1]), __uint_as_float(u[2 * j + 1]), p.clamp,
-                                  p.clamp_mode);
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(h0, h1);
-              pk[j] = *reinterpret_cast<uint32_t *>(&b2);
-            }
-            uint4 *dst = reinterpret_cast<uint4 *>(hrow + c);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-          }
-        }
-        ptx::fence_proxy_async_global();  // these h stores will be read by TMA
-      } else {
-        const int ncol0 = tl.n_blk * BN;
-        const float rw = (live && p.row_weight) ? p.row_weight[row] : 1.0f;
-        float *yrow = p.y + (long)row * p.D + ncol0;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t v[32];
-          ptx::tmem_ld32(tbase + c, v);
-          ptx::tmem_ld_wait();
-          if (live) {
-            float4 *dst = reinterpret_cast<float4 *>(yrow + c);
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              dst[j] = make_float4(__uint_as_float(v[4 * j]) * rw, __uint_as_float(v[4 * j + 1]) * rw,
-                                   __uint_as_float(v[4 * j + 2]) * rw, __uint_as_float(v[4 * j + 3]) * rw);
-          }
-        }
-      }
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        ptx::mbar_arrive(&sm.h_done[acc]);
-        ptx::mbar_arrive(&sm.tmem_empty[acc]);
-      }
-      if (tl.phase == 1 && warp == 2 && lane == 0) {
-        // all four epilogue warps have stored their rows of this gate/up tile
-        if (fwait(&sm.h_done[acc], aph, sm, p.status)) {
-          __threadfence();
-          ptx::red_release_gpu_add(&p.sched[1 + tl.gm], 1);
-        }
-      }
-    }
-  }
-
-  ptx::tc_fence_before();
-  __syncwarp();
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
-  }
-}
-
 // ------------------------------------------------------------------ host
-struct DevInfo {
-  int sms = 0;
-  int pair_clusters = 0;  // co-resident CTA pairs of the pair kernels
-};
-
 template <bool GATED, bool PAIR>
 size_t smem_bytes() {
   return 1024 + (size_t)Cfg<PAIR>::STAGES * Cfg<PAIR>::STAGE_BYTES + sizeof(Smem);
@@ -889,58 +502,21 @@ moe_status launch_tc(const Params &p, const void *a, const void *b0, const void 
 }
 
 
-// rows of A and of h, per launch
-moe_status launch_fused(const MoEConfig &c, int rows, const void *x_perm, const int32_t *offsets,
-                        const void *w_gate, const void *w_up, const void *w_down, const float *row_weight,
-                        __nv_bfloat16 *h, float *y, int *status, int *sched, cudaStream_t s) {
-  FusedParams p;
-  p.rows = rows;
-  p.D = c.hidden_dim;
-  p.F = c.intermediate_dim;
-  p.E = offsets ? c.num_experts : 1;
-  p.n1 = p.F / (BN / 2);
-  p.n2 = p.D / BN;
-  p.offsets = offsets;
-  p.h = h;
-  p.y = y;
-  p.row_weight = row_weight;
-  p.clamp = c.swiglu_clamp;
-  p.clamp_mode = c.clamp_mode;
-  p.status = status;
-  p.sched = sched;
-  CUtensorMap tx, twg, twu, th, twd;
-  if (!tma_map_bf16(&tx, x_perm, 2, (uint64_t)p.D, (uint64_t)rows, 1)) return MOE_ERR_CUDA;
-  if (!tma_map_bf16(&twg, w_gate, 3, (uint64_t)p.D, (uint64_t)p.F, (uint64_t)p.E)) return MOE_ERR_CUDA;
-  if (!tma_map_bf16(&twu, w_up, 3, (uint64_t)p.D, (uint64_t)p.F, (uint64_t)p.E)) return MOE_ERR_CUDA;
-  if (!tma_map_bf16(&th, h, 2, (uint64_t)p.F, (uint64_t)rows, 1)) return MOE_ERR_CUDA;
-  if (!tma_map_bf16(&twd, w_down, 3, (uint64_t)p.F, (uint64_t)p.D, (uint64_t)p.E)) return MOE_ERR_CUDA;
-  const long mt_ub = (long)(rows + BM - 1) / BM + p.E;
-  MOE_CUDA_TRY(cudaMemsetAsync(sched, 0, sizeof(int) * (size_t)(1 + mt_ub), s));
-  int dev = 0, sms = 148;
-  MOE_CUDA_TRY(cudaGetDevice(&dev));
-  MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  const long ub = mt_ub * (p.n1 + p.n2);
-  const int grid = (int)(ub < sms ? ub : sms);
-  const size_t smem = 1024 + (size_t)Cfg<false>::STAGES * Cfg<false>::STAGE_BYTES + sizeof(SmemF);
-  MOE_CUDA_TRY(cudaFuncSetAttribute(tc_experts_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  tc_experts_fused<<<grid, kThreads, smem, s>>>(tx, twg, twu, th, twd, p);
-  MOE_LAUNCH_CHECK();
-  return MOE_OK;
-}
-
 // Pairs pay off only when groups are so large that the padding of their last
 // 256-row tile is negligible (measured under the power cap, extra padded rows
-// cost more than the pair saves on operand traffic).  The
-// environment variable MOE_TC_TILE = 128 | 256 overrides the choice (for
-// tuning; both paths compute the same result).
-bool use_pair(int rows, int E, bool gated) {
-  const char *env = getenv("MOE_TC_TILE");
-  if (env && env[0] == '1') return false;
-  if (env && env[0] == '2') return true;
-  // measured (A/B in one process): gate/up gains only for very large groups;
-  // down, with 3.5x longer tiles and fewer of them, already at ~1000 rows
-  return rows >= (gated ? 2048L : 768L) * E;
-}
+// cost more than the pair saves on operand traffic): gate/up from
+// kPairRowsGated rows per group on average, down, with 3.5x longer tiles and
+// fewer of them, from kPairRowsDown.  Both tile shapes compute the same
+// result to fp32 rounding.
+#ifndef MOE_PAIR_ROWS_GATED
+#define MOE_PAIR_ROWS_GATED 2048
+#endif
+#ifndef MOE_PAIR_ROWS_DOWN
+#define MOE_PAIR_ROWS_DOWN 768
+#endif
+constexpr long kPairRowsGated = MOE_PAIR_ROWS_GATED;
+constexpr long kPairRowsDown = MOE_PAIR_ROWS_DOWN;
+bool use_pair(int rows, int E, bool gated) { return rows >= (gated ? kPairRowsGated : kPairRowsDown) * E; }
 
 // One thread waits on an mbarrier that nothing arrives on, with the bounded
 // wait of the pipelines above: it gives up after kWaitLimitNs and records the
@@ -1009,19 +585,6 @@ moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int
   p.status = status;
   if (use_pair(rows, p.E, false)) return launch_tc<false, true>(p, h, w_down, nullptr, c.hidden_dim, s);
   return launch_tc<false, false>(p, h, w_down, nullptr, c.hidden_dim, s);
-}
-
-size_t fused_sched_ints(const MoEConfig &c, int rows, bool grouped) {
-  return 1 + (size_t)(rows + BM - 1) / BM + (grouped ? c.num_experts : 1);
-}
-
-moe_status launch_experts_fused_tc(const MoEConfig &c, int rows, const void *x_perm, const int32_t *offsets,
-                                   const void *w_gate, const void *w_up, const void *w_down,
-                                   const float *row_weight, void *h, float *y, int *status, int *sched,
-                                   cudaStream_t s) {
-  if (rows == 0) return MOE_OK;
-  return launch_fused(c, rows, x_perm, offsets, w_gate, w_up, w_down, row_weight, (__nv_bfloat16 *)h, y, status,
-                      sched, s);
 }
 
 }  // namespace moe

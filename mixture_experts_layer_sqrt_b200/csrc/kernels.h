@@ -36,6 +36,10 @@ moe_status launch_dispatch(const MoEConfig &c, int T, const int32_t *topk_idx, c
                            int32_t *slot_row, int32_t *row_token, float *row_weight, void *x_perm,
                            int32_t *chunk_cnt, cudaStream_t s);
 
+// x_perm[r] = x[row_token[r]] for r < expert_offsets[E] (act dtype rows).
+moe_status launch_gather(const MoEConfig &c, int T, const int32_t *expert_offsets, const int32_t *row_token,
+                         const void *x, void *x_perm, cudaStream_t s);
+
 // x_perm rows in f16, each scaled by a power of two (row_scale[r] = 2^-s_r),
 // for the FP4 gate/up GEMM in f16 (bf16 activations only).
 moe_status launch_gather_f16(const MoEConfig &c, int T, const int32_t *expert_offsets, const int32_t *row_token,
@@ -80,15 +84,6 @@ moe_status launch_down_fp4(const MoEConfig &c, int rows, const void *h, const in
 
 // One block whose bounded wait never completes: records the timeout status.
 moe_status launch_wait_selftest(int *status, cudaStream_t s);
-
-// Both projections in one persistent launch (gate/up tiles, then down tiles
-// that wait for their m-block of h).  sched: fused_sched_ints() ints of
-// scratch, zeroed by the launcher.
-size_t fused_sched_ints(const MoEConfig &c, int rows, bool grouped);
-moe_status launch_experts_fused_tc(const MoEConfig &c, int rows, const void *x_perm, const int32_t *offsets,
-                                   const void *w_gate, const void *w_up, const void *w_down,
-                                   const float *row_weight, void *h, float *y, int *status, int *sched,
-                                   cudaStream_t s);
 
 // dequant.cu -------------------------------------------------------------
 // n_elems values (a multiple of 16): packed [n/2] bytes + scales [n/16] -> bf16 [n].

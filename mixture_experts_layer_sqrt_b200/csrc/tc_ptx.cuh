@@ -215,20 +215,6 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t *bar) {
                : "memory");
 }
 
-// ------------------------------------------- cross-CTA flags in global memory
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const int *p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void red_release_gpu_add(int *p, int v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-// Orders this thread's generic-proxy global accesses with async-proxy (TMA) ones.
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
 // ------------------------------------------------------------ FP4 codes
 // Eight e2m1 codes (byte i holds elements 2i in bits [3:0] and 2i+1 in bits
 // [7:4]) to four f16x2 words, element 2i in the low half of word i.

@@ -145,13 +145,14 @@ def test_profiled_forward_event_count(B):
     c = _cfg(B)
     w = B.MoEWeights(w_router=16, w_gate=16, w_up=16, w_down=16)
     need = B.lib.moe_workspace_size(ctypes.byref(c), 64)
-    ev = (ctypes.c_void_p * 7)()
-    for n in (1, 6, 8, -1):
+    assert B.STAGE_EVENTS == 8
+    ev = (ctypes.c_void_p * 9)()
+    for n in (1, 7, 9, -1):
         st = B.lib.moe_forward_profiled(ctypes.byref(c), 64, 16, ctypes.byref(w), None, 16, None, None, 16, need,
                                         None, ctypes.cast(ev, ctypes.c_void_p), n)
         assert st == B.MOE_ERR_INVALID_ARG
     st = B.lib.moe_forward_profiled(ctypes.byref(c), 64, 16, ctypes.byref(w), None, 16, None, None, 16, need,
-                                    None, None, 7)
+                                    None, None, 8)
     assert st == B.MOE_ERR_INVALID_ARG
 
 

@@ -41,15 +41,18 @@ def test_report_keys_and_roofline(name, kind, bound):
     assert res["dtype"] == ("f32" if p.act == "f32" else "bf16")
 
 
-def test_traffic_records_follow_their_kernel_sources(monkeypatch):
+def test_traffic_records_follow_their_kernel_sources(monkeypatch, tmp_path):
     # each recorded DRAM figure is keyed to a hash of its kernel's sources;
     # the record is void as soon as one of them differs
-    assert bench.profiled_traffic("gate_up_mixtral_bf16") > 0
-    assert bench.profiled_traffic("gate_up_sqrt_fp4") > 0
-    assert bench.profiled_traffic("gate_up_tiny_f32") is None
+    rec = tmp_path / "traffic.txt"
+    sha = bench.gemm_sources_sha(bench.TRAFFIC_SOURCES["gate_up_sqrt_fp4"])
+    rec.write_text(f"# comment\ngate_up_sqrt_fp4 {sha} 123456\ngate_up_mixtral_bf16 0000000000000000 99\n")
+    assert bench.profiled_traffic("gate_up_sqrt_fp4", str(rec)) == 123456.0
+    assert bench.profiled_traffic("gate_up_mixtral_bf16", str(rec)) is None  # stale sources hash
+    assert bench.profiled_traffic("gate_up_tiny_f32", str(rec)) is None
     changed = dict(bench.TRAFFIC_SOURCES, gate_up_sqrt_fp4=("gemm_fp4.cu", "api.cu"))
     monkeypatch.setattr(bench, "TRAFFIC_SOURCES", changed)
-    assert bench.profiled_traffic("gate_up_sqrt_fp4") is None
+    assert bench.profiled_traffic("gate_up_sqrt_fp4", str(rec)) is None
 
 
 def test_extrapolation_arithmetic():
@@ -88,3 +91,20 @@ def test_reference_arm_line_small_workload():
     assert res["e2e"]["value"] == res["value"] and res["e2e"]["h2d_bytes_per_step"] == 0
     assert res["config"] == bench.workload_config(p, 1, res["config"]["rows_after_capacity"])
     assert 0 < res["config"]["rows_after_capacity"] <= p.T * p.k
+
+
+def test_permute_combine_bandwidth():
+    # Mixtral shape: gather 2 * 8192 rows * 4096 * 2 B, combine 8192 * 4096 * 4 + 4096 * 4096 * 4 B
+    p = synth.PROBLEMS["mixtral_bf16"]
+    stage_ms = {n: 0.0 for n in bench.STAGES}
+    stage_ms.update(gather=0.02, combine=0.03)
+    pc = bench.permute_combine(p, 8192, stage_ms, {"hbm": 6000.0, "src": "test"})
+    assert pc["gather"]["bytes"] == 2 * 8192 * 4096 * 2
+    assert pc["combine"]["bytes"] == 8192 * 4096 * 4 + 4096 * 4096 * 4
+    assert pc["gather"]["gbs"] == pytest.approx(pc["gather"]["bytes"] / 0.02e-3 / 1e9)
+    assert pc["combine"]["frac"] == pytest.approx(pc["combine"]["gbs"] / 6000.0)
+    # the shared expert's fp32 row is read by combine too; NVFP4 rows carry a scale each
+    q = synth.PROBLEMS["sqrt_fp4"]
+    pq = bench.permute_combine(q, 49152, stage_ms, {"hbm": 6000.0, "src": "test"})
+    assert pq["combine"]["bytes"] == 49152 * 4096 * 4 + 2 * 8192 * 4096 * 4
+    assert pq["gather"]["bytes"] == 2 * 49152 * 4096 * 2 + 4 * 49152

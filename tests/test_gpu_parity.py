@@ -124,15 +124,10 @@ def test_stages_small(B, W, name):
     y_g = H.to_np(g["y"][:R])
     H.assert_close_f32(y_g, y_ref, "y_perm")
 
-    # both projections in one call (the fused persistent kernel on the tensor-core
-    # path): the same tiles as the staged kernels, so the same bits when both use
-    # 128-row tiles; within the fp32 bound otherwise
+    # both projections in one call: the same launches as the staged calls, so the same bits
     y2 = B.grouped_swiglu(c.cfg, g["x_perm"], g["expert_offsets"], c.w, g["row_weight"])
     torch.cuda.synchronize()
-    if p.name.endswith("_pair"):
-        H.assert_close_f32(H.to_np(y2[:R]), y_ref, "grouped_swiglu")
-    else:
-        assert torch.equal(y2[:R], g["y"][:R])
+    assert torch.equal(y2[:R], g["y"][:R])
 
     # a8 shared expert
     sh_g = None
@@ -352,28 +347,8 @@ def test_binding_rejects_mismatched_out(B, W):
         B.forward(c.cfg, c.x, c.w, ws, out=torch.empty((p.T - 1, p.D), dtype=torch.float32, device="cuda"))
 
 
-@pytest.mark.parametrize("name", ["mixtral_bf16", "finegrained_bf16", "capacity_bf16"])
-def test_fused_expert_kernel_matches(B, W, name, monkeypatch):
-    # the single persistent launch (gate/up tiles, then down tiles waiting on
-    # their m-block of h) gives the two-launch result bit for bit
-    p = H.small(name)
-    c = Case(B, W, p)
-    idx, w = B.route_topk(c.cfg, c.x, c.w, c.mask)
-    d = B.dispatch(c.cfg, c.x, idx, w)
-    rows = p.T * p.k
-    ws = B.workspace(B.grouped_swiglu_workspace_size(c.cfg, rows))
-    ref = B.grouped_swiglu(c.cfg, d["x_perm"], d["expert_offsets"], c.w, d["row_weight"], ws=ws)
-    torch.cuda.synchronize()
-    monkeypatch.setenv("MOE_EXPERTS_FUSED", "1")
-    got = B.grouped_swiglu(c.cfg, d["x_perm"], d["expert_offsets"], c.w, d["row_weight"], ws=ws)
-    torch.cuda.synchronize()
-    B.check_device_status(ws)
-    R = int(d["expert_offsets"][-1])
-    assert torch.equal(got[:R], ref[:R])
-
-
 @pytest.mark.parametrize("name", ["sqrt_fp4_pair", "sqrt_fp4"])
-def test_fp4_direct_matches_expanded_weights(B, W, name, monkeypatch):
+def test_fp4_direct_matches_expanded_weights(B, W, name):
     # NVFP4 codes converted to bf16 in shared memory give the MMA the same
     # operand bits as weights expanded beforehand (every e2m1 * e4m3 product is
     # exact in bf16): bit for bit the bf16 GEMM (same 128-row tiles) on the
@@ -393,7 +368,8 @@ def test_fp4_direct_matches_expanded_weights(B, W, name, monkeypatch):
         assert np.array_equal(v.astype(np.float32).astype(np.float64), v)  # exact in fp32 (and bf16)
         ex[k] = W.to_torch(synth.f32_to_bf16_bits(v.astype(np.float32)))
     cfg16 = W.config_of(p.with_(wdtype="bf16"))
-    monkeypatch.setenv("MOE_TC_TILE", "128")
+    # few rows per expert: the bf16 GEMMs take single 128-row tiles too
+    assert p.T * p.k < 768 * p.E
     h16 = B.expert_gate_up(cfg16, d["x_perm"], d["expert_offsets"], ex["w_gate"], ex["w_up"])
     y16 = B.expert_down(cfg16, h16, d["expert_offsets"], ex["w_down"], None, d["row_weight"])
     torch.cuda.synchronize()
