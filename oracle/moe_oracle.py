@@ -27,6 +27,9 @@ Sources (web pages on the subject; cited by title and section):
   (bias_vl=0 parity, softplus large-x branch, shared expert added once).
 * [ECHO] Echo's MoE quick reference (cybersecurityerial.github.io) -- the four
   stages Router, Dispatch, FFN, Combine.
+* [TH]   "กลยุทธ์การกำหนดเส้นทาง MoE: Top-K, Expert-Choice และ Sigmoid Gating"
+  (blogdee.com) -- the router scores every expert, keeps the top-scoring
+  ones, and a sigmoid gate gives the mixing weights of the selected experts.
 
 Readings where the pages are silent or disagree (each also listed in the
 design notes):
@@ -55,6 +58,11 @@ design notes):
    renormalised.
 9. The shared expert has weight 1 and is added once: out = shared(x) + routed.
 10. No Linear biases anywhere (the formulas have none).
+11. Sigmoid gate ([TH] names it as the function that gives the selected
+    experts' mixing weights, and no more): w_j = sigmoid(s_j) of the raw
+    router score, not renormalised; selection is top-k of the score plus the
+    selection bias exactly as in the sqrt-softplus gate (bias_vl at image
+    positions), the bias never entering the weight.
 
 Function pins (tests/test_oracle.py): every function below is pinned against
 the pages' worked example, closed forms, a library routine or a brute force,
@@ -142,6 +150,13 @@ def silu(z: np.ndarray) -> np.ndarray:
         return z / (1.0 + np.exp(-z))
 
 
+def sigmoid(z: np.ndarray) -> np.ndarray:
+    """sigmoid(z) = 1 / (1 + e^-z), evaluated without overflow on either side ([TH] "Sigmoid Gating")."""
+    z = np.asarray(z, dtype=np.float64)
+    e = np.exp(-np.abs(z))
+    return np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
 def softmax_rows(l: np.ndarray) -> np.ndarray:
     """Row softmax, p_i = e^{l_i} / sum_j e^{l_j} (max-shifted) ([FSM] sec. 3)."""
     m = l.max(axis=1, keepdims=True)
@@ -171,7 +186,8 @@ def selection_keys(logits: np.ndarray, gate: str, bias: Optional[np.ndarray] = N
     """The value the top-k compares.
 
     softmax mode: the (optionally logit-biased) router logit.
-    sqrt_softplus mode: s + bias_vl at image positions, s + bias elsewhere ([DSV] sec. 1, 3).
+    sqrt_softplus and sigmoid modes: s + bias_vl at image positions, s + bias
+    elsewhere ([DSV] sec. 1, 3; reading 11 for the sigmoid gate).
     """
     if gate == "softmax":
         return logits + (0.0 if bias is None else bias.astype(np.float64)[None, :])
@@ -192,13 +208,18 @@ def route_weights(logits: np.ndarray, idx: np.ndarray, gate: str,
     softmax: p = softmax over all experts of the (biased) logits, then the
     selected p renormalised to sum 1 ([FSM] sec. 3 example module).
     sqrt_softplus: sqrt(softplus(s)) of the raw logit, unnormalised ([DSV] sec. 1).
+    sigmoid: sigmoid(s) of the raw logit, unnormalised ([TH]; reading 11).
     """
     if gate == "softmax":
         l = logits + (0.0 if bias is None else bias.astype(np.float64)[None, :])
         p = softmax_rows(l)
         ps = np.take_along_axis(p, idx, axis=1)
         return ps / ps.sum(axis=1, keepdims=True)
-    return sqrt_softplus(np.take_along_axis(logits, idx, axis=1))
+    if gate == "sigmoid":
+        return sigmoid(np.take_along_axis(logits, idx, axis=1))
+    if gate == "sqrt_softplus":
+        return sqrt_softplus(np.take_along_axis(logits, idx, axis=1))
+    raise ValueError(gate)
 
 
 def route(logits: np.ndarray, k: int, gate: str, bias=None, bias_vl=None, image_mask=None):

@@ -315,11 +315,43 @@ def check_bf16_decode():
     np.testing.assert_array_equal(O.decode_bf16(bits), want)
 
 
+def check_sigmoid_closed_forms():
+    # sigmoid(0) = 1/2, sigmoid(ln 3) = 3/4, sigmoid(-ln 3) = 1/4, sigmoid(-z) = 1 - sigmoid(z);
+    # scipy's expit over the whole range, saturating cleanly at both ends
+    np.testing.assert_allclose(O.sigmoid(np.array([0.0, math.log(3.0), -math.log(3.0)])), [0.5, 0.75, 0.25],
+                               rtol=1e-15)
+    z = np.concatenate([np.linspace(-40, 40, 1601), [-800.0, -50.0, 50.0, 800.0]])
+    np.testing.assert_allclose(O.sigmoid(z) + O.sigmoid(-z), 1.0, rtol=1e-15)
+    np.testing.assert_allclose(O.sigmoid(z), scipy.special.expit(z), rtol=1e-14, atol=0)
+    assert O.sigmoid(np.array([-800.0]))[0] == 0.0 and O.sigmoid(np.array([800.0]))[0] == 1.0
+
+
+def check_sigmoid_route():
+    rng = np.random.default_rng(5)
+    T, E, k = 64, 16, 4
+    s = rng.standard_normal((T, E)) * 3
+    bias = rng.uniform(-0.5, 0.5, E)
+    bvl = rng.uniform(-0.5, 0.5, E)
+    img = (rng.random(T) < 0.3).astype(np.uint8)
+    idx, w, keys = O.route(s, k, "sigmoid", bias, bvl, img)
+    # weights: the library sigmoid of the raw score, unnormalised (sums are not 1)
+    np.testing.assert_allclose(w, scipy.special.expit(np.take_along_axis(s, idx, 1)), rtol=1e-14)
+    assert np.all((w > 0) & (w < 1)) and not np.allclose(w.sum(1), 1.0)
+    # selection: brute force over s + bias_vl at image rows, s + bias elsewhere
+    for t in range(T):
+        b = bvl if img[t] else bias
+        want = sorted(range(E), key=lambda e: (-(s[t, e] + b[e]), e))[:k]
+        assert list(idx[t]) == want
+    # without a bias the weights rank like the scores (sigmoid is increasing)
+    idxn, wn, _ = O.route(s, k, "sigmoid")
+    assert np.all(np.diff(wn, axis=1) <= 0)
+
+
 CHECKS = [check_worked_example, check_softplus_library, check_silu_library, check_softmax_library,
           check_topk_bruteforce, check_softmax_route, check_sqrt_route, check_capacity_table,
           check_dispatch_sort, check_expert_library, check_layer_e1k1, check_router_library,
           check_sparse_dense, check_shared_once, check_clamp, check_e2m1_table, check_e4m3_library,
-          check_nvfp4_dequant, check_bf16_decode]
+          check_nvfp4_dequant, check_bf16_decode, check_sigmoid_closed_forms, check_sigmoid_route]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=lambda c: c.__name__)
@@ -434,6 +466,18 @@ def _mut_selection_keys(logits, gate, bias=None, bias_vl=None, image_mask=None):
     return _orig["selection_keys"](logits, gate, bias, None, None)  # bias_vl ignored
 
 
+def _mut_sigmoid(z):
+    z = np.asarray(z, dtype=np.float64)
+    return 1.0 / (1.0 + np.exp(z))                                 # sign error: sigmoid(-z)
+
+
+def _mut_route_weights_sigmoid_renorm(logits, idx, gate, bias=None):
+    if gate != "sigmoid":
+        return _orig["route_weights"](logits, idx, gate, bias)
+    w = O.sigmoid(np.take_along_axis(logits, idx, axis=1))
+    return w / w.sum(axis=1, keepdims=True)                        # renormalised (not in the reading)
+
+
 def _mut_silu(z):
     return np.asarray(z, float) / (1.0 + np.exp(np.asarray(z, float)))  # sign error
 
@@ -459,6 +503,8 @@ MUTANTS = {
     "softmax_rows": _mut_softmax_rows,
     "selection_keys": _mut_selection_keys,
     "silu": _mut_silu,
+    "sigmoid": _mut_sigmoid,
+    "route_weights#sigmoid": _mut_route_weights_sigmoid_renorm,
 }
 
 
