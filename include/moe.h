@@ -60,7 +60,14 @@ typedef enum {
   /* selection: top-k of s_e + bias_vl[e] at image positions, s_e + bias[e]
    * elsewhere; multiplier: sqrt(softplus(s_e)) of the raw score, not
    * normalised ("5A · MoE fine-grained" sec. 1, 3). */
-  MOE_GATE_SQRT_SOFTPLUS_RAW = 1
+  MOE_GATE_SQRT_SOFTPLUS_RAW = 1,
+  /* selection as in MOE_GATE_SQRT_SOFTPLUS_RAW (bias / bias_vl enter the
+   * selection key only); multiplier: sigmoid(s_e) = 1 / (1 + e^-s_e) of the
+   * raw score, not normalised.  ("กลยุทธ์การกำหนดเส้นทาง MoE: Top-K,
+   * Expert-Choice และ Sigmoid Gating", blogdee.com: the sigmoid gives the
+   * mixing weights of the selected experts; the selection rule and the
+   * absence of renormalisation are this library's reading.) */
+  MOE_GATE_SIGMOID_RAW = 2
 } moe_gate;
 
 typedef enum {
@@ -105,8 +112,8 @@ typedef struct {
   const void *sh_gate;         /* [F_s, D] act dtype (shared expert) */
   const void *sh_up;           /* [F_s, D] */
   const void *sh_down;         /* [D, F_s] */
-  const float *bias;           /* [E] or NULL: softmax mode logit bias / sqrt mode selection bias */
-  const float *bias_vl;        /* [E] or NULL: sqrt mode selection bias at image positions */
+  const float *bias;           /* [E] or NULL: softmax mode logit bias / sqrt and sigmoid modes selection bias */
+  const float *bias_vl;        /* [E] or NULL: sqrt and sigmoid modes selection bias at image positions */
 } MoEWeights;
 
 /* ------------------------------------------------------------------ misc */
@@ -148,11 +155,11 @@ size_t moe_route_workspace_size(const MoEConfig *cfg, int T);
 /* Router GEMM + gate + top-k for T tokens (a1-a2).
  *   x          [T, D] act dtype
  *   w->w_router, w->bias, w->bias_vl as in MoEWeights (other fields unused)
- *   image_mask [T] uint8 (nonzero = image position) or NULL; sqrt gate only
+ *   image_mask [T] uint8 (nonzero = image position) or NULL; sqrt and sigmoid gates only
  *   topk_idx   [T, k] int32 out: selected experts, descending selection key,
  *              equal keys ordered by lower expert index
  *   topk_w     [T, k] float out: the multipliers (renormalised softmax, or raw
- *              sqrt(softplus(s)))
+ *              sqrt(softplus(s)), or raw sigmoid(s))
  *   ws         >= moe_route_workspace_size(cfg, T) bytes (status word)
  * Logits are accumulated in fp32 (ops-transformer walkthrough, 坑三).  With
  * E <= 32 (or fp32 activations) one kernel computes them on the CUDA cores

@@ -19,11 +19,12 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200
 # enums (include/moe.h)
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE_TIMEOUT = range(6)
 MOE_F32, MOE_BF16, MOE_NVFP4 = range(3)
-MOE_GATE_SOFTMAX_TOPK_RENORM, MOE_GATE_SQRT_SOFTPLUS_RAW = range(2)
+MOE_GATE_SOFTMAX_TOPK_RENORM, MOE_GATE_SQRT_SOFTPLUS_RAW, MOE_GATE_SIGMOID_RAW = range(3)
 MOE_CLAMP_PREACT, MOE_CLAMP_OUTPUT = range(2)
 
 DTYPES = {"f32": MOE_F32, "bf16": MOE_BF16, "nvfp4": MOE_NVFP4}
-GATES = {"softmax": MOE_GATE_SOFTMAX_TOPK_RENORM, "sqrt_softplus": MOE_GATE_SQRT_SOFTPLUS_RAW}
+GATES = {"softmax": MOE_GATE_SOFTMAX_TOPK_RENORM, "sqrt_softplus": MOE_GATE_SQRT_SOFTPLUS_RAW,
+         "sigmoid": MOE_GATE_SIGMOID_RAW}
 CLAMP_MODES = {"preact": MOE_CLAMP_PREACT, "output": MOE_CLAMP_OUTPUT}
 
 

@@ -42,7 +42,8 @@ moe_status validate_cfg(const MoEConfig *c) {
   if (c->hidden_dim <= 0 || c->intermediate_dim <= 0 || c->shared_intermediate_dim < 0)
     return MOE_ERR_INVALID_ARG;
   if (c->hidden_dim % 8 != 0) return MOE_ERR_UNSUPPORTED;  // 16-byte row vectors
-  if (c->gate != MOE_GATE_SOFTMAX_TOPK_RENORM && c->gate != MOE_GATE_SQRT_SOFTPLUS_RAW)
+  if (c->gate != MOE_GATE_SOFTMAX_TOPK_RENORM && c->gate != MOE_GATE_SQRT_SOFTPLUS_RAW &&
+      c->gate != MOE_GATE_SIGMOID_RAW)
     return MOE_ERR_INVALID_ARG;
   if (!(c->swiglu_clamp >= 0.0f)) return MOE_ERR_INVALID_ARG;
   if (c->clamp_mode != MOE_CLAMP_PREACT && c->clamp_mode != MOE_CLAMP_OUTPUT) return MOE_ERR_INVALID_ARG;

@@ -5,9 +5,11 @@
 // selection, as the ops-transformer MoE walkthrough's 优化二 intends, without
 // its heap); larger key first, equal keys to the lower expert index.  Keys:
 // the logit in softmax mode (any router logit bias already added), the raw
-// score plus bias (or bias_vl at image positions) in sqrt mode.  Weights:
-// the renormalised softmax of the selected logits, or sqrt(softplus(s))
-// ("FFN、SwiGLU 与 MoE" sec. 3; "5A · MoE fine-grained" sec. 1, 3).
+// score plus bias (or bias_vl at image positions) in the sqrt and sigmoid
+// modes.  Weights: the renormalised softmax of the selected logits,
+// sqrt(softplus(s)), or sigmoid(s) ("FFN、SwiGLU 与 MoE" sec. 3; "5A · MoE
+// fine-grained" sec. 1, 3; the blogdee.com routing-strategies page on
+// Sigmoid Gating).
 #pragma once
 
 #include <math.h>
@@ -23,7 +25,7 @@ __device__ __forceinline__ void select_topk(const float *lg, long t, int E, int 
                                             const uint8_t *__restrict__ image_mask, int32_t *__restrict__ topk_idx,
                                             float *__restrict__ topk_w, int lane) {
   const float *sel_bias = nullptr;
-  if (gate == MOE_GATE_SQRT_SOFTPLUS_RAW) sel_bias = (bias_vl && image_mask && image_mask[t]) ? bias_vl : bias;
+  if (gate != MOE_GATE_SOFTMAX_TOPK_RENORM) sel_bias = (bias_vl && image_mask && image_mask[t]) ? bias_vl : bias;
   uint32_t removed = 0;  // bit j: expert lane + 32 j already selected
   int my_e = 0;
   float my_l = 0.0f;
@@ -53,6 +55,8 @@ __device__ __forceinline__ void select_topk(const float *lg, long t, int E, int 
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     w = ex / sum;
+  } else if (gate == MOE_GATE_SIGMOID_RAW) {
+    w = 1.0f / (1.0f + expf(-my_l));  // -> 0 and 1 at the ends, never NaN
   } else {
     w = sqrtf(softplus_f32(my_l));
   }

@@ -297,10 +297,10 @@ moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void 
   MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   long sel_blocks = ((long)T + kSelWarps - 1) / kSelWarps;
   if (sel_blocks > (long)sms * 8) sel_blocks = (long)sms * 8;
-  const float *sel_bias = c.gate == MOE_GATE_SQRT_SOFTPLUS_RAW ? bias : nullptr;  // softmax: already in the logits
+  const bool sel = c.gate != MOE_GATE_SOFTMAX_TOPK_RENORM;  // softmax: the logit bias is already in the logits
   route_select_kernel<<<(unsigned)sel_blocks, 32 * kSelWarps, (size_t)kSelWarps * p.ld * sizeof(float), s>>>(
-      T, p.E, p.ld, p.k, p.gate, scratch, sel_bias, c.gate == MOE_GATE_SQRT_SOFTPLUS_RAW ? bias_vl : nullptr,
-      image_mask, topk_idx, topk_w);
+      T, p.E, p.ld, p.k, p.gate, scratch, sel ? bias : nullptr, sel ? bias_vl : nullptr, image_mask, topk_idx,
+      topk_w);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }

@@ -52,7 +52,7 @@ class MoEProblem:
     k: int                      # top_k
     act: str = "bf16"           # activations and router weights: "f32" | "bf16"
     wdtype: str = "bf16"        # routed expert weights: "f32" | "bf16" | "nvfp4"
-    gate: str = "softmax"       # "softmax" (renormalised top-k) | "sqrt_softplus"
+    gate: str = "softmax"       # "softmax" (renormalised top-k) | "sqrt_softplus" | "sigmoid"
     capacity_factor: float = 0.0  # 0 = unlimited capacity
     clamp: float = 0.0          # SwiGLU clamp limit, 0 = off
     Fs: int = 0                 # shared expert intermediate dim, 0 = none

@@ -29,6 +29,10 @@ def small(name: str) -> synth.MoEProblem:
     if name == "sqrt_fp4_pair":
         # F % 256 == 0: both projections read the packed FP4 weights directly
         return synth.PROBLEMS["sqrt_fp4"].with_(name=name, T=2100, D=512, F=512, E=12, k=3, Fs=256)
+    if name == "sigmoid_bf16":
+        # the sigmoid gate with selection biases, image positions and a shared expert
+        return synth.MoEProblem(name, T=300, D=512, F=384, E=16, k=4, gate="sigmoid", bias="uniform", Fs=256,
+                                clamp=10.0, seed=7)
     p = synth.PROBLEMS[name]
     if name == "tiny_f32":
         return p

@@ -20,7 +20,7 @@ from tests import harness as H
 pytestmark = pytest.mark.gpu
 
 NAMES = ["tiny_f32", "mixtral_bf16", "capacity_bf16", "finegrained_bf16", "sqrt_fp4"]
-SMALL_NAMES = NAMES + ["mixtral_bf16_pair", "sqrt_fp4_pair"]
+SMALL_NAMES = NAMES + ["mixtral_bf16_pair", "sqrt_fp4_pair", "sigmoid_bf16"]
 
 
 @pytest.fixture(scope="module")
@@ -224,7 +224,8 @@ def test_full_size_sampled(B, W, name, n_sample):
 @pytest.mark.parametrize("E,k,gate,bias", [(8, 2, "softmax", "none"), (6, 6, "softmax", "zipf"),
                                            (33, 16, "sqrt_softplus", "uniform"), (48, 4, "softmax", "none"),
                                            (64, 2, "softmax", "zipf"), (128, 16, "softmax", "none"),
-                                           (300, 6, "sqrt_softplus", "uniform"), (512, 8, "softmax", "none")])
+                                           (300, 6, "sqrt_softplus", "uniform"), (512, 8, "softmax", "none"),
+                                           (8, 2, "sigmoid", "uniform"), (96, 6, "sigmoid", "uniform")])
 def test_route_many_experts(B, W, E, k, gate, bias):
     # the router on both paths (CUDA cores up to 32 experts, tensor cores
     # above): ragged 128-token tiles, padded expert columns, one or two MMA
