@@ -271,7 +271,9 @@ def run_ours(args, p, rank, world, local_rank):
     counts = torch.empty(p.E, dtype=torch.int32, device=dev)
     B.forward(cfg, x, w, ws_f, mask, out, expert_counts_out=counts)
     cap = cfg.expert_capacity
-    rows = int((counts.clamp(max=cap) if cap else counts).sum().item())
+    counts_h = counts.cpu().numpy()
+    lb = load_balance(counts_h, T, k, cap)
+    rows = lb["kept"]
 
     dist = None
     if world > 1:
@@ -313,7 +315,68 @@ def run_ours(args, p, rank, world, local_rank):
     res = report(args, p, world, rows, value, ms, per_step, gemm_ms, e2e, n_launch, clocks)
     res["stage_ms"] = stage_ms
     res["permute_combine"] = permute_combine(p, rows, stage_ms, load_peaks())
+    res["load_balance"] = lb
     return res
+
+
+def shared_expert_alone(B, p, x, wt, clamp_mode="preact"):
+    """The always-on shared expert by itself (staged gate/up and down calls, one group)."""
+    sc = B.make_config(E=1, k=1, D=p.D, F=p.Fs, clamp=p.clamp, clamp_mode=clamp_mode, act=p.act, expert=p.act)
+    hs = B.expert_gate_up(sc, x, None, wt["sh_gate"], wt["sh_up"])
+    return B.expert_down(sc, hs, None, wt["sh_down"])
+
+
+def run_sweep(args, p, ks):
+    """Per-token time of the whole layer at several top-k values on one shape
+    ("5A · MoE fine-grained" sec. 4, Profiling: time per token at top-k 1, 2,
+    4, and the shared expert added once at each).  For each k: moe_forward
+    timed with CUDA events over args.steps steps, the load-balance diagnostic
+    of its routing, and, with a shared expert, the largest deviation of
+    out(shared) - out(shared weights zeroed) from the shared expert alone,
+    relative to the shared expert's largest magnitude."""
+    import torch
+    from mixture_experts_layer_sqrt_b200 import binding as B, synth, workload as WL
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    arrays = synth.generate(p)
+    wt = WL.device_weights(p, arrays, dev)
+    w = B.make_weights(wt)
+    x = WL.to_torch(arrays["x"], dev)
+    mask = WL.to_torch(arrays.get("image_mask"), dev)
+    stream = torch.cuda.current_stream(dev)
+    rows = []
+    for k in ks:
+        q = p.with_(k=k)
+        cfg = WL.config_of(q)
+        ws = B.workspace(B.workspace_size(cfg, q.T), dev)
+        out = torch.empty((q.T, q.D), dtype=torch.float32, device=dev)
+        for _ in range(args.warmup):
+            B.forward(cfg, x, w, ws, mask, out)
+        counts = torch.empty(q.E, dtype=torch.int32, device=dev)
+        B.forward(cfg, x, w, ws, mask, out, expert_counts_out=counts)
+        torch.cuda.synchronize()
+        lb = load_balance(counts.cpu().numpy(), q.T, k, cfg.expert_capacity)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            B.forward(cfg, x, w, ws, mask, out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        B.check_device_status(ws)
+        ms = e0.elapsed_time(e1) / args.steps
+        row = {"k": k, "ms_per_step": ms, "us_per_token": ms * 1e3 / q.T, "tokens_per_s": q.T / (ms / 1e3),
+               "layer_flops": layer_flops(q, lb["kept"]), "load_balance": lb}
+        if q.Fs:
+            zero = dict(wt, sh_gate=torch.zeros_like(wt["sh_gate"]), sh_up=torch.zeros_like(wt["sh_up"]),
+                        sh_down=torch.zeros_like(wt["sh_down"]))
+            out0 = B.forward(cfg, x, B.make_weights(zero), ws, mask)
+            sh = shared_expert_alone(B, q, x, wt)
+            torch.cuda.synchronize()
+            row["shared_added_once_rel_err"] = float((out - out0 - sh).abs().max() / sh.abs().max())
+        rows.append(row)
+    return {"metric": "MoE fwd per-token time vs top-k", "unit": "us/token", "higher_is_better": False,
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "dtype": "f32" if p.act == "f32" else "bf16",
+            "data": "synthetic", "config": {"workload": describe(p), "top_k": list(ks)}, "sweep": rows}
 
 
 def run_e2e(args, B, WL, cfg, wt, arrays, T, D, dev, stream, dist):
@@ -346,6 +409,19 @@ def run_e2e(args, B, WL, cfg, wt, arrays, T, D, dev, stream, dist):
             "h2d_bytes_per_step": int(x_h.numel() * x_h.element_size() + (m_h.numel() if m_h is not None else 0)),
             "d2h_bytes_per_step": int(out_h[0].numel() * out_h[0].element_size()),
             "copies": "overlapped with compute on separate streams (forward_host_batches)"}
+
+
+def load_balance(counts, T: int, k: int, capacity: int = 0):
+    """Routing diagnostics from the per-expert assignment counts (before capacity):
+    the load-balance measure E * sum_e (count_e / (T k))^2 of the ops-transformer
+    MoE walkthrough (坑二: 1 when every expert gets T k / E assignments, E when
+    one expert gets them all), the kept rows after capacity and the drops."""
+    c = np.asarray(counts, dtype=np.int64)
+    E = len(c)
+    ratio = c / float(max(T * k, 1))
+    kept = int(np.minimum(c, capacity).sum()) if capacity else int(c.sum())
+    return {"loss": float(E * np.sum(ratio ** 2)), "kept": kept, "drops": int(T * k - kept),
+            "max_count": int(c.max()) if E else 0, "min_count": int(c.min()) if E else 0}
 
 
 # the stage intervals moe_forward_profiled brackets with its events
@@ -482,6 +558,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--sweep-k", default="", metavar="K1,K2,...",
+                    help="time the layer at each top-k on the workload's shape instead of the bench step")
     ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
                     help="override a workload field (e.g. T=1024, E=2) for a smaller profiling case")
     args = ap.parse_args()
@@ -508,6 +586,9 @@ def main():
     from mixture_experts_layer_sqrt_b200 import build
     build.build()
     import torch
+    if args.sweep_k:
+        emit(run_sweep(args, p, [int(v) for v in args.sweep_k.split(",")]), rank)
+        return
     if world > 1:
         import datetime
         import torch.distributed as dist

@@ -108,3 +108,17 @@ def test_permute_combine_bandwidth():
     pq = bench.permute_combine(q, 49152, stage_ms, {"hbm": 6000.0, "src": "test"})
     assert pq["combine"]["bytes"] == 49152 * 4096 * 4 + 2 * 8192 * 4096 * 4
     assert pq["gather"]["bytes"] == 2 * 49152 * 4096 * 2 + 4 * 49152
+
+
+def test_load_balance_diagnostic_hand_cases():
+    # perfectly balanced: T k / E each -> 1; one expert takes everything -> E
+    lb = bench.load_balance([4, 4, 4, 4], T=8, k=2)
+    assert lb["loss"] == pytest.approx(1.0) and lb["kept"] == 16 and lb["drops"] == 0
+    lb = bench.load_balance([16, 0, 0, 0], T=16, k=1)
+    assert lb["loss"] == pytest.approx(4.0) and lb["max_count"] == 16 and lb["min_count"] == 0
+    # 3 experts, T=3, k=2: counts 3,2,1 -> 3 * ((3/6)^2 + (2/6)^2 + (1/6)^2) = 3 * 14/36
+    lb = bench.load_balance([3, 2, 1], T=3, k=2)
+    assert lb["loss"] == pytest.approx(3 * 14 / 36)
+    # capacity 2: kept min(count, 2) = 2 + 2 + 1, the rest dropped
+    lb = bench.load_balance([3, 2, 1], T=3, k=2, capacity=2)
+    assert lb["kept"] == 5 and lb["drops"] == 1

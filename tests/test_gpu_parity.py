@@ -459,3 +459,34 @@ def test_zero_tokens(B, W):
     x0 = c.x[:0]
     out = B.forward(c.cfg, x0, c.w, ws)
     assert out.shape == (0, p.D)
+
+
+@pytest.mark.parametrize("k", [1, 2, 4])
+def test_shared_expert_added_once_each_k(B, W, k):
+    # at each top-k: the layer matches the oracle, and out(shared) minus
+    # out(shared weights zeroed) is the shared expert alone (added once, weight 1)
+    import bench
+    p = H.small("sqrt_fp4").with_(k=k)
+    c = Case(B, W, p)
+    ws = B.workspace(B.workspace_size(c.cfg, p.T))
+    idx = torch.empty((p.T, k), dtype=torch.int32, device="cuda")
+    out = B.forward(c.cfg, c.x, c.w, ws, c.mask, topk_idx_out=idx)
+    zero = dict(c.wt, sh_gate=torch.zeros_like(c.wt["sh_gate"]), sh_up=torch.zeros_like(c.wt["sh_up"]),
+                sh_down=torch.zeros_like(c.wt["sh_down"]))
+    out0 = B.forward(c.cfg, c.x, B.make_weights(zero), ws, c.mask)
+    sh = bench.shared_expert_alone(B, p, c.x, c.wt)
+    torch.cuda.synchronize()
+    B.check_device_status(ws)
+    # combine adds the shared row last to the same routed sum r: out = fl(r + sh),
+    # out0 = r, so out - out0 - sh is two fp32 roundings: <= 2^-22 (|r| + |sh|)
+    r, s_ = H.to_np(out0).astype(np.float64), H.to_np(sh).astype(np.float64)
+    err = np.abs(H.to_np(out).astype(np.float64) - r - s_)
+    assert np.all(err <= 2.0 ** -22 * (np.abs(r) + np.abs(s_)) + 1e-30), "shared expert not added exactly once"
+    idx_g = H.to_np(idx).astype(np.int64)
+    logits, idx_o, w_o, keys = H.oracle_route(p, c.L, c.a)
+    H.check_selection(idx_g, keys, k)
+    w_sel = O.route_weights(logits, idx_g, p.gate)
+    o = O.moe_forward(c.L.x(), logits, idx_g, w_sel, c.L.expert, p.E, 0, p.clamp, "preact", c.L.shared())
+    H.assert_close_layer(p, H.to_np(out), o["out"], "out")
+    o0 = O.moe_forward(c.L.x(), logits, idx_g, w_sel, c.L.expert, p.E, 0, p.clamp, "preact", None)
+    H.assert_close_layer(p, H.to_np(out0), o0["out"], "out without the shared expert")
