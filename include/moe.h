@@ -132,6 +132,19 @@ int moe_expert_capacity(int T, int top_k, int num_experts, int cf_num, int cf_de
 /* Kernels launched by this library in this process so far (diagnostic). */
 uint64_t moe_launch_count(void);
 
+/* 1 in the checked build of this library (libmoe_b200_checked.so, built with
+ * MOE_CHECKED), 0 otherwise.  In the checked build every kernel checks the
+ * indices it reads from its inputs before using them -- row maps against the
+ * token count, slot rows against T * k, expert offsets for a negative start or
+ * a decrease -- and on a failed check skips the access (a row it cannot read
+ * is left unwritten, a group with bad offsets does no work) and counts a
+ * violation; nothing traps.  A substitute for a device memory checker. */
+int moe_checked_build(void);
+
+/* Violations the checked build's kernels counted since the last call, then
+ * reset; always 0 in other builds.  Synchronises the current device. */
+uint64_t moe_checked_violations(void);
+
 /* Synchronises `stream`, then reads and clears the device status word at the
  * start of `ws` (any workspace passed to the calls above).  Returns MOE_OK or
  * MOE_ERR_DEVICE_TIMEOUT; MOE_ERR_CUDA if the stream reports an error. */
@@ -147,9 +160,7 @@ moe_status moe_selftest_wait_timeout(void *ws, size_t ws_bytes, moe_stream_t str
 
 /* ------------------------------------------------------------ stage 1: route */
 
-/* Bytes of workspace moe_route_topk needs: its device status word, plus for
- * E > 32 with bf16 activations (the tensor-core router) the fp32 logit rows
- * [T, E rounded up to 32] it hands to its selection kernel. */
+/* Bytes of workspace moe_route_topk needs: its device status word. */
 size_t moe_route_workspace_size(const MoEConfig *cfg, int T);
 
 /* Router GEMM + gate + top-k for T tokens (a1-a2).
@@ -161,11 +172,11 @@ size_t moe_route_workspace_size(const MoEConfig *cfg, int T);
  *   topk_w     [T, k] float out: the multipliers (renormalised softmax, or raw
  *              sqrt(softplus(s)), or raw sigmoid(s))
  *   ws         >= moe_route_workspace_size(cfg, T) bytes (status word)
- * Logits are accumulated in fp32 (ops-transformer walkthrough, 坑三).  With
- * E <= 32 (or fp32 activations) one kernel computes them on the CUDA cores
- * and selects from shared memory.  With bf16 activations and 32 < E <= 512
- * they are computed on the tensor cores and each token's logit row is stored
- * to the route workspace, from which a second kernel selects. */
+ * Logits are accumulated in fp32 (ops-transformer walkthrough, 坑三) and
+ * never leave the SM: with E <= 32 (or fp32 activations) one kernel computes
+ * them on the CUDA cores and selects from shared memory; with bf16
+ * activations and 32 < E <= 512 one kernel computes them on the tensor cores
+ * and each thread selects its token's top k straight out of TMEM. */
 moe_status moe_route_topk(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
                           const uint8_t *image_mask, int32_t *topk_idx, float *topk_w, void *ws,
                           size_t ws_bytes, moe_stream_t stream);
@@ -280,13 +291,21 @@ size_t moe_workspace_size(const MoEConfig *cfg, int T);
  *   topk_idx_out [T, k] int32 or NULL: copy of the routing decision
  *   expert_counts_out [E] int32 or NULL: assignments per expert before capacity
  *   ws: workspace of at least moe_workspace_size(cfg, T) bytes
- * No host synchronisation; per-expert counts never leave the device.
+ * No host synchronisation; per-expert counts never leave the device.  The
+ * kept count of expert e is min(expert_counts_out[e], C) (all of it when
+ * C = 0) and the layer drops T*k minus their sum.
  * Same kernels and results as the stage entry points called in order, with
- * one difference in operand format: for NVFP4 experts whose gate/up reduction
- * length D is a multiple of 256, the gate/up GEMM multiplies f16 operands
- * (x rows scaled by a power of two each, expanded FP4 weights) instead of
- * bf16 ones.  Both are exact, so the results are identical whenever every
- * element of a token row satisfies |x| >= max|row| * 2^-31 or x = 0. */
+ * two differences in how they are arranged:
+ *  - for NVFP4 experts whose gate/up reduction length D is a multiple of 256,
+ *    the gate/up GEMM multiplies f16 operands (x rows scaled by a power of two
+ *    each, expanded FP4 weights) instead of bf16 ones.  Both are exact, so the
+ *    results are identical whenever every element of a token row satisfies
+ *    |x| >= max|row| * 2^-31 or x = 0;
+ *  - with a shared expert whose GEMMs run on the tensor cores (bf16, D a
+ *    multiple of 256, F_s of 128), the combine is folded into the shared
+ *    expert's down GEMM: its epilogue adds each token's routed rows in slot
+ *    order and then its own row, the same sums in the same order as
+ *    moe_combine, and stores the layer output directly. */
 moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
                        const uint8_t *image_mask, void *out, int32_t *topk_idx_out,
                        int32_t *expert_counts_out, void *ws, size_t ws_bytes, moe_stream_t stream);
@@ -299,7 +318,9 @@ moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeig
  *   into x_perm (a5), [4] after the expert gate/up GEMM (a6), [5] after the
  *   down GEMM (a7), [6] after the shared expert (a8), [7] after combine (a9).
  * Each interval brackets exactly the kernels of its stage, so the elapsed
- * time between events i and i+1 is that stage's device time.
+ * time between events i and i+1 is that stage's device time.  When the
+ * combine is folded into the shared expert's down GEMM (see moe_forward),
+ * interval [6, 7] is empty and [5, 6] holds both.
  * n_events is 0 (then events may be NULL and this is moe_forward) or
  * MOE_STAGE_EVENTS; anything else is MOE_ERR_INVALID_ARG.  A failed event
  * record returns MOE_ERR_CUDA. */

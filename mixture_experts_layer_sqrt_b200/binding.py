@@ -15,6 +15,8 @@ from typing import Dict, Optional
 import torch
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+# the bounds-checking build (build.py --checked): same ABI, loaded only on request
+LIB_CHECKED_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200_checked.so")
 
 # enums (include/moe.h)
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE_TIMEOUT = range(6)
@@ -60,6 +62,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_version": (c_char_p, []),
         "moe_expert_capacity": (I, [I, I, I, I, I]),
         "moe_launch_count": (c_uint64, []),
+        "moe_checked_build": (I, []),
+        "moe_checked_violations": (c_uint64, []),
         "moe_check_device_status": (I, [P, P]),
         "moe_route_workspace_size": (S, [cfgp, I]),
         "moe_route_topk": (I, [cfgp, I, P, wp, P, P, P, P, S, P]),
@@ -87,7 +91,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 lib = load_library()
 
 # Every function the header declares (checked by the tests).
-EXPORTS = ("moe_status_string", "moe_version", "moe_expert_capacity", "moe_launch_count",
+EXPORTS = ("moe_status_string", "moe_version", "moe_expert_capacity", "moe_launch_count", "moe_checked_build",
+           "moe_checked_violations",
            "moe_check_device_status", "moe_route_workspace_size", "moe_route_topk", "moe_dispatch_workspace_size",
            "moe_dispatch", "moe_dispatch_noalloc", "moe_grouped_swiglu_workspace_size", "moe_expert_workspace_size",
            "moe_expert_gate_up", "moe_expert_down", "moe_grouped_swiglu", "moe_combine",

@@ -1,11 +1,15 @@
 """Builds libmoe_b200.so (sm_100a) in-tree with nvcc.
 
-    python -m mixture_experts_layer_sqrt_b200.build [--force] [--verbose]
+    python -m mixture_experts_layer_sqrt_b200.build [--force] [--verbose] [--checked]
 
 Each csrc/*.cu is compiled to an object under _build/ (skipped when newer than
 its sources and every header), then linked into
 mixture_experts_layer_sqrt_b200/libmoe_b200.so with the CUDA runtime linked
 statically, so the library needs only libc/libstdc++ to load.
+
+--checked builds the same sources with MOE_CHECKED defined (kernels check the
+indices they read and count violations instead of touching memory out of
+range) into _build_checked/ and libmoe_b200_checked.so.
 """
 from __future__ import annotations
 
@@ -23,6 +27,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libmoe_b200.so")
+BUILD_CHECKED = os.path.join(ROOT, "_build_checked")
+LIB_CHECKED = os.path.join(HERE, "libmoe_b200_checked.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3", "--expt-relaxed-constexpr",
@@ -48,17 +54,19 @@ def _stale(obj: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False, checked: bool = False) -> str:
     """Compile every kernel source and link the shared library; returns its path."""
-    os.makedirs(BUILD, exist_ok=True)
+    build_dir, lib = (BUILD_CHECKED, LIB_CHECKED) if checked else (BUILD, LIB)
+    flags = FLAGS + (["-DMOE_CHECKED=1"] if checked else [])
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdrs = _headers()
     cc = nvcc()
     jobs = []
     for s in srcs:
-        obj = os.path.join(BUILD, os.path.basename(s)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(s)[:-3] + ".o")
         if force or _stale(obj, [s] + hdrs):
-            cmd = [cc] + FLAGS + (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", s, "-o", obj]
+            cmd = [cc] + flags + (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", s, "-o", obj]
             jobs.append((s, cmd))
 
     def run(job):
@@ -75,16 +83,16 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
                 failed.append(s)
     if failed:
         raise RuntimeError("nvcc failed on: " + ", ".join(os.path.basename(f) for f in failed))
-    objs = [os.path.join(BUILD, os.path.basename(s)[:-3] + ".o") for s in srcs]
-    if force or jobs or _stale(LIB, objs):
-        cmd = [cc] + ARCH + ["-shared", "-cudart", "static", "-o", LIB + ".tmp"] + objs
+    objs = [os.path.join(build_dir, os.path.basename(s)[:-3] + ".o") for s in srcs]
+    if force or jobs or _stale(lib, objs):
+        cmd = [cc] + ARCH + ["-shared", "-cudart", "static", "-o", lib + ".tmp"] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if verbose or r.returncode != 0:
             sys.stderr.write(f"$ {' '.join(cmd)}\n{r.stdout}{r.stderr}")
         if r.returncode != 0:
-            raise RuntimeError("linking libmoe_b200.so failed")
-        os.replace(LIB + ".tmp", LIB)
-    return LIB
+            raise RuntimeError("linking " + os.path.basename(lib) + " failed")
+        os.replace(lib + ".tmp", lib)
+    return lib
 
 
 def main():
@@ -92,8 +100,9 @@ def main():
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas", action="store_true", help="print register / spill / smem usage")
+    ap.add_argument("--checked", action="store_true", help="the bounds-checking build (MOE_CHECKED)")
     a = ap.parse_args()
-    print(build(a.force, a.verbose, a.ptxas))
+    print(build(a.force, a.verbose, a.ptxas, a.checked))
 
 
 if __name__ == "__main__":

@@ -5,6 +5,8 @@
 
 #include <atomic>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -109,7 +111,7 @@ moe_status run_gate_up(const MoEConfig &c, int rows, const void *a, int a_rows, 
   }
   if (tc_shapes_ok(cc, c.intermediate_dim))
     return launch_gate_up_tc(cc, rows, a, a_rows, row_token, offsets, wg, wu, c.intermediate_dim, h, ws.status, s);
-  return launch_gate_up_simt(cc, rows, a, row_token, offsets, wg, wu, c.intermediate_dim, h, s);
+  return launch_gate_up_simt(cc, rows, a, a_rows, row_token, offsets, wg, wu, c.intermediate_dim, h, s);
 }
 
 moe_status run_down(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
@@ -140,6 +142,29 @@ moe_status run_experts(const MoEConfig &c, int rows, const void *a, int a_rows, 
   return run_down(c, rows, h, offsets, wd, sd, row_weight, y, ws, s);
 }
 
+// NVTX ranges around the whole layer and each of its stages, so a timeline
+// profiler shows which stage enqueued which kernels.  Without a profiler
+// attached the calls return at once.  The destructor closes whatever is still
+// open when a stage returns early.
+struct NvtxStages {
+  int depth = 0;
+  void enter(const char *name) {
+    nvtxRangePushA(name);
+    ++depth;
+  }
+  void leave() {
+    if (depth > 0) {
+      nvtxRangePop();
+      --depth;
+    }
+  }
+  ~NvtxStages() {
+    while (depth > 0) leave();
+  }
+};
+const char *const kStageNames[MOE_STAGE_EVENTS - 1] = {"moe.route", "moe.dispatch_maps", "moe.gather",
+                                                       "moe.gate_up", "moe.down", "moe.shared", "moe.combine"};
+
 // The shared expert viewed as a one-expert layer of width F_s in the act dtype.
 MoEConfig shared_cfg(const MoEConfig &c) {
   MoEConfig sc = c;
@@ -150,11 +175,19 @@ MoEConfig shared_cfg(const MoEConfig &c) {
   return sc;
 }
 
+// moe_forward folds the combine into the shared expert's down GEMM when that
+// GEMM runs on the tensor cores.
+bool combine_folded(const MoEConfig &c) {
+  if (!c.shared_intermediate_dim) return false;
+  const MoEConfig sc = shared_cfg(c);
+  return tc_shapes_ok(sc, sc.intermediate_dim);
+}
+
 // ---- whole-layer workspace
 struct ForwardWs {
   int *status;
   int32_t *topk_idx, *counts, *offsets, *slot_row, *row_token, *chunk_cnt;
-  float *topk_w, *row_weight, *row_scale, *route_logits;
+  float *topk_w, *row_weight, *row_scale;
   void *x_perm, *h, *y_perm, *sh_y;
   ExpertWs ex;
 };
@@ -171,14 +204,13 @@ ForwardWs carve_forward(Carve &cv, const MoEConfig &c, int T) {
   w.row_token = cv.take<int32_t>(Tk);
   w.row_weight = cv.take<float>(Tk);
   w.row_scale = gate_up_direct(c) ? cv.take<float>(Tk) : nullptr;
-  w.route_logits = cv.take<float>(route_scratch_floats(c, T));
   w.chunk_cnt = cv.take<int32_t>((size_t)num_chunks(T) * E);
   w.x_perm = cv.take<char>(Tk * D * as);
   size_t hrows = Tk * c.intermediate_dim;
   if ((size_t)T * c.shared_intermediate_dim > hrows) hrows = (size_t)T * c.shared_intermediate_dim;
   w.h = cv.take<char>(hrows * as);
   w.y_perm = cv.take<float>(Tk * D);
-  w.sh_y = c.shared_intermediate_dim ? cv.take<float>((size_t)T * D) : nullptr;
+  w.sh_y = (c.shared_intermediate_dim && !combine_folded(c)) ? cv.take<float>((size_t)T * D) : nullptr;
   w.ex.status = w.status;
   w.ex.wexp = carve_expert(cv, c, false).wexp;  // NVFP4 expansion space, if any projection needs it
   return w;
@@ -216,6 +248,13 @@ int moe_expert_capacity(int T, int top_k, int num_experts, int cf_num, int cf_de
 
 uint64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+int moe_checked_build(void) { return kChecked ? 1 : 0; }
+
+uint64_t moe_checked_violations(void) {
+  return (uint64_t)violations_dispatch() + violations_combine() + violations_gemm_tc() + violations_gemm_fp4() +
+         violations_gemm_simt();
+}
+
 moe_status moe_check_device_status(void *ws, moe_stream_t stream) {
   if (!ws) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
@@ -239,7 +278,6 @@ size_t moe_route_workspace_size(const MoEConfig *cfg, int T) {
   if (validate_cfg(cfg) != MOE_OK || T < 0) return 0;
   Carve cv(nullptr);
   cv.take<int>(kStatusBytes / sizeof(int));
-  cv.take<float>(route_scratch_floats(*cfg, T));
   return align_up(cv.off, 256);
 }
 
@@ -255,8 +293,7 @@ moe_status moe_route_topk(const MoEConfig *cfg, int T, const void *x, const MoEW
   if (!w || !ok_ptr(x) || !ok_ptr(w->w_router) || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
   Carve cv(ws);
   int *status = cv.take<int>(kStatusBytes / sizeof(int));
-  float *scratch = cv.take<float>(route_scratch_floats(*cfg, T));
-  return launch_route(*cfg, T, x, w->w_router, w->bias, w->bias_vl, image_mask, topk_idx, topk_w, status, scratch,
+  return launch_route(*cfg, T, x, w->w_router, w->bias, w->bias_vl, image_mask, topk_idx, topk_w, status,
                       (cudaStream_t)stream);
 }
 
@@ -410,14 +447,18 @@ static moe_status forward_impl(const MoEConfig *cfg, int T, const void *x, const
   int32_t *counts = expert_counts_out ? expert_counts_out : f.counts;
   const int rows = T * c.top_k;
   // stage boundary i: record events[i] when the caller asked for it
+  NvtxStages nvtx;
+  nvtx.enter("moe_forward");
   auto mark = [&](int i) -> moe_status {
+    if (i > 0) nvtx.leave();
+    if (i + 1 < MOE_STAGE_EVENTS) nvtx.enter(kStageNames[i]);
     if (events && events[i] && cudaEventRecord((cudaEvent_t)events[i], s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
   };
 
   if ((st = mark(0)) != MOE_OK) return st;
-  if ((st = launch_route(c, T, x, w->w_router, w->bias, w->bias_vl, image_mask, idx, f.topk_w, f.status,
-                         f.route_logits, s)) != MOE_OK)
+  if ((st = launch_route(c, T, x, w->w_router, w->bias, w->bias_vl, image_mask, idx, f.topk_w, f.status, s)) !=
+      MOE_OK)
     return st;
   if ((st = mark(1)) != MOE_OK) return st;
   // the row maps (histogram, scan, positions), then the row gather
@@ -444,14 +485,23 @@ static moe_status forward_impl(const MoEConfig *cfg, int T, const void *x, const
   if ((st = run_down(c, rows, f.h, f.offsets, w->w_down, w->s_down, f.row_weight, f.y_perm, f.ex, s)) != MOE_OK)
     return st;
   if ((st = mark(5)) != MOE_OK) return st;
+  // with a shared expert on the tensor cores, its down GEMM also sums each
+  // token's routed rows and stores the layer output (combine folded in)
+  const MoEConfig sc = shared_cfg(c);
+  const bool fold = combine_folded(c);
   if (c.shared_intermediate_dim) {
-    const MoEConfig sc = shared_cfg(c);
-    if ((st = run_experts(sc, T, x, T, nullptr, nullptr, w->sh_gate, w->sh_up, w->sh_down, nullptr, nullptr,
-                          nullptr, nullptr, f.h, f.sh_y, f.ex, s)) != MOE_OK)
+    if ((st = run_gate_up(sc, T, x, T, nullptr, nullptr, w->sh_gate, w->sh_up, nullptr, nullptr, f.h, f.ex, s)) !=
+        MOE_OK)
       return st;
+    if (fold)
+      st = launch_down_combine_tc(sc, T, f.h, nullptr, w->sh_down, sc.intermediate_dim, nullptr, out, f.ex.status,
+                                  (const float *)f.y_perm, f.slot_row, c.top_k, c.out_dtype == MOE_BF16, s);
+    else
+      st = run_down(sc, T, f.h, nullptr, w->sh_down, nullptr, nullptr, f.sh_y, f.ex, s);
+    if (st != MOE_OK) return st;
   }
   if ((st = mark(6)) != MOE_OK) return st;
-  if ((st = launch_combine(c, T, f.y_perm, f.slot_row, f.sh_y, out, s)) != MOE_OK) return st;
+  if (!fold && (st = launch_combine(c, T, f.y_perm, f.slot_row, f.sh_y, out, s)) != MOE_OK) return st;
   return mark(7);
 }
 

@@ -12,6 +12,9 @@
 #include "kernels.h"
 
 namespace moe {
+
+MOE_VIOLATION_COUNTER(violations_combine)
+
 namespace {
 
 constexpr int kCombineThreads = 128;  // small blocks: every SM holds 16, so the last wave is even
@@ -23,7 +26,7 @@ __device__ __forceinline__ void st_stream(float *p, float4 v) { __stcs(reinterpr
 // kK > 0: the layer's top-k fixed at compile time (rows held in registers, the
 // column loop unrolled with every row's load in flight); kK == 0: any k <= 16.
 template <typename TOut, int kK>
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(int T, int D, int k_rt,
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(int T, int D, int k_rt, int max_row,
                                                                   const float *__restrict__ y_perm,
                                                                   const int32_t *__restrict__ slot_row,
                                                                   const float *__restrict__ shared_y,
@@ -35,7 +38,11 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(int T, int D, 
   const int warps = gridDim.x * (blockDim.x >> 5);
   for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
     // the token's k rows: lane j < k loads slot j, then every lane gets all of them
-    const int my_row = lane < k ? slot_row[(long)t * k + lane] : -1;
+    int my_row = lane < k ? slot_row[(long)t * k + lane] : -1;
+    if (kChecked && my_row >= max_row) {  // rows of y_perm: at most T * k
+      note_violation();
+      my_row = -1;
+    }
     int rows[kMaxK];
 #pragma unroll
     for (int j = 0; j < kMaxK; ++j) rows[j] = __shfl_sync(0xffffffffu, my_row, j);
@@ -75,12 +82,12 @@ template <typename TOut>
 void launch_combine_k(int k, int blocks, int T, int D, const float *y, const int32_t *slot_row, const float *sh,
                       TOut *out, cudaStream_t s) {
   switch (k) {
-    case 1: combine_kernel<TOut, 1><<<blocks, kCombineThreads, 0, s>>>(T, D, k, y, slot_row, sh, out); break;
-    case 2: combine_kernel<TOut, 2><<<blocks, kCombineThreads, 0, s>>>(T, D, k, y, slot_row, sh, out); break;
-    case 4: combine_kernel<TOut, 4><<<blocks, kCombineThreads, 0, s>>>(T, D, k, y, slot_row, sh, out); break;
-    case 6: combine_kernel<TOut, 6><<<blocks, kCombineThreads, 0, s>>>(T, D, k, y, slot_row, sh, out); break;
-    case 8: combine_kernel<TOut, 8><<<blocks, kCombineThreads, 0, s>>>(T, D, k, y, slot_row, sh, out); break;
-    default: combine_kernel<TOut, 0><<<blocks, kCombineThreads, 0, s>>>(T, D, k, y, slot_row, sh, out); break;
+    case 1: combine_kernel<TOut, 1><<<blocks, kCombineThreads, 0, s>>>(T, D, k, T * k, y, slot_row, sh, out); break;
+    case 2: combine_kernel<TOut, 2><<<blocks, kCombineThreads, 0, s>>>(T, D, k, T * k, y, slot_row, sh, out); break;
+    case 4: combine_kernel<TOut, 4><<<blocks, kCombineThreads, 0, s>>>(T, D, k, T * k, y, slot_row, sh, out); break;
+    case 6: combine_kernel<TOut, 6><<<blocks, kCombineThreads, 0, s>>>(T, D, k, T * k, y, slot_row, sh, out); break;
+    case 8: combine_kernel<TOut, 8><<<blocks, kCombineThreads, 0, s>>>(T, D, k, T * k, y, slot_row, sh, out); break;
+    default: combine_kernel<TOut, 0><<<blocks, kCombineThreads, 0, s>>>(T, D, k, T * k, y, slot_row, sh, out); break;
   }
 }
 

@@ -33,6 +33,33 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
     if (_e != cudaSuccess) return MOE_ERR_CUDA;             \
   } while (0)
 
+// ---------------------------------------------------------- checked builds
+// Built with MOE_CHECKED (build.py --checked -> libmoe_b200_checked.so), the
+// kernels check the indices they read from their inputs (row maps, slot rows,
+// expert offsets) before using them: an index out of range skips the access
+// and counts a violation in the compiling file's device counter, which
+// moe_checked_violations() reads; nothing traps.  Other builds trust their
+// inputs and compile the checks away.
+#ifdef MOE_CHECKED
+constexpr bool kChecked = true;
+#else
+constexpr bool kChecked = false;
+#endif
+
+// One counter per source file (device variables are not shared between files
+// without relocatable device code); `reader` returns the count and clears it.
+#define MOE_VIOLATION_COUNTER(reader)                                                 \
+  namespace {                                                                         \
+  __device__ unsigned int g_violations;                                               \
+  __device__ __forceinline__ void note_violation() { atomicAdd(&g_violations, 1u); }  \
+  }                                                                                   \
+  unsigned int reader() {                                                             \
+    unsigned int h = 0, z = 0;                                                        \
+    if (cudaMemcpyFromSymbol(&h, g_violations, sizeof(h)) != cudaSuccess) return 0;   \
+    if (cudaMemcpyToSymbol(g_violations, &z, sizeof(z)) != cudaSuccess) return h;     \
+    return h;                                                                         \
+  }
+
 // ------------------------------------------------------------ element types
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }

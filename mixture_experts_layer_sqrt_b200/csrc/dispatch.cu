@@ -20,6 +20,9 @@
 #include "kernels.h"
 
 namespace moe {
+
+MOE_VIOLATION_COUNTER(violations_dispatch)
+
 namespace {
 
 constexpr int kThreads = 256;
@@ -195,14 +198,19 @@ template <typename TA>
 __global__ void __launch_bounds__(256) gather_kernel(int max_rows, int D,
                                                      const int32_t *__restrict__ expert_offsets,
                                                      int E, const int32_t *__restrict__ row_token,
-                                                     const TA *__restrict__ x,
+                                                     const TA *__restrict__ x, int src_rows,
                                                      TA *__restrict__ x_perm) {
   constexpr int V = Vec16<TA>::N;
   const int R = min(expert_offsets[E], max_rows);
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (blockDim.x >> 5);
   for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += warps) {
-    const TA *src = x + (long)row_token[r] * D;
+    const int tok = row_token[r];
+    if (kChecked && (unsigned)tok >= (unsigned)src_rows) {  // whole warp: same row
+      if (lane == 0) note_violation();
+      continue;
+    }
+    const TA *src = x + (long)tok * D;
     TA *dst = x_perm + (long)r * D;
 #pragma unroll 8
     for (int c = lane * V; c < D; c += 32 * V) store16(dst + c, load16(src + c));
@@ -218,14 +226,19 @@ __global__ void __launch_bounds__(256) gather_kernel(int max_rows, int D,
 __global__ void __launch_bounds__(256) gather_f16_kernel(int max_rows, int D,
                                                          const int32_t *__restrict__ expert_offsets, int E,
                                                          const int32_t *__restrict__ row_token,
-                                                         const __nv_bfloat16 *__restrict__ x,
+                                                         const __nv_bfloat16 *__restrict__ x, int src_rows,
                                                          __half *__restrict__ x_perm, float *__restrict__ row_scale) {
   constexpr int V = 8;
   const int R = min(expert_offsets[E], max_rows);
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (blockDim.x >> 5);
   for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += warps) {
-    const __nv_bfloat16 *src = x + (long)row_token[r] * D;
+    const int tok = row_token[r];
+    if (kChecked && (unsigned)tok >= (unsigned)src_rows) {  // whole warp: same row
+      if (lane == 0) note_violation();
+      continue;
+    }
+    const __nv_bfloat16 *src = x + (long)tok * D;
     float m = 0.0f;
 #pragma unroll 8
     for (int c = lane * V; c < D; c += 32 * V) {
@@ -269,7 +282,7 @@ moe_status launch_gather_f16(const MoEConfig &c, int T, const int32_t *expert_of
   MOE_CUDA_TRY(cudaGetDevice(&dev));
   MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   gather_f16_kernel<<<sms * 8, 256, 0, s>>>(T * c.top_k, c.hidden_dim, expert_offsets, c.num_experts, row_token,
-                                            (const __nv_bfloat16 *)x, (__half *)x_perm, row_scale);
+                                            (const __nv_bfloat16 *)x, T, (__half *)x_perm, row_scale);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
@@ -309,10 +322,10 @@ moe_status launch_gather(const MoEConfig &c, int T, const int32_t *expert_offset
   const int max_rows = T * c.top_k, E = c.num_experts;
   if (c.act_dtype == MOE_F32) {
     gather_kernel<float><<<sms * 8, 256, 0, s>>>(max_rows, c.hidden_dim, expert_offsets, E, row_token,
-                                                 (const float *)x, (float *)x_perm);
+                                                 (const float *)x, T, (float *)x_perm);
   } else {
     gather_kernel<__nv_bfloat16><<<sms * 8, 256, 0, s>>>(max_rows, c.hidden_dim, expert_offsets, E,
-                                                         row_token, (const __nv_bfloat16 *)x,
+                                                         row_token, (const __nv_bfloat16 *)x, T,
                                                          (__nv_bfloat16 *)x_perm);
   }
   MOE_LAUNCH_CHECK();

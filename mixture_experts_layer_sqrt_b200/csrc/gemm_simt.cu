@@ -14,6 +14,9 @@
 #include "kernels.h"
 
 namespace moe {
+
+MOE_VIOLATION_COUNTER(violations_gemm_simt)
+
 namespace {
 
 constexpr int BM = 64, BN = 64, BK = 16;
@@ -22,7 +25,7 @@ template <typename TIn, typename TOut, bool GATED>
 __global__ void __launch_bounds__(256) grouped_gemm_simt(int rows, int K, int N,
                                                          const int32_t *__restrict__ offsets, int E,
                                                          const int32_t *__restrict__ row_token,
-                                                         const TIn *__restrict__ A,
+                                                         int src_rows, const TIn *__restrict__ A,
                                                          const TIn *__restrict__ B0,
                                                          const TIn *__restrict__ B1, float clamp,
                                                          int clamp_mode,
@@ -44,6 +47,10 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt(int rows, int K, int N,
     int acc = 0;
     for (int ee = 0; ee < E; ++ee) {
       int s0 = offsets[ee], s1 = offsets[ee + 1];
+      if (kChecked && (s0 < 0 || s1 < s0)) {  // offsets must not decrease or start below 0
+        if (threadIdx.x == 0) note_violation();
+        return;
+      }
       int nt = (s1 - s0 + BM - 1) / BM;
       if (mt < acc + nt) {
         e = ee;
@@ -69,8 +76,13 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt(int rows, int K, int N,
       int idx = threadIdx.x + 256 * q;
       int r = idx / BK, kk = idx % BK;
       int gr = m0 + r, gk = k0 + kk;
-      const long ar = (gr < seg_end && row_token) ? (long)row_token[gr] : (long)gr;  // gathered A row
-      As[kk][r] = (gr < seg_end && gk < K) ? to_f32(A[ar * K + gk]) : 0.0f;
+      long ar = (gr < seg_end && row_token) ? (long)row_token[gr] : (long)gr;  // gathered A row
+      bool a_ok = gr < seg_end && gk < K;
+      if (kChecked && a_ok && row_token && (unsigned long)ar >= (unsigned long)src_rows) {
+        if (kk == 0) note_violation();
+        a_ok = false;
+      }
+      As[kk][r] = a_ok ? to_f32(A[ar * K + gk]) : 0.0f;
       int gn = n0 + r;
       Bs0[kk][r] = (gn < N && gk < K) ? to_f32(Be0[(long)gn * K + gk]) : 0.0f;
       if (GATED) Bs1[kk][r] = (gn < N && gk < K) ? to_f32(Be1[(long)gn * K + gk]) : 0.0f;
@@ -115,28 +127,30 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt(int rows, int K, int N,
 }
 
 template <typename TIn, typename TOut, bool GATED>
-void launch_one(int rows, int K, int N, const int32_t *offsets, int E, const int32_t *row_token, const void *A,
+void launch_one(int rows, int K, int N, const int32_t *offsets, int E, const int32_t *row_token, int src_rows,
+                const void *A,
                 const void *B0, const void *B1, float clamp, int clamp_mode,
                 const float *row_weight, void *out, cudaStream_t s) {
   long mt = (rows + BM - 1) / BM + (offsets ? E : 0);
   dim3 grid((unsigned)mt, (N + BN - 1) / BN);
-  grouped_gemm_simt<TIn, TOut, GATED><<<grid, 256, 0, s>>>(rows, K, N, offsets, E, row_token, (const TIn *)A,
+  grouped_gemm_simt<TIn, TOut, GATED><<<grid, 256, 0, s>>>(rows, K, N, offsets, E, row_token, src_rows,
+                                                           (const TIn *)A,
                                                            (const TIn *)B0, (const TIn *)B1, clamp,
                                                            clamp_mode, row_weight, (TOut *)out);
 }
 
 }  // namespace
 
-moe_status launch_gate_up_simt(const MoEConfig &c, int rows, const void *a, const int32_t *row_token,
-                               const int32_t *offsets, const void *w_gate, const void *w_up,
-                               int F, void *h, cudaStream_t s) {
+moe_status launch_gate_up_simt(const MoEConfig &c, int rows, const void *a, int a_rows,
+                               const int32_t *row_token, const int32_t *offsets, const void *w_gate,
+                               const void *w_up, int F, void *h, cudaStream_t s) {
   if (rows == 0) return MOE_OK;
   const int E = offsets ? c.num_experts : 1;
   if (c.act_dtype == MOE_F32)
-    launch_one<float, float, true>(rows, c.hidden_dim, F, offsets, E, row_token, a, w_gate, w_up,
+    launch_one<float, float, true>(rows, c.hidden_dim, F, offsets, E, row_token, a_rows, a, w_gate, w_up,
                                    c.swiglu_clamp, c.clamp_mode, nullptr, h, s);
   else
-    launch_one<__nv_bfloat16, __nv_bfloat16, true>(rows, c.hidden_dim, F, offsets, E, row_token, a, w_gate,
+    launch_one<__nv_bfloat16, __nv_bfloat16, true>(rows, c.hidden_dim, F, offsets, E, row_token, a_rows, a, w_gate,
                                                    w_up, c.swiglu_clamp, c.clamp_mode, nullptr, h, s);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
@@ -148,10 +162,10 @@ moe_status launch_down_simt(const MoEConfig &c, int rows, const void *h, const i
   if (rows == 0) return MOE_OK;
   const int E = offsets ? c.num_experts : 1;
   if (c.act_dtype == MOE_F32)
-    launch_one<float, float, false>(rows, F, c.hidden_dim, offsets, E, nullptr, h, w_down, nullptr, 0.0f, 0,
+    launch_one<float, float, false>(rows, F, c.hidden_dim, offsets, E, nullptr, rows, h, w_down, nullptr, 0.0f, 0,
                                     row_weight, y, s);
   else
-    launch_one<__nv_bfloat16, float, false>(rows, F, c.hidden_dim, offsets, E, nullptr, h, w_down, nullptr,
+    launch_one<__nv_bfloat16, float, false>(rows, F, c.hidden_dim, offsets, E, nullptr, rows, h, w_down, nullptr,
                                             0.0f, 0, row_weight, y, s);
   MOE_LAUNCH_CHECK();
   return MOE_OK;

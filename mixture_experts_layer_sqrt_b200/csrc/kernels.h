@@ -15,18 +15,16 @@ inline int num_chunks(int T) { return (T + kChunkTokens - 1) / kChunkTokens; }
 
 // route.cu ---------------------------------------------------------------
 // Picks the tensor-core router (route_tc.cu) when route_tc_ok(c), else CUDA
-// cores.  scratch: route_scratch_floats(c, T) floats (null when that is 0).
+// cores.  status: the workspace's device status word (bounded waits).
 moe_status launch_route(const MoEConfig &c, int T, const void *x, const void *w_router,
                         const float *bias, const float *bias_vl, const uint8_t *image_mask,
-                        int32_t *topk_idx, float *topk_w, int *status, float *scratch, cudaStream_t s);
+                        int32_t *topk_idx, float *topk_w, int *status, cudaStream_t s);
 
 // route_tc.cu ------------------------------------------------------------
 bool route_tc_ok(const MoEConfig &c);
-// fp32 logit rows [T, E_pad] the tensor-core router stores for its selection pass
-size_t route_scratch_floats(const MoEConfig &c, int T);
 moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void *w_router, const float *bias,
                            const float *bias_vl, const uint8_t *image_mask, int32_t *topk_idx, float *topk_w,
-                           int *status, float *scratch, cudaStream_t s);
+                           int *status, cudaStream_t s);
 
 // dispatch.cu ------------------------------------------------------------
 // chunk_cnt: [num_chunks(T), E] int32 scratch.  x_perm may be null: the row
@@ -48,9 +46,9 @@ moe_status launch_gather_f16(const MoEConfig &c, int T, const int32_t *expert_of
 // gemm_simt.cu -----------------------------------------------------------
 // Grouped GEMMs on CUDA cores (fp32 FMA), any shape.  act: F32 or BF16 for
 // activations and weights alike.
-moe_status launch_gate_up_simt(const MoEConfig &c, int rows, const void *a, const int32_t *row_token,
-                               const int32_t *offsets, const void *w_gate, const void *w_up,
-                               int F, void *h, cudaStream_t s);
+moe_status launch_gate_up_simt(const MoEConfig &c, int rows, const void *a, int a_rows,
+                               const int32_t *row_token, const int32_t *offsets, const void *w_gate,
+                               const void *w_up, int F, void *h, cudaStream_t s);
 moe_status launch_down_simt(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
                             const void *w_down, int F, const float *row_weight, void *y,
                             cudaStream_t s);
@@ -67,6 +65,15 @@ moe_status launch_gate_up_tc(const MoEConfig &c, int rows, const void *a, int a_
 moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
                           const void *w_down, int F, const float *row_weight, float *y, int *status,
                           cudaStream_t s);
+// The down GEMM of one group whose rows are the layer's T tokens (the shared
+// expert) with the combine folded into its epilogue: out[t] = (sum over j of
+// comb_y[comb_slot[t, j]], j = 0..comb_k-1, dropped slots skipped) + this
+// GEMM's row t, in that order -- the same sums as launch_combine with this
+// GEMM's output as shared_y.  comb_y null: the plain down GEMM into (float *)out.
+moe_status launch_down_combine_tc(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
+                                  const void *w_down, int F, const float *row_weight, void *out, int *status,
+                                  const float *comb_y, const int32_t *comb_slot, int comb_k, bool comb_bf16,
+                                  cudaStream_t s);
 
 // gemm_fp4.cu ------------------------------------------------------------
 // The same projections with NVFP4 weights read in their packed form (codes
@@ -84,6 +91,14 @@ moe_status launch_down_fp4(const MoEConfig &c, int rows, const void *h, const in
 
 // One block whose bounded wait never completes: records the timeout status.
 moe_status launch_wait_selftest(int *status, cudaStream_t s);
+
+// Violation counters of the checked build, one per file that checks (each
+// returns its count and clears it; always 0 in other builds).
+unsigned int violations_dispatch();
+unsigned int violations_combine();
+unsigned int violations_gemm_tc();
+unsigned int violations_gemm_fp4();
+unsigned int violations_gemm_simt();
 
 // dequant.cu -------------------------------------------------------------
 // n_elems values (a multiple of 16): packed [n/2] bytes + scales [n/16] -> bf16 [n].

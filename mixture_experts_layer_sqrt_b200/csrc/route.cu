@@ -143,10 +143,9 @@ moe_status launch_route_t(const MoEConfig &c, int T, const void *x, const void *
 
 moe_status launch_route(const MoEConfig &c, int T, const void *x, const void *w_router,
                         const float *bias, const float *bias_vl, const uint8_t *image_mask,
-                        int32_t *topk_idx, float *topk_w, int *status, float *scratch, cudaStream_t s) {
+                        int32_t *topk_idx, float *topk_w, int *status, cudaStream_t s) {
   if (T == 0) return MOE_OK;
-  if (route_tc_ok(c))
-    return launch_route_tc(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, status, scratch, s);
+  if (route_tc_ok(c)) return launch_route_tc(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, status, s);
   // CUDA cores: 4 tokens x 8 experts per lane and pass; 2-warp blocks keep
   // the grid several blocks per SM deep at a few thousand tokens
   if (c.act_dtype == MOE_F32)

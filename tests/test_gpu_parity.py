@@ -350,10 +350,10 @@ def test_binding_rejects_mismatched_out(B, W):
 
 @pytest.mark.parametrize("name", ["sqrt_fp4_pair", "sqrt_fp4"])
 def test_fp4_direct_matches_expanded_weights(B, W, name):
-    # NVFP4 codes converted to bf16 in shared memory give the MMA the same
-    # operand bits as weights expanded beforehand (every e2m1 * e4m3 product is
-    # exact in bf16): bit for bit the bf16 GEMM (same 128-row tiles) on the
-    # expanded weights
+    # NVFP4 codes expanded on chip (into TMEM, the MMA's A operand) give the
+    # MMA the same operand bits as weights expanded beforehand (every e2m1 *
+    # e4m3 product is exact in bf16), and the k-blocks are accumulated in the
+    # same order: bit for bit the bf16 GEMM on the expanded weights
     p = H.small(name)
     c = Case(B, W, p)
     idx, w = B.route_topk(c.cfg, c.x, c.w, c.mask)
