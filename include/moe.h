@@ -27,7 +27,9 @@
  *    synchronously, before anything is enqueued.  Device-side errors (a
  *    bounded wait inside a kernel that gave up) are recorded in the status
  *    word at the start of `ws`; read them with moe_check_device_status().
- *  - Nothing is kept between calls: no global state besides a launch counter.
+ *  - Nothing about a layer is kept between calls.  The library's only global
+ *    state is a launch counter, the fixed scratch array of
+ *    moe_dispatch_noalloc and, in the checked build, its violation counters.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
