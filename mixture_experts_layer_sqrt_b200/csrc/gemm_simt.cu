@@ -44,13 +44,16 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt(int rows, int K, int N,
     seg_end = rows;
     if (m0 >= rows) return;
   } else {
+    if (kChecked) {  // offsets must not start below 0 or decrease: otherwise no block does any work
+      for (int ee = 0; ee < E; ++ee)
+        if (offsets[ee] < 0 || offsets[ee + 1] < offsets[ee]) {
+          if (threadIdx.x == 0 && mt == 0 && blockIdx.y == 0) note_violation();
+          return;
+        }
+    }
     int acc = 0;
     for (int ee = 0; ee < E; ++ee) {
       int s0 = offsets[ee], s1 = offsets[ee + 1];
-      if (kChecked && (s0 < 0 || s1 < s0)) {  // offsets must not decrease or start below 0
-        if (threadIdx.x == 0) note_violation();
-        return;
-      }
       int nt = (s1 - s0 + BM - 1) / BM;
       if (mt < acc + nt) {
         e = ee;
