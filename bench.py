@@ -428,12 +428,6 @@ def load_balance(counts, T: int, k: int, capacity: int = 0):
 STAGES = ["route", "dispatch_maps", "gather", "gate_up", "down", "shared", "combine"]
 
 
-def combine_folded(p) -> bool:
-    """moe_forward folds the combine into the shared expert's down GEMM when
-    that GEMM runs on the tensor cores (bf16, D % 256 == 0, F_s % 128 == 0)."""
-    return bool(p.Fs) and p.act == "bf16" and p.D % 256 == 0 and p.Fs % 128 == 0
-
-
 def permute_combine(p, rows: int, stage_ms, peaks):
     """Achieved HBM bandwidth of the two data-movement stages, from their
     algorithmic bytes and their stage event times:
@@ -445,11 +439,6 @@ def permute_combine(p, rows: int, stage_ms, peaks):
     g_bytes = 2.0 * rows * p.D * a + (4.0 * rows if p.wdtype == "nvfp4" else 0.0)
     out = {}
     for name, b in (("gather", g_bytes), ("combine", 4.0 * rows * p.D + 4.0 * p.T * p.D * (2 if p.Fs else 1))):
-        if name == "combine" and combine_folded(p):
-            # the shared expert's down GEMM sums the routed rows: no separate launch
-            out[name] = {"folded_into": "shared expert down GEMM epilogue", "ms": stage_ms[name],
-                         "bytes": 4.0 * rows * p.D + 4.0 * p.T * p.D}
-            continue
         ms = stage_ms[name]
         gbs = b / (ms / 1e3) / 1e9 if ms > 0 else None
         out[name] = {"bytes": b, "ms": ms, "gbs": gbs, "frac": gbs / peaks["hbm"] if gbs else None}

@@ -297,17 +297,11 @@ size_t moe_workspace_size(const MoEConfig *cfg, int T);
  * kept count of expert e is min(expert_counts_out[e], C) (all of it when
  * C = 0) and the layer drops T*k minus their sum.
  * Same kernels and results as the stage entry points called in order, with
- * two differences in how they are arranged:
- *  - for NVFP4 experts whose gate/up reduction length D is a multiple of 256,
- *    the gate/up GEMM multiplies f16 operands (x rows scaled by a power of two
- *    each, expanded FP4 weights) instead of bf16 ones.  Both are exact, so the
- *    results are identical whenever every element of a token row satisfies
- *    |x| >= max|row| * 2^-31 or x = 0;
- *  - with a shared expert whose GEMMs run on the tensor cores (bf16, D a
- *    multiple of 256, F_s of 128), the combine is folded into the shared
- *    expert's down GEMM: its epilogue adds each token's routed rows in slot
- *    order and then its own row, the same sums in the same order as
- *    moe_combine, and stores the layer output directly. */
+ * one difference in operand format: for NVFP4 experts whose gate/up reduction
+ * length D is a multiple of 256, the gate/up GEMM multiplies f16 operands
+ * (x rows scaled by a power of two each, expanded FP4 weights) instead of
+ * bf16 ones.  Both are exact, so the results are identical whenever every
+ * element of a token row satisfies |x| >= max|row| * 2^-31 or x = 0. */
 moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
                        const uint8_t *image_mask, void *out, int32_t *topk_idx_out,
                        int32_t *expert_counts_out, void *ws, size_t ws_bytes, moe_stream_t stream);
@@ -320,9 +314,7 @@ moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeig
  *   into x_perm (a5), [4] after the expert gate/up GEMM (a6), [5] after the
  *   down GEMM (a7), [6] after the shared expert (a8), [7] after combine (a9).
  * Each interval brackets exactly the kernels of its stage, so the elapsed
- * time between events i and i+1 is that stage's device time.  When the
- * combine is folded into the shared expert's down GEMM (see moe_forward),
- * interval [6, 7] is empty and [5, 6] holds both.
+ * time between events i and i+1 is that stage's device time.
  * n_events is 0 (then events may be NULL and this is moe_forward) or
  * MOE_STAGE_EVENTS; anything else is MOE_ERR_INVALID_ARG.  A failed event
  * record returns MOE_ERR_CUDA. */

@@ -175,13 +175,6 @@ MoEConfig shared_cfg(const MoEConfig &c) {
   return sc;
 }
 
-// moe_forward folds the combine into the shared expert's down GEMM when that
-// GEMM runs on the tensor cores.
-bool combine_folded(const MoEConfig &c) {
-  if (!c.shared_intermediate_dim) return false;
-  const MoEConfig sc = shared_cfg(c);
-  return tc_shapes_ok(sc, sc.intermediate_dim);
-}
 
 // ---- whole-layer workspace
 struct ForwardWs {
@@ -210,7 +203,7 @@ ForwardWs carve_forward(Carve &cv, const MoEConfig &c, int T) {
   if ((size_t)T * c.shared_intermediate_dim > hrows) hrows = (size_t)T * c.shared_intermediate_dim;
   w.h = cv.take<char>(hrows * as);
   w.y_perm = cv.take<float>(Tk * D);
-  w.sh_y = (c.shared_intermediate_dim && !combine_folded(c)) ? cv.take<float>((size_t)T * D) : nullptr;
+  w.sh_y = c.shared_intermediate_dim ? cv.take<float>((size_t)T * D) : nullptr;
   w.ex.status = w.status;
   w.ex.wexp = carve_expert(cv, c, false).wexp;  // NVFP4 expansion space, if any projection needs it
   return w;
@@ -485,23 +478,14 @@ static moe_status forward_impl(const MoEConfig *cfg, int T, const void *x, const
   if ((st = run_down(c, rows, f.h, f.offsets, w->w_down, w->s_down, f.row_weight, f.y_perm, f.ex, s)) != MOE_OK)
     return st;
   if ((st = mark(5)) != MOE_OK) return st;
-  // with a shared expert on the tensor cores, its down GEMM also sums each
-  // token's routed rows and stores the layer output (combine folded in)
-  const MoEConfig sc = shared_cfg(c);
-  const bool fold = combine_folded(c);
   if (c.shared_intermediate_dim) {
-    if ((st = run_gate_up(sc, T, x, T, nullptr, nullptr, w->sh_gate, w->sh_up, nullptr, nullptr, f.h, f.ex, s)) !=
-        MOE_OK)
+    const MoEConfig sc = shared_cfg(c);
+    if ((st = run_experts(sc, T, x, T, nullptr, nullptr, w->sh_gate, w->sh_up, w->sh_down, nullptr, nullptr,
+                          nullptr, nullptr, f.h, f.sh_y, f.ex, s)) != MOE_OK)
       return st;
-    if (fold)
-      st = launch_down_combine_tc(sc, T, f.h, nullptr, w->sh_down, sc.intermediate_dim, nullptr, out, f.ex.status,
-                                  (const float *)f.y_perm, f.slot_row, c.top_k, c.out_dtype == MOE_BF16, s);
-    else
-      st = run_down(sc, T, f.h, nullptr, w->sh_down, nullptr, nullptr, f.sh_y, f.ex, s);
-    if (st != MOE_OK) return st;
   }
   if ((st = mark(6)) != MOE_OK) return st;
-  if (!fold && (st = launch_combine(c, T, f.y_perm, f.slot_row, f.sh_y, out, s)) != MOE_OK) return st;
+  if ((st = launch_combine(c, T, f.y_perm, f.slot_row, f.sh_y, out, s)) != MOE_OK) return st;
   return mark(7);
 }
 

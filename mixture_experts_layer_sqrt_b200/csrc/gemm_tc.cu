@@ -99,13 +99,6 @@ struct Params {
   float clamp;
   int clamp_mode;
   int *status;
-  // down of a single group whose rows are the layer's tokens (the shared
-  // expert), with the combine folded into the epilogue: out[t] = (sum over
-  // j of comb_y[comb_slot[t, j]]) + this GEMM's row, summed in that order
-  const float *comb_y;       // y_perm [>= R, N] fp32, or null: a plain down GEMM
-  const int32_t *comb_slot;  // slot_row [rows, comb_k], -1 = dropped
-  int comb_k;
-  int comb_bf16;             // out in bf16 (else fp32)
 };
 
 template <bool PAIR>
@@ -425,52 +418,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
           }
         }
-      } else if (p.comb_y) {
-        // combine: the token's routed rows in slot order, then this row
-        const int ncol0 = tl.n_blk * BN;
-        int slot[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          slot[j] = (live && j < p.comb_k) ? p.comb_slot[(long)row * p.comb_k + j] : -1;
-          if (kChecked && slot[j] >= p.rows * p.comb_k) {  // rows of comb_y: at most T * k
-            note_violation();
-            slot[j] = -1;
-          }
-        }
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t v[32];
-          ptx::tmem_ld32(tbase + c, v);
-          ptx::tmem_ld_wait();
-          if (live) {
-#pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-              const long col = ncol0 + c + 4 * q4;
-#pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                if (slot[j] >= 0) {
-                  const float4 y = __ldcs(reinterpret_cast<const float4 *>(p.comb_y + (long)slot[j] * p.N + col));
-                  a.x += y.x;
-                  a.y += y.y;
-                  a.z += y.z;
-                  a.w += y.w;
-                }
-              }
-              a.x += __uint_as_float(v[4 * q4]);
-              a.y += __uint_as_float(v[4 * q4 + 1]);
-              a.z += __uint_as_float(v[4 * q4 + 2]);
-              a.w += __uint_as_float(v[4 * q4 + 3]);
-              if (p.comb_bf16) {
-                __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
-                *reinterpret_cast<uint2 *>((__nv_bfloat16 *)p.out + (long)row * p.N + col) =
-                    make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
-              } else {
-                __stcs(reinterpret_cast<float4 *>((float *)p.out + (long)row * p.N + col), a);
-              }
-            }
-          }
-        }
       } else {
         const int ncol0 = tl.n_blk * BN;
         const float rw = (live && p.row_weight) ? p.row_weight[row] : 1.0f;
@@ -624,10 +571,6 @@ moe_status launch_gate_up_tc(const MoEConfig &c, int rows, const void *a, int a_
   p.clamp = c.swiglu_clamp;
   p.clamp_mode = c.clamp_mode;
   p.status = status;
-  p.comb_y = nullptr;
-  p.comb_slot = nullptr;
-  p.comb_k = 0;
-  p.comb_bf16 = 0;
   if (use_pair(rows, p.E, true)) return launch_tc<true, true>(p, a, w_gate, w_up, F, s);
   return launch_tc<true, false>(p, a, w_gate, w_up, F, s);
 }
@@ -635,13 +578,6 @@ moe_status launch_gate_up_tc(const MoEConfig &c, int rows, const void *a, int a_
 moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
                           const void *w_down, int F, const float *row_weight, float *y, int *status,
                           cudaStream_t s) {
-  return launch_down_combine_tc(c, rows, h, offsets, w_down, F, row_weight, y, status, nullptr, nullptr, 0, false, s);
-}
-
-moe_status launch_down_combine_tc(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
-                                  const void *w_down, int F, const float *row_weight, void *out, int *status,
-                                  const float *comb_y, const int32_t *comb_slot, int comb_k, bool comb_bf16,
-                                  cudaStream_t s) {
   if (rows == 0) return MOE_OK;
   Params p;
   p.rows = rows;
@@ -652,15 +588,11 @@ moe_status launch_down_combine_tc(const MoEConfig &c, int rows, const void *h, c
   p.E = offsets ? c.num_experts : 1;
   p.n_tiles = c.hidden_dim / BN;
   p.offsets = offsets;
-  p.out = out;
+  p.out = y;
   p.row_weight = row_weight;
   p.clamp = 0.0f;
   p.clamp_mode = 0;
   p.status = status;
-  p.comb_y = comb_y;
-  p.comb_slot = comb_slot;
-  p.comb_k = comb_k;
-  p.comb_bf16 = comb_bf16 ? 1 : 0;
   if (use_pair(rows, p.E, false)) return launch_tc<false, true>(p, h, w_down, nullptr, c.hidden_dim, s);
   return launch_tc<false, false>(p, h, w_down, nullptr, c.hidden_dim, s);
 }

@@ -65,15 +65,6 @@ moe_status launch_gate_up_tc(const MoEConfig &c, int rows, const void *a, int a_
 moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
                           const void *w_down, int F, const float *row_weight, float *y, int *status,
                           cudaStream_t s);
-// The down GEMM of one group whose rows are the layer's T tokens (the shared
-// expert) with the combine folded into its epilogue: out[t] = (sum over j of
-// comb_y[comb_slot[t, j]], j = 0..comb_k-1, dropped slots skipped) + this
-// GEMM's row t, in that order -- the same sums as launch_combine with this
-// GEMM's output as shared_y.  comb_y null: the plain down GEMM into (float *)out.
-moe_status launch_down_combine_tc(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
-                                  const void *w_down, int F, const float *row_weight, void *out, int *status,
-                                  const float *comb_y, const int32_t *comb_slot, int comb_k, bool comb_bf16,
-                                  cudaStream_t s);
 
 // gemm_fp4.cu ------------------------------------------------------------
 // The same projections with NVFP4 weights read in their packed form (codes

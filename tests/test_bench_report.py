@@ -103,9 +103,8 @@ def test_permute_combine_bandwidth():
     assert pc["combine"]["bytes"] == 8192 * 4096 * 4 + 4096 * 4096 * 4
     assert pc["gather"]["gbs"] == pytest.approx(pc["gather"]["bytes"] / 0.02e-3 / 1e9)
     assert pc["combine"]["frac"] == pytest.approx(pc["combine"]["gbs"] / 6000.0)
-    # the shared expert's fp32 row is read by combine too (when not folded); NVFP4 rows carry a scale each
-    q = synth.PROBLEMS["sqrt_fp4"].with_(Fs=2000)
-    assert not bench.combine_folded(q)
+    # the shared expert's fp32 row is read by combine too; NVFP4 rows carry a scale each
+    q = synth.PROBLEMS["sqrt_fp4"]
     pq = bench.permute_combine(q, 49152, stage_ms, {"hbm": 6000.0, "src": "test"})
     assert pq["combine"]["bytes"] == 49152 * 4096 * 4 + 2 * 8192 * 4096 * 4
     assert pq["gather"]["bytes"] == 2 * 49152 * 4096 * 2 + 4 * 49152
@@ -123,12 +122,3 @@ def test_load_balance_diagnostic_hand_cases():
     # capacity 2: kept min(count, 2) = 2 + 2 + 1, the rest dropped
     lb = bench.load_balance([3, 2, 1], T=3, k=2, capacity=2)
     assert lb["kept"] == 5 and lb["drops"] == 1
-
-
-def test_permute_combine_folded_combine():
-    # with a shared expert on the tensor cores the combine has no launch of its own
-    q = synth.PROBLEMS["sqrt_fp4"]
-    assert bench.combine_folded(q) and not bench.combine_folded(synth.PROBLEMS["mixtral_bf16"])
-    stage_ms = {n: 0.0 for n in bench.STAGES}
-    pc = bench.permute_combine(q, 49152, stage_ms, {"hbm": 6000.0, "src": "test"})
-    assert pc["combine"]["folded_into"].startswith("shared expert")
