@@ -25,19 +25,25 @@
 // weights straight into TMEM (tcgen05.st): shared memory carries only the
 // packed codes and the token rows, and the MMAs read only B from it.
 //
-// Roles (448 threads per CTA):
-//   warp 0       TMA producer: the tile's token rows (boxes of 32 rows x 64
-//                columns, or 4-row gathers through a row map), the packed
-//                codes ([half][128 rows][16 B]) and the scales of the k-block
-//                into a 5-stage ring.
+// Roles (480 threads per CTA):
+//   warp 0       token producer: the tile's token rows (boxes of 32 rows x 64
+//                columns, or 4-row gathers through a row map) into a 4-stage
+//                ring (the rows of an expert are read by all its weight
+//                blocks, so they mostly come from L2).
+//   warp 14      weight producer: the packed codes ([half][128 rows][16 B])
+//                and scales of each k-block into a 16-stage ring.  Every
+//                weight block is read once, from HBM, so this ring runs far
+//                ahead (16 k-blocks, ~2 us of MMA work) to cover DRAM latency.
 //   warp 1       TMEM owner; one thread issues the MMAs (A from a 4-stage TMEM
-//                ring, B from the TMA ring) and commits stages back.
+//                ring, B from the token ring) and commits stages back.
 //   warps 2-5    epilogue: TMEM -> registers -> SwiGLU (u handed from the
 //                upper lanes to the lower ones through shared memory) or
 //                routing weight -> global stores; two accumulators of NMAX
 //                columns overlap a tile's epilogue with the next tile's MMAs.
-//   warps 6-13   converters: warp w expands, for the 32 rows of its TMEM lane
-//                quarter (w % 4), one half (32 values) of the k-block's codes.
+//   warps 6-13   converters: warp w expands the k-blocks of one parity
+//                ((w - 6) / 4) for the 32 rows of its TMEM lane quarter
+//                (w % 4), all 64 values of a row per k-block, so two k-blocks
+//                are in flight per quarter.
 //
 // F16 (gate/up inside moe_forward): the token rows arrive as f16 scaled by a
 // power of two per row (launch_gather_f16), the codes are expanded to f16,
@@ -71,11 +77,13 @@ constexpr int NBOX = 32;                        // token rows per TMA box
 constexpr int B_BYTES = NMAX * BK * 2;          // 24 KB of token rows per stage
 constexpr int CODE_BYTES = WM * BK / 2;         // 4 KB: [half][row][16 B]
 constexpr int SCL_BYTES = WM * 16;              // 2 KB: [row][16 B] (scales of 4 k-blocks)
-constexpr int STAGE_BYTES = B_BYTES + CODE_BYTES + SCL_BYTES;
-constexpr int STAGES = 5;
-constexpr int A_STAGES = 4;
+constexpr int STAGES = 4;                       // token ring
+constexpr int C_STAGES = 16;                    // weight (codes + scales) ring
+constexpr int A_STAGES = 4;                     // expanded-weight ring in TMEM
 constexpr int kConv = 8;                        // converter warps
-constexpr int kThreads = 192 + 32 * kConv;
+constexpr int kConvPerBlock = kConv / 2;        // warps that expand one k-block (one per lane quarter)
+constexpr int kWProducerWarp = 6 + kConv;       // the weight producer
+constexpr int kThreads = 32 * (kWProducerWarp + 1);
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t A_COL0 = 2 * NMAX;           // TMEM: acc0 [0,192), acc1 [192,384), A ring [384,512)
 constexpr int XPAD = 33;                        // exchange rows padded against bank conflicts
@@ -86,9 +94,11 @@ static_assert(A_COL0 + A_STAGES * (BK / 2) == TMEM_COLS, "TMEM budget");
 static_assert(NMAX % NBOX == 0 && NMAX % 32 == 0 && NMAX <= 256, "token tile");
 
 struct Smem {
-  uint64_t full[STAGES];       // token rows, codes and scales of the k-block landed
+  uint64_t full[STAGES];       // token rows of the k-block landed
   uint64_t empty[STAGES];      // the MMAs reading the stage completed
-  uint64_t a_full[A_STAGES];   // expanded weights of the k-block in TMEM (kConv arrivals)
+  uint64_t c_full[C_STAGES];   // codes and scales of the k-block landed
+  uint64_t c_empty[C_STAGES];  // the converters read them
+  uint64_t a_full[A_STAGES];   // expanded weights of the k-block in TMEM (one arrival per lane quarter)
   uint64_t a_empty[A_STAGES];  // the MMAs reading them completed
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
@@ -266,9 +276,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t *stage_b = base;                                   // STAGES x 24 KB (1024-aligned)
-  uint8_t *stage_code = stage_b + STAGES * B_BYTES;          // STAGES x 4 KB
-  uint8_t *stage_scl = stage_code + STAGES * CODE_BYTES;     // STAGES x 2 KB
-  float *xbuf = reinterpret_cast<float *>(stage_scl + STAGES * SCL_BYTES);  // 2 pairs x 32 x XPAD
+  uint8_t *stage_code = stage_b + STAGES * B_BYTES;          // C_STAGES x 4 KB
+  uint8_t *stage_scl = stage_code + C_STAGES * CODE_BYTES;   // C_STAGES x 2 KB
+  float *xbuf = reinterpret_cast<float *>(stage_scl + C_STAGES * SCL_BYTES);  // 2 pairs x 32 x XPAD
   uint32_t *lut = reinterpret_cast<uint32_t *>(xbuf + 2 * 32 * XPAD);
   Smem &sm = *reinterpret_cast<Smem *>(lut + 256);
 
@@ -280,8 +290,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&sm.full[s], 1);
       ptx::mbar_init(&sm.empty[s], 1);
     }
+    for (int s = 0; s < C_STAGES; ++s) {
+      ptx::mbar_init(&sm.c_full[s], 1);
+      ptx::mbar_init(&sm.c_empty[s], kConvPerBlock);
+    }
     for (int s = 0; s < A_STAGES; ++s) {
-      ptx::mbar_init(&sm.a_full[s], kConv);
+      ptx::mbar_init(&sm.a_full[s], kConvPerBlock);
       ptx::mbar_init(&sm.a_empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -336,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (any_bad && blockIdx.x == 0) note_violation();
     }
   }
-  if (warp >= 6) {
+  if (warp >= 6 && warp < kWProducerWarp) {
     for (int b = (int)threadIdx.x - 192; b < 256; b += 32 * kConv)
       lut[b] = F16 ? scale_f16x2((uint32_t)b) : scale_bf16x2((uint32_t)b);
   }
@@ -366,9 +380,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
         const Tile tl = decode_tile(p, sm, t);
-        const int w0 = tl.blk * W_ROWS;  // first weight row of each weight tensor
         const int n_box = (tl.n_mma + NBOX - 1) / NBOX;
-        const uint32_t tx = (gather ? tl.n_mma * BK * 2 : n_box * NBOX * BK * 2) + CODE_BYTES + SCL_BYTES;
+        const uint32_t tx = gather ? tl.n_mma * BK * 2 : n_box * NBOX * BK * 2;
         int tok[2][4];
         if (gather) {
 #pragma unroll
@@ -391,21 +404,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t *b = stage_b + s * B_BYTES;
           if (lane == 0) {
-            uint8_t *code = stage_code + s * CODE_BYTES;
-            uint8_t *scl = stage_scl + s * SCL_BYTES;
             ptx::mbar_arrive_expect_tx(&sm.full[s], tx);
             if (!gather)
               for (int i = 0; i < n_box; ++i)
                 ptx::tma_load_2d(b + i * NBOX * BK * 2, &tmX, &sm.full[s], kb * BK, tl.r0 + i * NBOX);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              ptx::tma_load_3d(code + h * (CODE_BYTES / 2), &tmW0, &sm.full[s], kb * (BK / 2) + h * 16, w0, tl.e);
-              if (GATED)
-                ptx::tma_load_3d(code + h * (CODE_BYTES / 2) + W_ROWS * 16, &tmW1, &sm.full[s],
-                                 kb * (BK / 2) + h * 16, w0, tl.e);
-            }
-            ptx::tma_load_3d(scl, &tmS0, &sm.full[s], (kb >> 2) * 16, w0, tl.e);
-            if (GATED) ptx::tma_load_3d(scl + W_ROWS * 16, &tmS1, &sm.full[s], (kb >> 2) * 16, w0, tl.e);
           }
           if (gather) {
             __syncwarp();
@@ -425,6 +427,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < STAGES; ++s)
           if (used[s]) drain_bar(&sm.full[s], last_parity[s], p.status);
       }
+    }
+  } else if (warp == kWProducerWarp) {
+    // ================================================= weight producer
+    if (lane == 0) {
+      uint32_t last_parity[C_STAGES];
+      bool used[C_STAGES];
+#pragma unroll
+      for (int s = 0; s < C_STAGES; ++s) {
+        used[s] = false;
+        last_parity[s] = 0;
+      }
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const Tile tl = decode_tile(p, sm, t);
+        const int w0 = tl.blk * W_ROWS;  // first weight row of each weight tensor
+        for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+          const int s = it % C_STAGES;
+          const uint32_t ph = (it / C_STAGES) & 1u;
+          if (!wait_bar(&sm.c_empty[s], ph ^ 1u, sm, p.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t *code = stage_code + s * CODE_BYTES;
+          uint8_t *scl = stage_scl + s * SCL_BYTES;
+          ptx::mbar_arrive_expect_tx(&sm.c_full[s], CODE_BYTES + SCL_BYTES);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            ptx::tma_load_3d(code + h * (CODE_BYTES / 2), &tmW0, &sm.c_full[s], kb * (BK / 2) + h * 16, w0, tl.e);
+            if (GATED)
+              ptx::tma_load_3d(code + h * (CODE_BYTES / 2) + W_ROWS * 16, &tmW1, &sm.c_full[s],
+                               kb * (BK / 2) + h * 16, w0, tl.e);
+          }
+          ptx::tma_load_3d(scl, &tmS0, &sm.c_full[s], (kb >> 2) * 16, w0, tl.e);
+          if (GATED) ptx::tma_load_3d(scl + W_ROWS * 16, &tmS1, &sm.c_full[s], (kb >> 2) * 16, w0, tl.e);
+          used[s] = true;
+          last_parity[s] = ph;
+        }
+      }
+      for (int s = 0; s < C_STAGES; ++s)
+        if (used[s]) drain_bar(&sm.c_full[s], last_parity[s], p.status);
     }
   } else if (warp == 1) {
     // ================================================= MMA issuer
@@ -539,22 +582,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ================================================= converters (warps 6..13)
-    // Warp w: TMEM lane quarter q = w % 4 (weight rows 32q..32q+31), half h of
-    // each k-block's 64 values.  A thread reads its row's 16 code bytes (the
-    // rows of a half lie 16 bytes apart: conflict-free) and two scales, and
-    // writes 16 expanded words to 16 TMEM columns of its lane.
-    const int q = warp & 3, h = (warp - 6) >> 2;
+    // Warp w: TMEM lane quarter q = w % 4 (weight rows 32q..32q+31) and the
+    // k-blocks of parity (w - 6) / 4 in the common k-block sequence.  A
+    // thread reads its row's 32 code bytes (two 16-byte halves; the rows of a
+    // half lie 16 bytes apart: conflict-free) and four scales, releases the
+    // weight stage, and writes 32 expanded words to 32 TMEM columns.
+    const int q = warp & 3, par = (warp - 6) >> 2;
     const int r = q * 32 + lane;
-    const uint32_t taddr0 = tmem_base + ((uint32_t)(q * 32) << 16) + A_COL0 + h * 16;
+    const uint32_t taddr0 = tmem_base + ((uint32_t)(q * 32) << 16) + A_COL0;
     uint32_t it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
       for (int kb = 0; kb < k_blocks; ++kb, ++it) {
-        const int s = it % STAGES;
+        if ((int)(it & 1u) != par) continue;
+        const int sc = it % C_STAGES;
         const int as = it % A_STAGES;
         bool got = true;
         if (lane == 0) {
-          got = wait_bar(&sm.full[s], (it / STAGES) & 1u, sm, p.status) &&
+          got = wait_bar(&sm.c_full[sc], (it / C_STAGES) & 1u, sm, p.status) &&
                 wait_bar(&sm.a_empty[as], ((it / A_STAGES) & 1u) ^ 1u, sm, p.status);
         }
         if (!__shfl_sync(0xffffffffu, got, 0)) {
@@ -562,17 +607,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         ptx::tc_fence_after();
-        const uint4 q4 = *reinterpret_cast<const uint4 *>(stage_code + s * CODE_BYTES + h * (CODE_BYTES / 2) + r * 16);
-        const uint8_t *sc = stage_scl + s * SCL_BYTES + r * 16 + (kb & 3) * 4 + h * 2;
-        const uint32_t s0 = lut[sc[0]], s1 = lut[sc[1]];
-        uint32_t w[16];
-        const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
+        const uint8_t *code = stage_code + sc * CODE_BYTES + r * 16;
+        const uint4 c0 = *reinterpret_cast<const uint4 *>(code);
+        const uint4 c1 = *reinterpret_cast<const uint4 *>(code + CODE_BYTES / 2);
+        const uint32_t s4 = *reinterpret_cast<const uint32_t *>(stage_scl + sc * SCL_BYTES + r * 16 + (kb & 3) * 4);
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&sm.c_empty[sc]);  // codes and scales are in registers
+        const uint32_t qw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        uint32_t w[32];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (F16) expand_e2m1x8_f16(qw[j], j < 2 ? s0 : s1, w + 4 * j);
-          else expand_e2m1x8_bf16(qw[j], j < 2 ? s0 : s1, p.hi_mul, w + 4 * j);
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t sc2 = lut[(s4 >> (8 * (j >> 1))) & 0xFFu];  // 16 values per scale
+          if (F16) expand_e2m1x8_f16(qw[j], sc2, w + 4 * j);
+          else expand_e2m1x8_bf16(qw[j], sc2, p.hi_mul, w + 4 * j);
         }
-        ptx::tmem_st16(taddr0 + as * (BK / 2), w);
+        ptx::tmem_st32(taddr0 + as * (BK / 2), w);
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         __syncwarp();
@@ -591,8 +640,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-constexpr size_t kSmemBytes =
-    1024 + (size_t)STAGES * STAGE_BYTES + 2 * 32 * XPAD * sizeof(float) + 256 * sizeof(uint32_t) + sizeof(Smem);
+constexpr size_t kSmemBytes = 1024 + (size_t)STAGES * B_BYTES + (size_t)C_STAGES * (CODE_BYTES + SCL_BYTES) +
+                              2 * 32 * XPAD * sizeof(float) + 256 * sizeof(uint32_t) + sizeof(Smem);
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 // tokens: [rows, K] 16-bit (or the gather source); codes [E, Nw, K/2] bytes

@@ -490,3 +490,31 @@ def test_shared_expert_added_once_each_k(B, W, k):
     H.assert_close_layer(p, H.to_np(out), o["out"], "out")
     o0 = O.moe_forward(c.L.x(), logits, idx_g, w_sel, c.L.expert, p.E, 0, p.clamp, "preact", None)
     H.assert_close_layer(p, H.to_np(out0), o0["out"], "out without the shared expert")
+
+
+def test_fp4_uneven_experts(B, W):
+    # the NVFP4 GEMMs size each token tile to its expert: an empty expert, one
+    # expert with most rows (several token tiles) and odd counts elsewhere;
+    # both projections read the packed weights (F % 256 == 0)
+    p = synth.PROBLEMS["sqrt_fp4"].with_(name="fp4_uneven", T=333, D=512, F=512, E=8, k=2, Fs=256)
+    a = synth.generate(p)
+    bias = np.zeros(p.E, dtype=np.float32)
+    bias[0] = -100.0
+    bias[3] = 3.0
+    a["bias"] = bias
+    a["bias_vl"] = bias
+    c = Case(B, W, p, a)
+    g = _stages(B, c)
+    idx_g = H.to_np(g["idx"]).astype(np.int64)
+    d = O.dispatch(idx_g, p.E, 0)
+    assert d["counts"][0] == 0 and d["counts"][3] > 256
+    logits, idx_o, w_o, keys = H.oracle_route(p, c.L, a)
+    H.check_route(p, idx_g, H.to_np(g["w"]), logits, idx_o, keys, bias)
+    w_sel = O.route_weights(logits, idx_g, p.gate)
+    o = O.moe_forward(c.L.x(), logits, idx_g, w_sel, c.L.expert, p.E, 0, p.clamp, "preact", c.L.shared())
+    H.assert_close_layer(p, H.to_np(g["out"]), o["out"], "out")
+    ws = B.workspace(B.workspace_size(c.cfg, p.T))
+    out_f = B.forward(c.cfg, c.x, c.w, ws, c.mask)
+    torch.cuda.synchronize()
+    B.check_device_status(ws)
+    H.assert_close_layer(p, H.to_np(out_f), o["out"], "forward")
