@@ -162,7 +162,9 @@ moe_status moe_selftest_wait_timeout(void *ws, size_t ws_bytes, moe_stream_t str
 
 /* ------------------------------------------------------------ stage 1: route */
 
-/* Bytes of workspace moe_route_topk needs: its device status word. */
+/* Bytes of workspace moe_route_topk needs: its device status word, plus for
+ * E > 32 with bf16 activations (the tensor-core router) the fp32 logit rows
+ * [T, E rounded up to 32] it hands to its selection kernel. */
 size_t moe_route_workspace_size(const MoEConfig *cfg, int T);
 
 /* Router GEMM + gate + top-k for T tokens (a1-a2).
@@ -174,11 +176,11 @@ size_t moe_route_workspace_size(const MoEConfig *cfg, int T);
  *   topk_w     [T, k] float out: the multipliers (renormalised softmax, or raw
  *              sqrt(softplus(s)), or raw sigmoid(s))
  *   ws         >= moe_route_workspace_size(cfg, T) bytes (status word)
- * Logits are accumulated in fp32 (ops-transformer walkthrough, 坑三) and
- * never leave the SM: with E <= 32 (or fp32 activations) one kernel computes
- * them on the CUDA cores and selects from shared memory; with bf16
- * activations and 32 < E <= 512 one kernel computes them on the tensor cores
- * and each thread selects its token's top k straight out of TMEM. */
+ * Logits are accumulated in fp32 (ops-transformer walkthrough, 坑三).  With
+ * E <= 32 (or fp32 activations) one kernel computes them on the CUDA cores
+ * and selects from shared memory.  With bf16 activations and 32 < E <= 512
+ * they are computed on the tensor cores and each token's logit row is stored
+ * to the route workspace, from which a second kernel selects. */
 moe_status moe_route_topk(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
                           const uint8_t *image_mask, int32_t *topk_idx, float *topk_w, void *ws,
                           size_t ws_bytes, moe_stream_t stream);

@@ -180,7 +180,7 @@ MoEConfig shared_cfg(const MoEConfig &c) {
 struct ForwardWs {
   int *status;
   int32_t *topk_idx, *counts, *offsets, *slot_row, *row_token, *chunk_cnt;
-  float *topk_w, *row_weight, *row_scale;
+  float *topk_w, *row_weight, *row_scale, *route_logits;
   void *x_perm, *h, *y_perm, *sh_y;
   ExpertWs ex;
 };
@@ -197,6 +197,7 @@ ForwardWs carve_forward(Carve &cv, const MoEConfig &c, int T) {
   w.row_token = cv.take<int32_t>(Tk);
   w.row_weight = cv.take<float>(Tk);
   w.row_scale = gate_up_direct(c) ? cv.take<float>(Tk) : nullptr;
+  w.route_logits = cv.take<float>(route_scratch_floats(c, T));
   w.chunk_cnt = cv.take<int32_t>((size_t)num_chunks(T) * E);
   w.x_perm = cv.take<char>(Tk * D * as);
   size_t hrows = Tk * c.intermediate_dim;
@@ -271,6 +272,7 @@ size_t moe_route_workspace_size(const MoEConfig *cfg, int T) {
   if (validate_cfg(cfg) != MOE_OK || T < 0) return 0;
   Carve cv(nullptr);
   cv.take<int>(kStatusBytes / sizeof(int));
+  cv.take<float>(route_scratch_floats(*cfg, T));
   return align_up(cv.off, 256);
 }
 
@@ -286,7 +288,8 @@ moe_status moe_route_topk(const MoEConfig *cfg, int T, const void *x, const MoEW
   if (!w || !ok_ptr(x) || !ok_ptr(w->w_router) || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
   Carve cv(ws);
   int *status = cv.take<int>(kStatusBytes / sizeof(int));
-  return launch_route(*cfg, T, x, w->w_router, w->bias, w->bias_vl, image_mask, topk_idx, topk_w, status,
+  float *scratch = cv.take<float>(route_scratch_floats(*cfg, T));
+  return launch_route(*cfg, T, x, w->w_router, w->bias, w->bias_vl, image_mask, topk_idx, topk_w, status, scratch,
                       (cudaStream_t)stream);
 }
 
@@ -450,8 +453,8 @@ static moe_status forward_impl(const MoEConfig *cfg, int T, const void *x, const
   };
 
   if ((st = mark(0)) != MOE_OK) return st;
-  if ((st = launch_route(c, T, x, w->w_router, w->bias, w->bias_vl, image_mask, idx, f.topk_w, f.status, s)) !=
-      MOE_OK)
+  if ((st = launch_route(c, T, x, w->w_router, w->bias, w->bias_vl, image_mask, idx, f.topk_w, f.status,
+                         f.route_logits, s)) != MOE_OK)
     return st;
   if ((st = mark(1)) != MOE_OK) return st;
   // the row maps (histogram, scan, positions), then the row gather

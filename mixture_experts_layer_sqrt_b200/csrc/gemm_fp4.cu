@@ -107,7 +107,8 @@ struct Smem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  int tile_start[MAX_E + 1];
+  int tile_start[MAX_E + 1];  // over the experts in `order`
+  int order[MAX_E];           // experts by token-tile width, widest first
 };
 
 struct Params {
@@ -132,7 +133,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Smem &s
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   while (true) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (ptx::mbar_try_wait_sleep(bar, parity, ptx::kWaitHintNs)) return true;
     if (*(volatile int *)&sm.abort) return false;
     if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
       *(volatile int *)&sm.abort = 1;
@@ -181,7 +182,8 @@ struct Tile {
   int n_mma;    // MMA N: live rounded up to 16
 };
 
-// Largest e with tile_start[e] <= t (empty experts share the next start).
+// Tile t: the largest position j with tile_start[j] <= t (empty experts share
+// the next start), expert order[j].
 __device__ __forceinline__ Tile decode_tile(const Params &p, const Smem &sm, int t) {
   int lo = 0, hi = p.E - 1;
   while (lo < hi) {
@@ -190,16 +192,25 @@ __device__ __forceinline__ Tile decode_tile(const Params &p, const Smem &sm, int
     else hi = mid - 1;
   }
   const int local = t - sm.tile_start[lo];
-  const int b = seg_begin(p, lo), n = seg_end(p, lo) - b;
+  const int e = sm.order[lo];
+  const int b = seg_begin(p, e), n = seg_end(p, e) - b;
   const int step = token_step(n);
   const int nt = local / p.blocks;
   Tile r;
-  r.e = lo;
+  r.e = e;
   r.blk = local - nt * p.blocks;
   r.r0 = b + nt * step;
   r.live = min(step, n - nt * step);
   r.n_mma = (r.live + 15) & ~15;
   return r;
+}
+
+// The i-th tile of this CTA: rounds of gridDim.x tiles, taken left to right in
+// even rounds and right to left in odd ones; -1 past the end.
+__device__ __forceinline__ int tile_of(int i, int total) {
+  const int g = gridDim.x, b = blockIdx.x;
+  const int t = i * g + ((i & 1) ? g - 1 - b : b);
+  return t < total ? t : -1;
 }
 
 // e4m3 scale byte -> bf16x2 of (scale * 2^112), both halves.  The factor
@@ -323,14 +334,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tmem_relinquish();
   }
   if (warp == 2) {
-    // tile_start[e] = sum over e' < e of (token tiles of e') * blocks
-    int carry = 0;
+    // Schedule: experts ordered by token-tile width, widest first (a counting
+    // sort over the widths 16..NMAX, stable in e), then tile_start[j] = sum
+    // over positions j' < j of (token tiles of order[j']) * blocks.  The CTAs
+    // take the tiles in snake order (tile_of), so the long tiles are spread
+    // first and the short ones even out the end.
     bool bad = false;  // checked build: offsets must not decrease or start below 0
-    for (int e0 = 0; e0 < p.E; e0 += 32) {
-      const int e = e0 + lane;
+    int pos = 0;
+    for (int w = NMAX / 16; w >= 0; --w) {  // width bucket: step / 16 (0: empty experts)
+      for (int e0 = 0; e0 < p.E; e0 += 32) {
+        const int e = e0 + lane;
+        bool in = false;
+        if (e < p.E) {
+          if (kChecked && w == 0 && p.offsets && (p.offsets[e] < 0 || p.offsets[e + 1] < p.offsets[e])) bad = true;
+          const int n = seg_end(p, e) - seg_begin(p, e);
+          in = (n > 0 ? token_step(n) / 16 : 0) == w;
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, in);
+        if (in) sm.order[pos + __popc(m & ((1u << lane) - 1u))] = e;
+        pos += __popc(m);
+      }
+    }
+    __syncwarp();
+    int carry = 0;
+    for (int j0 = 0; j0 < p.E; j0 += 32) {
+      const int j = j0 + lane;
       int v = 0;
-      if (e < p.E) {
-        if (kChecked && p.offsets && (p.offsets[e] < 0 || p.offsets[e + 1] < p.offsets[e])) bad = true;
+      if (j < p.E) {
+        const int e = sm.order[j];
         const int n = seg_end(p, e) - seg_begin(p, e);
         v = n > 0 ? (n + token_step(n) - 1) / token_step(n) * p.blocks : 0;
       }
@@ -340,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int o = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += o;
       }
-      if (e < p.E) sm.tile_start[e] = carry + incl - v;
+      if (j < p.E) sm.tile_start[j] = carry + incl - v;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
     const bool any_bad = kChecked && __any_sync(0xffffffffu, bad);
@@ -378,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint32_t it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      for (int ti = 0, t; (t = tile_of(ti, total_tiles)) >= 0 && ok; ++ti) {
         const Tile tl = decode_tile(p, sm, t);
         const int n_box = (tl.n_mma + NBOX - 1) / NBOX;
         const uint32_t tx = gather ? tl.n_mma * BK * 2 : n_box * NBOX * BK * 2;
@@ -440,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint32_t it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      for (int ti = 0, t; (t = tile_of(ti, total_tiles)) >= 0 && ok; ++ti) {
         const Tile tl = decode_tile(p, sm, t);
         const int w0 = tl.blk * W_ROWS;  // first weight row of each weight tensor
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
@@ -475,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       int i = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++i) {
+      for (int t; (t = tile_of(i, total_tiles)) >= 0 && ok; ++i) {
         const Tile tl = decode_tile(p, sm, t);
         const int acc = i & 1;
         if (!wait_bar(&sm.tmem_empty[acc], ((i >> 1) & 1u) ^ 1u, sm, p.status)) break;
@@ -513,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     int i = 0;
     uint32_t xc = 0;  // exchange rounds so far (gate/up)
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++i) {
+    for (int t; (t = tile_of(i, total_tiles)) >= 0; ++i) {
       const Tile tl = decode_tile(p, sm, t);
       const int acc = i & 1;
       if (!warp_wait(&sm.tmem_full[acc], (i >> 1) & 1u, sm, p.status, lane)) break;
@@ -592,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t taddr0 = tmem_base + ((uint32_t)(q * 32) << 16) + A_COL0;
     uint32_t it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+    for (int ti = 0; tile_of(ti, total_tiles) >= 0 && ok; ++ti) {
       for (int kb = 0; kb < k_blocks; ++kb, ++it) {
         if ((int)(it & 1u) != par) continue;
         const int sc = it % C_STAGES;

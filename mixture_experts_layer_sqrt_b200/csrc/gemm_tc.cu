@@ -63,14 +63,6 @@ constexpr int MAX_E = 1024;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s
 constexpr int kThreads = 192;
-// The producer asks L2 for the weight boxes this many k-blocks ahead of their
-// loads (crossing into the CTA's next tile), so that the loads, which a ring
-// of a few stages cannot keep in flight long enough to cover HBM latency, hit
-// L2.  The weights of a tile are read once from HBM either way.
-#ifndef MOE_TC_PREFETCH_KB
-#define MOE_TC_PREFETCH_KB 8
-#endif
-constexpr int kPrefetchKb = MOE_TC_PREFETCH_KB;
 
 template <bool PAIR>
 struct Cfg {
@@ -121,7 +113,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Smem &s
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   while (true) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (ptx::mbar_try_wait_sleep(bar, parity, ptx::kWaitHintNs)) return true;
     if (*(volatile int *)&sm.abort) return false;
     if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
       raise_abort<PAIR>(sm, rank);
@@ -278,26 +270,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       uint32_t it = 0;
       bool ok = true;
-      // the weight boxes the loads below read for (tile, k-block), asked of L2 ahead
-      auto prefetch_b = [&](const Tile &pt, int kb2) {
-        const int k2 = kb2 * BK;
-        if (PAIR) {
-          if (GATED) ptx::tma_prefetch_3d(rank == 0 ? &tmB0 : &tmB1, k2, pt.n_blk * (BN / 2), pt.e);
-          else ptx::tma_prefetch_3d(&tmB0, k2, pt.n_blk * BN + (int)rank * (BN / 2), pt.e);
-        } else if (GATED) {
-          ptx::tma_prefetch_3d(&tmB0, k2, pt.n_blk * (BN / 2), pt.e);
-          ptx::tma_prefetch_3d(&tmB1, k2, pt.n_blk * (BN / 2), pt.e);
-        } else {
-          ptx::tma_prefetch_3d(&tmB0, k2, pt.n_blk * BN, pt.e);
-          ptx::tma_prefetch_3d(&tmB0, k2, pt.n_blk * BN + BN / 2, pt.e);
-        }
-      };
       for (int t = unit; t < total_tiles && ok; t += n_units) {
         const Tile tl = decode_tile(p, sm, t, C::TILE_M);
-        const bool has_next = t + n_units < total_tiles;
-        const Tile tl_next = has_next ? decode_tile(p, sm, t + n_units, C::TILE_M) : tl;
-        if (kPrefetchKb > 0 && lane == 0 && t == unit)  // the first tile's first boxes
-          for (int kb2 = 0; kb2 < kPrefetchKb && kb2 < k_blocks; ++kb2) prefetch_b(tl, kb2);
         int tok[4] = {0, 0, 0, 0};
         if (gather) {
 #pragma unroll
@@ -316,11 +290,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
           }
           if (!got) { ok = false; break; }
-          if (kPrefetchKb > 0 && lane == 0) {
-            const int kb2 = kb + kPrefetchKb;
-            if (kb2 < k_blocks) prefetch_b(tl, kb2);
-            else if (has_next && kb2 - k_blocks < k_blocks) prefetch_b(tl_next, kb2 - k_blocks);
-          }
           const int k0 = kb * BK;
           uint8_t *a = stage_a + s * A_BYTES;
           uint8_t *b = stage_b + s * C::B_BYTES;

@@ -15,16 +15,19 @@ inline int num_chunks(int T) { return (T + kChunkTokens - 1) / kChunkTokens; }
 
 // route.cu ---------------------------------------------------------------
 // Picks the tensor-core router (route_tc.cu) when route_tc_ok(c), else CUDA
-// cores.  status: the workspace's device status word (bounded waits).
+// cores.  status: the workspace's device status word (bounded waits);
+// scratch: route_scratch_floats(c, T) floats (null when that is 0).
 moe_status launch_route(const MoEConfig &c, int T, const void *x, const void *w_router,
                         const float *bias, const float *bias_vl, const uint8_t *image_mask,
-                        int32_t *topk_idx, float *topk_w, int *status, cudaStream_t s);
+                        int32_t *topk_idx, float *topk_w, int *status, float *scratch, cudaStream_t s);
 
 // route_tc.cu ------------------------------------------------------------
 bool route_tc_ok(const MoEConfig &c);
+// fp32 logit rows [T, E_pad] the tensor-core router stores for its selection pass
+size_t route_scratch_floats(const MoEConfig &c, int T);
 moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void *w_router, const float *bias,
                            const float *bias_vl, const uint8_t *image_mask, int32_t *topk_idx, float *topk_w,
-                           int *status, cudaStream_t s);
+                           int *status, float *scratch, cudaStream_t s);
 
 // dispatch.cu ------------------------------------------------------------
 // chunk_cnt: [num_chunks(T), E] int32 scratch.  x_perm may be null: the row

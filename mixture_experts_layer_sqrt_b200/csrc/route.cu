@@ -7,17 +7,22 @@
 // over the selected logits, or the raw sqrt(softplus(s)) gate with the
 // selection bias kept out of the weight ("5A · MoE fine-grained" sec. 1, 3).
 //
-// Work split: each warp owns 4 tokens and sweeps the experts in chunks of 8.
-// A lane accumulates 4 x 8 partial dot products over its slice of D, with the
-// x loads of several 16-byte strides issued ahead; a 31-shuffle transpose
-// reduction leaves lane l with dot product number l.  Logits go to shared
-// memory, never to HBM, and the owning warp selects from there.  (Many
-// experts with bf16 activations use the tensor-core router, route_tc.cu.)
+// Work split: a block of W warps owns 4 W consecutive tokens, whose x rows one
+// thread brings into shared memory with bulk copies (a whole row per copy, all
+// of the block's rows in flight at once, so the kernel streams x at the rate
+// HBM allows).  Each warp then computes 4 tokens x 8 experts per pass over the
+// experts: a lane accumulates 32 partial dot products over its slice of D
+// (x from shared memory, W_r from L1/L2, each W_r vector used for all 4
+// tokens) and a 31-shuffle transpose reduction leaves lane l with dot product
+// number l.  Logits go to shared memory, never to HBM, and the owning warp
+// selects from there.  (Many experts with bf16 activations use the
+// tensor-core router, route_tc.cu.)
 #include <math.h>
 
 #include "common.cuh"
 #include "kernels.h"
 #include "route_select.cuh"
+#include "tc_ptx.cuh"
 
 namespace moe {
 namespace {
@@ -38,120 +43,120 @@ __device__ __forceinline__ float transpose_reduce32(float (&a)[32], int lane) {
   return a[0];
 }
 
-// Each warp owns kTokPerWarp tokens and sweeps the experts in chunks of
-// kExpChunk = 32 / (kTokPerWarp * kParts).  Per pass over D the lanes first
-// issue kAhead strides of 16-byte x loads for all of the warp's tokens (held
-// in registers: several DRAM round trips in flight per lane), then reuse each
-// W_r vector (L1/L2 resident) across those tokens.
-template <typename TIn, int kTokPerWarp, int kParts, int kWarps, int kAhead>
-__global__ void __launch_bounds__(kWarps * 32) route_kernel(int T, int D, int E, int k, int gate,
-                                                           const TIn *__restrict__ x,
-                                                           const TIn *__restrict__ wr,
-                                                           const float *__restrict__ bias,
-                                                           const float *__restrict__ bias_vl,
-                                                           const uint8_t *__restrict__ image_mask,
-                                                           int32_t *__restrict__ topk_idx,
-                                                           float *__restrict__ topk_w) {
-  extern __shared__ float logits[];  // [kTokPerBlock][E]
-  constexpr int kExpChunk = 32 / (kTokPerWarp * kParts);
-  static_assert(kExpChunk * kTokPerWarp * kParts == 32, "32 partial sums per lane");
-  static_assert(kAhead % kParts == 0, "whole groups of parts per pass");
-  constexpr int V = Vec16<TIn>::N;
-  constexpr int kStride = 32 * V;     // elements covered by one warp-wide 16-byte load
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tb = warp * kTokPerWarp;  // first token of this warp within the block
-  const long t_base = (long)blockIdx.x * (kTokPerWarp * kWarps) + tb;
+constexpr int kTokPerWarp = 4;
+constexpr int kExpChunk = 8;  // kTokPerWarp * kExpChunk = 32 partial sums per lane
+constexpr uint64_t kRouteWaitNs = 2000000000ull;
 
-  // ---- phase 1: logits of this warp's tokens
+template <typename TIn>
+__global__ void __launch_bounds__(128) route_kernel(int T, int D, int E, int k, int gate, const TIn *__restrict__ x,
+                                                    const TIn *__restrict__ wr, const float *__restrict__ bias,
+                                                    const float *__restrict__ bias_vl,
+                                                    const uint8_t *__restrict__ image_mask,
+                                                    int32_t *__restrict__ topk_idx, float *__restrict__ topk_w,
+                                                    int *status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int V = Vec16<TIn>::N;
+  const int warps = blockDim.x >> 5;
+  const int tpb = kTokPerWarp * warps;
+  TIn *xs = reinterpret_cast<TIn *>(smem);                               // [tpb][D]
+  float *logits = reinterpret_cast<float *>(smem + (size_t)tpb * D * sizeof(TIn));  // [tpb][E]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(logits + (size_t)tpb * E + 1) ;
+  bar = reinterpret_cast<uint64_t *>(((uintptr_t)bar + 7) & ~(uintptr_t)7);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long t0 = (long)blockIdx.x * tpb;
+  const int nt = (int)min((long)tpb, (long)T - t0);
+  const uint32_t row_bytes = (uint32_t)D * sizeof(TIn);
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar, 1);
+    ptx::fence_mbar_init();
+    ptx::mbar_arrive_expect_tx(bar, row_bytes * nt);
+    for (int i = 0; i < nt; ++i) ptx::bulk_load(xs + (size_t)i * D, x + (t0 + i) * D, row_bytes, bar);
+  }
+  __syncthreads();
+  // every thread waits for the rows (bounded; on expiry record it and leave)
+  if (!ptx::mbar_try_wait(bar, 0)) {
+    const uint64_t ts = ptx::globaltimer_ns();
+    while (!ptx::mbar_try_wait_sleep(bar, 0, ptx::kWaitHintNs)) {
+      if (ptx::globaltimer_ns() - ts > kRouteWaitNs) {
+        if (status) atomicExch(status, kDevTimeout);
+        return;  // the copies target this block's own shared memory; nothing else waits on it
+      }
+    }
+  }
+
+  const int tb = warp * kTokPerWarp;  // this warp's first token within the block
   for (int e0 = 0; e0 < E; e0 += kExpChunk) {
-    float acc[32];  // index ((i * kExpChunk + ee) * kParts + part)
+    float acc[32];  // index i * kExpChunk + ee
 #pragma unroll
     for (int q = 0; q < 32; ++q) acc[q] = 0.0f;
-    for (int d0 = 0; d0 < D; d0 += kAhead * kStride) {
-      Vec16<TIn> xv[kAhead][kTokPerWarp];
+    for (int d = lane * V; d < D; d += 32 * V) {
+      Vec16<TIn> xv[kTokPerWarp];
 #pragma unroll
-      for (int u = 0; u < kAhead; ++u) {
-        const int d = d0 + u * kStride + lane * V;
-#pragma unroll
-        for (int i = 0; i < kTokPerWarp; ++i) {
-          const long t = t_base + i;
-          if (d < D && t < T) xv[u][i] = load16(x + t * D + d);
-          else xv[u][i].v = {};
-        }
+      for (int i = 0; i < kTokPerWarp; ++i) {
+        if (tb + i < nt) xv[i] = load16(xs + (size_t)(tb + i) * D + d);
+        else xv[i].v = {};
       }
 #pragma unroll
-      for (int u = 0; u < kAhead; ++u) {
-        const int part = u % kParts;
-        const int d = d0 + u * kStride + lane * V;
-        if (d < D) {
+      for (int ee = 0; ee < kExpChunk; ++ee) {
+        const int e = e0 + ee;
+        if (e < E) {
+          const Vec16<TIn> wv = load16(wr + (long)e * D + d);
 #pragma unroll
-          for (int ee = 0; ee < kExpChunk; ++ee) {
-            const int e = e0 + ee;
-            if (e < E) {
-              const Vec16<TIn> wv = load16(wr + (long)e * D + d);
+          for (int v = 0; v < V; ++v) {
+            const float wf = wv.get(v);
 #pragma unroll
-              for (int v = 0; v < V; ++v) {
-                const float wf = wv.get(v);
-#pragma unroll
-                for (int i = 0; i < kTokPerWarp; ++i) {
-                  float &a = acc[(i * kExpChunk + ee) * kParts + part];
-                  a = fmaf(xv[u][i].get(v), wf, a);
-                }
-              }
+            for (int i = 0; i < kTokPerWarp; ++i) {
+              float &a = acc[i * kExpChunk + ee];
+              a = fmaf(xv[i].get(v), wf, a);
             }
           }
         }
       }
     }
-    float r = transpose_reduce32(acc, lane);
-#pragma unroll
-    for (int off = 1; off < kParts; off <<= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
-    const int q = lane / kParts;
-    const int i = q / kExpChunk, e = e0 + q % kExpChunk;
-    if (lane % kParts == 0 && e < E) {
-      if (gate == MOE_GATE_SOFTMAX_TOPK_RENORM && bias) r += bias[e];  // router logit bias
-      logits[(tb + i) * E + e] = r;
-    }
+    const float r = transpose_reduce32(acc, lane);
+    const int i = lane / kExpChunk, e = e0 + lane % kExpChunk;
+    if (e < E && tb + i < nt)
+      logits[(tb + i) * E + e] = r + ((gate == MOE_GATE_SOFTMAX_TOPK_RENORM && bias) ? bias[e] : 0.0f);
   }
   __syncwarp();
-
-  for (int i = 0; i < kTokPerWarp; ++i) {
-    const long t = t_base + i;
-    if (t >= T) break;
-    select_topk(logits + (tb + i) * E, t, E, k, gate, bias, bias_vl, image_mask, topk_idx, topk_w, lane);
-  }
+  for (int i = 0; i < kTokPerWarp && tb + i < nt; ++i)
+    select_topk(logits + (tb + i) * E, t0 + tb + i, E, k, gate, bias, bias_vl, image_mask, topk_idx, topk_w, lane);
 }
 
 }  // namespace
 
-template <typename TIn, int TPW, int PARTS, int WARPS, int AHEAD>
+// Warps per block: as many as keep a block's x rows within 160 KB of shared
+// memory (1..4, 4 tokens each).
+template <typename TIn>
 moe_status launch_route_t(const MoEConfig &c, int T, const void *x, const void *w_router, const float *bias,
                           const float *bias_vl, const uint8_t *image_mask, int32_t *topk_idx, float *topk_w,
-                          cudaStream_t s) {
-  constexpr int kTokPerBlock = TPW * WARPS;
-  const int E = c.num_experts;
-  const size_t smem = (size_t)kTokPerBlock * E * sizeof(float);
-  const dim3 grid((T + kTokPerBlock - 1) / kTokPerBlock);
-  auto kern = route_kernel<TIn, TPW, PARTS, WARPS, AHEAD>;
-  if (smem > 48 * 1024)
-    MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  kern<<<grid, WARPS * 32, smem, s>>>(T, c.hidden_dim, E, c.top_k, c.gate, (const TIn *)x, (const TIn *)w_router,
-                                      bias, bias_vl, image_mask, topk_idx, topk_w);
+                          int *status, cudaStream_t s) {
+  const int E = c.num_experts, D = c.hidden_dim;
+  const size_t row = (size_t)D * sizeof(TIn);
+  int warps = (int)((160 * 1024) / (kTokPerWarp * row));
+  if (warps > 4) warps = 4;
+  if (warps < 1) return MOE_ERR_UNSUPPORTED;
+  const int tpb = kTokPerWarp * warps;
+  const size_t smem = (size_t)tpb * row + ((size_t)tpb * E + 1) * sizeof(float) + 16;
+  auto kern = route_kernel<TIn>;
+  MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const dim3 grid((unsigned)((T + tpb - 1) / tpb));
+  kern<<<grid, 32 * warps, smem, s>>>(T, D, E, c.top_k, c.gate, (const TIn *)x, (const TIn *)w_router, bias, bias_vl,
+                                      image_mask, topk_idx, topk_w, status);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
 
 moe_status launch_route(const MoEConfig &c, int T, const void *x, const void *w_router,
                         const float *bias, const float *bias_vl, const uint8_t *image_mask,
-                        int32_t *topk_idx, float *topk_w, int *status, cudaStream_t s) {
+                        int32_t *topk_idx, float *topk_w, int *status, float *scratch, cudaStream_t s) {
   if (T == 0) return MOE_OK;
-  if (route_tc_ok(c)) return launch_route_tc(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, status, s);
-  // CUDA cores: 4 tokens x 8 experts per lane and pass; 2-warp blocks keep
-  // the grid several blocks per SM deep at a few thousand tokens
+  if (route_tc_ok(c))
+    return launch_route_tc(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, status, scratch, s);
   if (c.act_dtype == MOE_F32)
-    return launch_route_t<float, 4, 1, 2, 4>(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, s);
-  return launch_route_t<__nv_bfloat16, 4, 1, 2, 4>(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w,
-                                                   s);
+    return launch_route_t<float>(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, status, s);
+  return launch_route_t<__nv_bfloat16>(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, status, s);
 }
 
 }  // namespace moe

@@ -2,15 +2,13 @@
 //
 // logits r = W_r x ("FFN、SwiGLU 与 MoE" sec. 3; ops-transformer MoE walkthrough,
 // 优化一) with fp32 accumulation (坑三), then the gate and a partial top-k
-// selection (优化二) in the same kernel, without a heap and without writing
-// the logits anywhere: each epilogue thread owns one token (a TMEM lane),
-// streams its logits out of TMEM 32 columns at a time and keeps its k best
-// keys in registers (a compare against the current k-th key, and for the rare
-// key that beats it an unrolled insertion).  Softmax mode: weights are the
-// renormalised softmax of the selected (optionally logit-biased) logits.
-// Sqrt and sigmoid modes: selection on s + bias / bias_vl, weights
-// sqrt(softplus(s)) or sigmoid(s) of the raw score ("5A · MoE fine-grained"
-// sec. 1, 3; the blogdee.com routing-strategies page on Sigmoid Gating).
+// selection (优化二) -- here without a heap and without writing the logits to
+// HBM: the tensor-core kernel leaves them in an L2-resident scratch row per
+// token and a second kernel selects each token's top-k with one warp (k rounds
+// of a warp argmax) on every SM.  Softmax mode: weights
+// are the renormalised softmax of the selected (optionally logit-biased)
+// logits.  Sqrt mode: selection on s + bias / bias_vl, weights
+// sqrt(softplus(s)) of the raw score ("5A · MoE fine-grained" sec. 1, 3).
 //
 // One CTA per 128 tokens, 192 threads: warp 0 loads x (128 x 64) and W_r
 // (E_pad x 64, in 128-row boxes) per k-block with TMA; warp 1 issues
@@ -18,7 +16,12 @@
 // E_pad > 256) into fp32 TMEM accumulators of E_pad columns -- up to four,
 // fed by interleaved k-blocks and summed in a fixed order afterwards, which
 // keeps each fp32 sum short.  Warps 2-5 then sum the accumulators of their
-// tokens (TMEM lanes) and select.  All waits bounded.
+// tokens (TMEM lanes) and store the logit rows.  Selecting in this kernel
+// leaves one thread per token, 4 warps per 128 tokens, on at most T / 128 SMs;
+// the separate selection kernel (a warp per token) spreads it over the GPU.
+// Measured at T = 8192: selecting in the epilogue with a register top-k took
+// 120 us at E = 384 and 103 us at E = 128, against 90 us and 57 us here.
+// All waits bounded.
 #include "common.cuh"
 #include "kernels.h"
 #include "route_select.cuh"
@@ -38,19 +41,13 @@ constexpr uint64_t kRDrainNs = 200000000ull;
 
 struct RParams {
   int T, D, E, E_pad, k, gate, stages, b_rows;
+  float *logits;  // [T, ld] fp32 out (router logit bias included in softmax mode)
+  int ld;         // logit row stride: E_pad rounded up to whole 32-column chunks
   int n_acc;  // independent accumulators over interleaved k-blocks (shorter fp32 sums)
   uint32_t tmem_cols;
-  const float *bias, *bias_vl;
-  const uint8_t *image_mask;
-  int32_t *topk_idx;
-  float *topk_w;
+  const float *bias;
   int *status;
 };
-
-constexpr int kMaxK = 16;
-
-// a beats b: larger key, or an equal key at a lower expert index
-__device__ __forceinline__ bool beats(float a, int ai, float b, int bi) { return a > b || (a == b && ai < bi); }
 
 struct RSmem {
   uint64_t full[kMaxStages];
@@ -59,16 +56,14 @@ struct RSmem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  float bias[kMaxEPad];      // softmax mode: router logit bias (0 otherwise)
-  float sel_bias[kMaxEPad];  // sqrt / sigmoid modes: selection bias (0 otherwise)
-  float sel_bias_vl[kMaxEPad];
+  float bias[kMaxEPad];
 };
 
 __device__ __forceinline__ bool rwait(uint64_t *bar, uint32_t parity, RSmem &sm, int *status) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   while (true) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (ptx::mbar_try_wait_sleep(bar, parity, ptx::kWaitHintNs)) return true;
     if (*(volatile int *)&sm.abort) return false;
     if (ptx::globaltimer_ns() - t0 > kRWaitNs) {
       *(volatile int *)&sm.abort = 1;
@@ -118,13 +113,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
     ptx::tmem_alloc(&sm.tmem_base, p.tmem_cols);
     ptx::tmem_relinquish();
   }
-  if (warp >= 2) {  // biases: the logit bias (softmax mode) or the selection biases (sqrt, sigmoid)
-    const bool soft = p.gate == MOE_GATE_SOFTMAX_TOPK_RENORM;
-    for (int e = threadIdx.x - 64; e < p.E; e += kRThreads - 64) {
-      sm.bias[e] = (p.bias && soft) ? p.bias[e] : 0.0f;
-      sm.sel_bias[e] = (p.bias && !soft) ? p.bias[e] : 0.0f;
-      sm.sel_bias_vl[e] = (p.bias_vl && !soft) ? p.bias_vl[e] : sm.sel_bias[e];
-    }
+  if (warp >= 2) {  // router logit bias (softmax mode), added before the logits are stored
+    for (int e = threadIdx.x - 64; e < p.E; e += kRThreads - 64)
+      sm.bias[e] = (p.bias && p.gate == MOE_GATE_SOFTMAX_TOPK_RENORM) ? p.bias[e] : 0.0f;
   }
   ptx::tc_fence_before();
   __syncwarp();
@@ -183,31 +174,15 @@ __global__ void __launch_bounds__(kRThreads, 1)
       rdrain(&sm.drain, 0, p.status);
     }
   } else {
-    // ---- selection: one token (TMEM lane) per thread
+    // ---- logit rows: one token (TMEM lane) per thread
     const int q = warp & 3;
-    const long t = (long)m0 + q * 32 + lane;
+    const int row = m0 + q * 32 + lane;
     bool ok = true;
     if (lane == 0) ok = rwait(&sm.acc_full, 0, sm, p.status);
     if (__shfl_sync(0xffffffffu, ok, 0)) {
       ptx::tc_fence_after();
-      const bool live = t < p.T;
-      const float *sel = (live && p.image_mask && p.image_mask[t]) ? sm.sel_bias_vl : sm.sel_bias;
-      const int k = p.k;
-      float tk[kMaxK], tl[kMaxK];  // best keys (descending) and their logits
-      int ti[kMaxK];
-#pragma unroll
-      for (int j = 0; j < kMaxK; ++j) {
-        tk[j] = -INFINITY;
-        tl[j] = 0.0f;
-        ti[j] = p.E;  // no expert yet: any key beats it
-      }
-      float thr = -INFINITY;  // the k-th best key so far and its expert
-      int thr_i = p.E;
-      // candidate buffer: this thread's row in the stage memory, which the
-      // finished GEMM no longer reads (every copy was consumed before acc_full)
-      ptx::fence_proxy_async_smem();
-      float *ckey = reinterpret_cast<float *>(base) + (q * 32 + lane) * 65;
-      float *clog = ckey + 32;
+      const bool live = row < p.T;
+      float *dst = p.logits + (long)row * p.ld;  // chunk c writes columns [c, c + 32) < ld
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16);
       for (int c = 0; c < p.E_pad; c += 32) {
         uint32_t v[32];
@@ -222,74 +197,17 @@ __global__ void __launch_bounds__(kRThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) lsum[j] += __uint_as_float(v[j]);
         }
-        // keys of this chunk that beat the current k-th go to the thread's
-        // row of the candidate buffer; the rare insertions then run from there
-        uint32_t cand = 0;
+        if (live) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int e = c + j;
-          const float l = lsum[j] + sm.bias[e < p.E ? e : 0];  // softmax mode: the biased logit
-          float key = l + sel[e < p.E ? e : 0];
-          if (key != key) key = -INFINITY;
-          if (e < p.E && beats(key, e, thr, thr_i)) {
-            cand |= 1u << j;
-            ckey[j] = key;
-            clog[j] = l;
+          for (int j = 0; j < 32; j += 4) {
+            float4 o;
+            o.x = c + j < p.E ? lsum[j] + sm.bias[c + j] : -INFINITY;
+            o.y = c + j + 1 < p.E ? lsum[j + 1] + sm.bias[c + j + 1] : -INFINITY;
+            o.z = c + j + 2 < p.E ? lsum[j + 2] + sm.bias[c + j + 2] : -INFINITY;
+            o.w = c + j + 3 < p.E ? lsum[j + 3] + sm.bias[c + j + 3] : -INFINITY;
+            *reinterpret_cast<float4 *>(dst + c + j) = o;
           }
         }
-        while (cand) {
-          const int j = __ffs(cand) - 1;
-          cand &= cand - 1;
-          float kk = ckey[j], ll = clog[j];
-          int ii = c + j;
-#pragma unroll
-          for (int r = 0; r < kMaxK; ++r) {
-            if (r < k && beats(kk, ii, tk[r], ti[r])) {
-              const float k2 = tk[r], l2 = tl[r];
-              const int i2 = ti[r];
-              tk[r] = kk;
-              tl[r] = ll;
-              ti[r] = ii;
-              kk = k2;
-              ll = l2;
-              ii = i2;
-            }
-          }
-          // the new k-th key: the last of the first k slots (predicated moves)
-          thr = tk[0];
-          thr_i = ti[0];
-#pragma unroll
-          for (int r = 1; r < kMaxK; ++r) {
-            const bool in = r < k;
-            thr = in ? tk[r] : thr;
-            thr_i = in ? ti[r] : thr_i;
-          }
-        }
-      }
-      if (live) {
-        float w[kMaxK];
-        if (p.gate == MOE_GATE_SOFTMAX_TOPK_RENORM) {
-          float sum = 0.0f;
-#pragma unroll
-          for (int r = 0; r < kMaxK; ++r) {
-            w[r] = r < k ? expf(tl[r] - tl[0]) : 0.0f;  // tl[0]: the largest selected logit
-            sum += w[r];
-          }
-#pragma unroll
-          for (int r = 0; r < kMaxK; ++r) w[r] /= sum;
-        } else if (p.gate == MOE_GATE_SIGMOID_RAW) {
-#pragma unroll
-          for (int r = 0; r < kMaxK; ++r) w[r] = 1.0f / (1.0f + expf(-tl[r]));
-        } else {
-#pragma unroll
-          for (int r = 0; r < kMaxK; ++r) w[r] = sqrtf(softplus_f32(tl[r]));
-        }
-#pragma unroll
-        for (int r = 0; r < kMaxK; ++r)
-          if (r < k) {
-            p.topk_idx[t * k + r] = ti[r];
-            p.topk_w[t * k + r] = w[r];
-          }
       }
     }
   }
@@ -304,7 +222,36 @@ __global__ void __launch_bounds__(kRThreads, 1)
   }
 }
 
+// One warp per token: copy its logit row to shared memory, then select.
+constexpr int kSelWarps = 8;
+__global__ void __launch_bounds__(32 * kSelWarps) route_select_kernel(int T, int E, int ld, int k, int gate,
+                                                                     const float *__restrict__ logits,
+                                                                     const float *__restrict__ bias,
+                                                                     const float *__restrict__ bias_vl,
+                                                                     const uint8_t *__restrict__ image_mask,
+                                                                     int32_t *__restrict__ topk_idx,
+                                                                     float *__restrict__ topk_w) {
+  extern __shared__ float rows[];  // [kSelWarps][ld]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float *lg = rows + warp * ld;
+  for (long t = (long)blockIdx.x * kSelWarps + warp; t < T; t += (long)gridDim.x * kSelWarps) {
+    const float *src = logits + t * ld;
+    for (int e = lane; e < E; e += 32) lg[e] = src[e];
+    __syncwarp();
+    select_topk(lg, t, E, k, gate, bias, bias_vl, image_mask, topk_idx, topk_w, lane);
+    __syncwarp();
+  }
+}
+
 }  // namespace
+
+// Logit row stride of the tensor-core router: E padded to 16 (the MMA's N
+// granularity), then to whole 32-column TMEM load chunks.
+static int route_ld(int E) { return ((E + 15) / 16 * 16 + 31) / 32 * 32; }
+
+size_t route_scratch_floats(const MoEConfig &c, int T) {
+  return route_tc_ok(c) ? (size_t)T * route_ld(c.num_experts) : 0;
+}
 
 // Few experts: one CTA per 128 tokens leaves most SMs idle while it streams x,
 // and the CUDA-core router (all SMs) is faster (measured 52 vs 84 us at E=8).
@@ -315,7 +262,7 @@ bool route_tc_ok(const MoEConfig &c) {
 
 moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void *w_router, const float *bias,
                            const float *bias_vl, const uint8_t *image_mask, int32_t *topk_idx, float *topk_w,
-                           int *status, cudaStream_t s) {
+                           int *status, float *scratch, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   RParams p;
   p.T = T;
@@ -333,10 +280,8 @@ moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void 
   while (cols < need) cols <<= 1;
   p.tmem_cols = cols;
   p.bias = bias;
-  p.bias_vl = bias_vl;
-  p.image_mask = image_mask;
-  p.topk_idx = topk_idx;
-  p.topk_w = topk_w;
+  p.logits = scratch;
+  p.ld = route_ld(c.num_experts);
   p.status = status;
   const int stage_bytes = RBM * RBK * 2 + p.b_rows * RBK * 2;
   int stages = (192 * 1024) / stage_bytes;
@@ -348,6 +293,16 @@ moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void 
   const dim3 grid((T + RBM - 1) / RBM);
   MOE_CUDA_TRY(cudaFuncSetAttribute(tc_route_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   tc_route_topk<<<grid, kRThreads, smem, s>>>(tx, tw, p);
+  MOE_LAUNCH_CHECK();
+  int dev = 0, sms = 148;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  long sel_blocks = ((long)T + kSelWarps - 1) / kSelWarps;
+  if (sel_blocks > (long)sms * 8) sel_blocks = (long)sms * 8;
+  const bool sel = c.gate != MOE_GATE_SOFTMAX_TOPK_RENORM;  // softmax: the logit bias is already in the logits
+  route_select_kernel<<<(unsigned)sel_blocks, 32 * kSelWarps, (size_t)kSelWarps * p.ld * sizeof(float), s>>>(
+      T, p.E, p.ld, p.k, p.gate, scratch, sel ? bias : nullptr, sel ? bias_vl : nullptr, image_mask, topk_idx,
+      topk_w);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
