@@ -35,7 +35,9 @@
 //                weight block is read once, from HBM, so this ring runs far
 //                ahead (16 k-blocks, ~2 us of MMA work) to cover DRAM latency.
 //   warp 1       TMEM owner; one thread issues the MMAs (A from a 4-stage TMEM
-//                ring, B from the token ring) and commits stages back.
+//                ring, B from the token ring) and commits stages back.  It
+//                waits on one barrier per k-block: the converters arrive only
+//                after the k-block's token rows have landed as well.
 //   warps 2-5    epilogue: TMEM -> registers -> SwiGLU (u handed from the
 //                upper lanes to the lower ones through shared memory) or
 //                routing weight -> global stores; two accumulators of NMAX
@@ -516,8 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
           const int s = it % STAGES;
           const int as = it % A_STAGES;
-          if (!wait_bar(&sm.full[s], (it / STAGES) & 1u, sm, p.status) ||
-              !wait_bar(&sm.a_full[as], (it / A_STAGES) & 1u, sm, p.status)) {
+          // a_full implies the token stage too: its converters waited for it
+          if (!wait_bar(&sm.a_full[as], (it / A_STAGES) & 1u, sm, p.status)) {
             ok = false;
             break;
           }
@@ -630,8 +632,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int as = it % A_STAGES;
         bool got = true;
         if (lane == 0) {
+          // the codes, a free TMEM stage, and the token rows the MMAs of this
+          // k-block will read (so the MMA thread waits on a_full alone)
           got = wait_bar(&sm.c_full[sc], (it / C_STAGES) & 1u, sm, p.status) &&
-                wait_bar(&sm.a_empty[as], ((it / A_STAGES) & 1u) ^ 1u, sm, p.status);
+                wait_bar(&sm.a_empty[as], ((it / A_STAGES) & 1u) ^ 1u, sm, p.status) &&
+                wait_bar(&sm.full[it % STAGES], (it / STAGES) & 1u, sm, p.status);
         }
         if (!__shfl_sync(0xffffffffu, got, 0)) {
           ok = false;

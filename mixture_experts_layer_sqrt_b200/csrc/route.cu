@@ -7,15 +7,18 @@
 // over the selected logits, or the raw sqrt(softplus(s)) gate with the
 // selection bias kept out of the weight ("5A · MoE fine-grained" sec. 1, 3).
 //
-// Work split: a block of W warps owns 4 W consecutive tokens, whose x rows one
+// Work split: a block owns up to 16 consecutive tokens, whose x rows one
 // thread brings into shared memory with bulk copies (a whole row per copy, all
-// of the block's rows in flight at once, so the kernel streams x at the rate
-// HBM allows).  Each warp then computes 4 tokens x 8 experts per pass over the
-// experts: a lane accumulates 32 partial dot products over its slice of D
-// (x from shared memory, W_r from L1/L2, each W_r vector used for all 4
-// tokens) and a 31-shuffle transpose reduction leaves lane l with dot product
-// number l.  Logits go to shared memory, never to HBM, and the owning warp
-// selects from there.  (Many experts with bf16 activations use the
+// of the block's rows in flight at once).  16 warps then split the work four
+// ways by token group and four ways by the reduction: warp w computes 4
+// tokens x 8 experts over one interleaved quarter of D (a lane accumulates 32
+// partial dot products, x from shared memory, each W_r vector from L1/L2 used
+// for all 4 tokens), a 31-shuffle transpose reduction leaves lane l with
+// partial sum number l, and the four quarters are added in a fixed order
+// through shared memory.  Sixteen warps per SM keep enough independent
+// instruction streams to hide the load and FMA latencies that left a
+// four-warp version at 0.36 TB/s.  Logits go to shared memory, never to HBM,
+// and the token group's first warp selects from there.  (Many experts with bf16 activations use the
 // tensor-core router, route_tc.cu.)
 #include <math.h>
 
@@ -44,11 +47,14 @@ __device__ __forceinline__ float transpose_reduce32(float (&a)[32], int lane) {
 }
 
 constexpr int kTokPerWarp = 4;
-constexpr int kExpChunk = 8;  // kTokPerWarp * kExpChunk = 32 partial sums per lane
+constexpr int kExpChunk = 8;   // kTokPerWarp * kExpChunk = 32 partial sums per lane
+constexpr int kDParts = 4;     // warps sharing a token group, each a quarter of D
 constexpr uint64_t kRouteWaitNs = 2000000000ull;
 
+// blockDim.x = 32 * groups * kDParts: warp w covers token group w % groups and
+// D part w / groups.
 template <typename TIn>
-__global__ void __launch_bounds__(128) route_kernel(int T, int D, int E, int k, int gate, const TIn *__restrict__ x,
+__global__ void __launch_bounds__(512) route_kernel(int T, int D, int E, int k, int gate, const TIn *__restrict__ x,
                                                     const TIn *__restrict__ wr, const float *__restrict__ bias,
                                                     const float *__restrict__ bias_vl,
                                                     const uint8_t *__restrict__ image_mask,
@@ -56,13 +62,14 @@ __global__ void __launch_bounds__(128) route_kernel(int T, int D, int E, int k, 
                                                     int *status) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int V = Vec16<TIn>::N;
-  const int warps = blockDim.x >> 5;
-  const int tpb = kTokPerWarp * warps;
-  TIn *xs = reinterpret_cast<TIn *>(smem);                               // [tpb][D]
-  float *logits = reinterpret_cast<float *>(smem + (size_t)tpb * D * sizeof(TIn));  // [tpb][E]
-  uint64_t *bar = reinterpret_cast<uint64_t *>(logits + (size_t)tpb * E + 1) ;
-  bar = reinterpret_cast<uint64_t *>(((uintptr_t)bar + 7) & ~(uintptr_t)7);
+  const int groups = (blockDim.x >> 5) / kDParts;
+  const int tpb = kTokPerWarp * groups;
+  TIn *xs = reinterpret_cast<TIn *>(smem);                                          // [tpb][D]
+  float *part = reinterpret_cast<float *>(smem + (size_t)tpb * D * sizeof(TIn));    // [kDParts][tpb][kExpChunk]
+  float *logits = part + kDParts * tpb * kExpChunk;                                  // [tpb][E]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(((uintptr_t)(logits + (size_t)tpb * E) + 15) & ~(uintptr_t)15);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = warp % groups, dp = warp / groups;
   const long t0 = (long)blockIdx.x * tpb;
   const int nt = (int)min((long)tpb, (long)T - t0);
   const uint32_t row_bytes = (uint32_t)D * sizeof(TIn);
@@ -74,23 +81,25 @@ __global__ void __launch_bounds__(128) route_kernel(int T, int D, int E, int k, 
     for (int i = 0; i < nt; ++i) ptx::bulk_load(xs + (size_t)i * D, x + (t0 + i) * D, row_bytes, bar);
   }
   __syncthreads();
-  // every thread waits for the rows (bounded; on expiry record it and leave)
-  if (!ptx::mbar_try_wait(bar, 0)) {
+  // every thread waits for the rows (bounded); a timeout is recorded and the
+  // whole block leaves before any further barrier
+  bool ok = ptx::mbar_try_wait(bar, 0);
+  if (!ok) {
     const uint64_t ts = ptx::globaltimer_ns();
-    while (!ptx::mbar_try_wait_sleep(bar, 0, ptx::kWaitHintNs)) {
-      if (ptx::globaltimer_ns() - ts > kRouteWaitNs) {
-        if (status) atomicExch(status, kDevTimeout);
-        return;  // the copies target this block's own shared memory; nothing else waits on it
-      }
-    }
+    while (!(ok = ptx::mbar_try_wait_sleep(bar, 0, ptx::kWaitHintNs)))
+      if (ptx::globaltimer_ns() - ts > kRouteWaitNs) break;
+  }
+  if (!__syncthreads_and(ok)) {
+    if (threadIdx.x == 0 && status) atomicExch(status, kDevTimeout);
+    return;
   }
 
-  const int tb = warp * kTokPerWarp;  // this warp's first token within the block
+  const int tb = grp * kTokPerWarp;  // this warp's first token within the block
   for (int e0 = 0; e0 < E; e0 += kExpChunk) {
     float acc[32];  // index i * kExpChunk + ee
 #pragma unroll
     for (int q = 0; q < 32; ++q) acc[q] = 0.0f;
-    for (int d = lane * V; d < D; d += 32 * V) {
+    for (int d = (dp * 32 + lane) * V; d < D; d += kDParts * 32 * V) {
       Vec16<TIn> xv[kTokPerWarp];
 #pragma unroll
       for (int i = 0; i < kTokPerWarp; ++i) {
@@ -114,35 +123,44 @@ __global__ void __launch_bounds__(128) route_kernel(int T, int D, int E, int k, 
         }
       }
     }
-    const float r = transpose_reduce32(acc, lane);
-    const int i = lane / kExpChunk, e = e0 + lane % kExpChunk;
-    if (e < E && tb + i < nt)
-      logits[(tb + i) * E + e] = r + ((gate == MOE_GATE_SOFTMAX_TOPK_RENORM && bias) ? bias[e] : 0.0f);
+    const float r = transpose_reduce32(acc, lane);  // lane l: token l / 8, expert e0 + l % 8
+    part[(dp * tpb + tb) * kExpChunk + lane] = r;
+    __syncthreads();
+    if (dp == 0) {
+      const int i = lane / kExpChunk, e = e0 + lane % kExpChunk;
+      float sum = 0.0f;
+#pragma unroll
+      for (int q = 0; q < kDParts; ++q) sum += part[(q * tpb + tb) * kExpChunk + lane];  // fixed order
+      if (e < E && tb + i < nt)
+        logits[(tb + i) * E + e] = sum + ((gate == MOE_GATE_SOFTMAX_TOPK_RENORM && bias) ? bias[e] : 0.0f);
+    }
+    __syncthreads();
   }
-  __syncwarp();
-  for (int i = 0; i < kTokPerWarp && tb + i < nt; ++i)
-    select_topk(logits + (tb + i) * E, t0 + tb + i, E, k, gate, bias, bias_vl, image_mask, topk_idx, topk_w, lane);
+  if (dp == 0)
+    for (int i = 0; i < kTokPerWarp && tb + i < nt; ++i)
+      select_topk(logits + (tb + i) * E, t0 + tb + i, E, k, gate, bias, bias_vl, image_mask, topk_idx, topk_w,
+                  lane);
 }
 
 }  // namespace
 
-// Warps per block: as many as keep a block's x rows within 160 KB of shared
-// memory (1..4, 4 tokens each).
+// Token groups per block (4 tokens each): as many as keep a block's x rows
+// within 160 KB of shared memory, at most 4 (16 warps).
 template <typename TIn>
 moe_status launch_route_t(const MoEConfig &c, int T, const void *x, const void *w_router, const float *bias,
                           const float *bias_vl, const uint8_t *image_mask, int32_t *topk_idx, float *topk_w,
                           int *status, cudaStream_t s) {
   const int E = c.num_experts, D = c.hidden_dim;
   const size_t row = (size_t)D * sizeof(TIn);
-  int warps = (int)((160 * 1024) / (kTokPerWarp * row));
-  if (warps > 4) warps = 4;
-  if (warps < 1) return MOE_ERR_UNSUPPORTED;
-  const int tpb = kTokPerWarp * warps;
-  const size_t smem = (size_t)tpb * row + ((size_t)tpb * E + 1) * sizeof(float) + 16;
+  int groups = (int)((160 * 1024) / (kTokPerWarp * row));
+  if (groups > 4) groups = 4;
+  if (groups < 1) return MOE_ERR_UNSUPPORTED;
+  const int tpb = kTokPerWarp * groups;
+  const size_t smem = (size_t)tpb * row + ((size_t)kDParts * tpb * kExpChunk + (size_t)tpb * E) * sizeof(float) + 32;
   auto kern = route_kernel<TIn>;
   MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   const dim3 grid((unsigned)((T + tpb - 1) / tpb));
-  kern<<<grid, 32 * warps, smem, s>>>(T, D, E, c.top_k, c.gate, (const TIn *)x, (const TIn *)w_router, bias, bias_vl,
+  kern<<<grid, 32 * groups * kDParts, smem, s>>>(T, D, E, c.top_k, c.gate, (const TIn *)x, (const TIn *)w_router, bias, bias_vl,
                                       image_mask, topk_idx, topk_w, status);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
