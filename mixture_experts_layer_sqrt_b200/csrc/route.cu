@@ -142,6 +142,120 @@ __global__ void __launch_bounds__(512) route_kernel(int T, int D, int E, int k, 
                   lane);
 }
 
+// bf16 activations, E <= 32: the logits on the tensor cores with the
+// warp-level mma.sync (m16n8k16, bf16 in, fp32 accumulate), so the kernel is
+// left with streaming x.  A block owns 8 tokens: one thread bulk-copies their
+// x rows into shared memory (rows padded by 16 bytes so the fragment loads of
+// the 8 rows fall in different banks), and 4 warps each take every fourth
+// 16-wide step of D into two accumulator sets (alternate steps).  The 8
+// partial sums per logit (4 warps x 2 sets) are added in a fixed order,
+// which keeps each fp32 sum short, as the tensor-core router's split-K
+// accumulators do.  Rows 8..15 of every MMA are zero.
+constexpr int kMmaTok = 8;
+constexpr int kMmaWarps = 4;
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(32 * kMmaWarps) route_mma_kernel(int T, int D, int E, int k, int gate,
+                                                                   const __nv_bfloat16 *__restrict__ x,
+                                                                   const __nv_bfloat16 *__restrict__ wr,
+                                                                   const float *__restrict__ bias,
+                                                                   const float *__restrict__ bias_vl,
+                                                                   const uint8_t *__restrict__ image_mask,
+                                                                   int32_t *__restrict__ topk_idx,
+                                                                   float *__restrict__ topk_w, int *status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int ld = D + 8;  // padded row length in bf16 (16 bytes of padding)
+  __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(smem);                      // [kMmaTok][ld]
+  float *part = reinterpret_cast<float *>(smem + (size_t)kMmaTok * ld * 2);         // [8 sums][kMmaTok][32]
+  float *logits = part + 8 * kMmaTok * 32;                                           // [kMmaTok][E]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(((uintptr_t)(logits + kMmaTok * E) + 15) & ~(uintptr_t)15);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const long t0 = (long)blockIdx.x * kMmaTok;
+  const int nt = (int)min((long)kMmaTok, (long)T - t0);
+  const uint32_t row_bytes = (uint32_t)D * 2;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar, 1);
+    ptx::fence_mbar_init();
+    ptx::mbar_arrive_expect_tx(bar, row_bytes * nt);
+    for (int i = 0; i < nt; ++i) ptx::bulk_load(xs + (size_t)i * ld, x + (t0 + i) * D, row_bytes, bar);
+  }
+  // rows past the last token read as zeros
+  for (int i = nt + warp; i < kMmaTok; i += kMmaWarps)
+    for (int j = lane * 8; j < D; j += 32 * 8) *reinterpret_cast<uint4 *>(xs + (size_t)i * ld + j) = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+  bool ok = ptx::mbar_try_wait(bar, 0);
+  if (!ok) {
+    const uint64_t ts = ptx::globaltimer_ns();
+    while (!(ok = ptx::mbar_try_wait_sleep(bar, 0, ptx::kWaitHintNs)))
+      if (ptx::globaltimer_ns() - ts > kRouteWaitNs) break;
+  }
+  if (!__syncthreads_and(ok)) {
+    if (threadIdx.x == 0 && status) atomicExch(status, kDevTimeout);
+    return;
+  }
+
+  const int n_tiles = (E + 7) >> 3;  // <= 4
+  float acc[2][4][4];
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[h][n][q] = 0.0f;
+  const __nv_bfloat16 *xr = xs + (size_t)g * ld + 2 * c;
+  int step = 0;
+  for (int k0 = warp * 16; k0 < D; k0 += kMmaWarps * 16, ++step) {
+    uint32_t a[4];
+    a[0] = *reinterpret_cast<const uint32_t *>(xr + k0);
+    a[1] = 0u;  // rows 8..15
+    a[2] = *reinterpret_cast<const uint32_t *>(xr + k0 + 8);
+    a[3] = 0u;
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+      if (n < n_tiles) {
+        const int e = n * 8 + g;
+        uint32_t b0 = 0u, b1 = 0u;
+        if (e < E) {
+          const __nv_bfloat16 *wrow = wr + (long)e * D + k0 + 2 * c;
+          b0 = __ldg(reinterpret_cast<const unsigned int *>(wrow));
+          b1 = __ldg(reinterpret_cast<const unsigned int *>(wrow + 8));
+        }
+        if (step & 1) mma_bf16_16816(acc[1][n], a, b0, b1);
+        else mma_bf16_16816(acc[0][n], a, b0, b1);
+      }
+    }
+  }
+  // C fragment: d0, d1 = token g, experts n*8 + 2c, 2c + 1 (d2, d3: rows 8..15, unused)
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+      float *dst = part + ((warp * 2 + h) * kMmaTok + g) * 32 + n * 8 + 2 * c;
+      dst[0] = acc[h][n][0];
+      dst[1] = acc[h][n][1];
+    }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < kMmaTok * E; idx += blockDim.x) {
+    const int i = idx / E, e = idx - i * E;
+    float sum = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) sum += part[(q * kMmaTok + i) * 32 + e];  // fixed order
+    logits[i * E + e] = sum + ((gate == MOE_GATE_SOFTMAX_TOPK_RENORM && bias) ? bias[e] : 0.0f);
+  }
+  __syncthreads();
+  for (int i = warp; i < nt; i += kMmaWarps)
+    select_topk(logits + i * E, t0 + i, E, k, gate, bias, bias_vl, image_mask, topk_idx, topk_w, lane);
+}
+
 }  // namespace
 
 // Token groups per block (4 tokens each): as many as keep a block's x rows
@@ -174,6 +288,16 @@ moe_status launch_route(const MoEConfig &c, int T, const void *x, const void *w_
     return launch_route_tc(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, status, scratch, s);
   if (c.act_dtype == MOE_F32)
     return launch_route_t<float>(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, status, s);
+  if (c.num_experts <= 32 && c.hidden_dim % 16 == 0 && (size_t)kMmaTok * (c.hidden_dim + 8) * 2 <= 160 * 1024) {
+    const int E = c.num_experts;
+    const size_t smem = (size_t)kMmaTok * (c.hidden_dim + 8) * 2 + (8 * kMmaTok * 32 + (size_t)kMmaTok * E) * 4 + 32;
+    MOE_CUDA_TRY(cudaFuncSetAttribute(route_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    route_mma_kernel<<<(unsigned)((T + kMmaTok - 1) / kMmaTok), 32 * kMmaWarps, smem, s>>>(
+        T, c.hidden_dim, E, c.top_k, c.gate, (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w_router, bias,
+        bias_vl, image_mask, topk_idx, topk_w, status);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+  }
   return launch_route_t<__nv_bfloat16>(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, status, s);
 }
 

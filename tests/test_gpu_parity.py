@@ -350,10 +350,10 @@ def test_binding_rejects_mismatched_out(B, W):
 
 @pytest.mark.parametrize("name", ["sqrt_fp4_pair", "sqrt_fp4"])
 def test_fp4_direct_matches_expanded_weights(B, W, name):
-    # NVFP4 codes expanded on chip (into TMEM, the MMA's A operand) give the
-    # MMA the same operand bits as weights expanded beforehand (every e2m1 *
-    # e4m3 product is exact in bf16), and the k-blocks are accumulated in the
-    # same order: bit for bit the bf16 GEMM on the expanded weights
+    # NVFP4 codes converted to bf16 in shared memory give the MMA the same
+    # operand bits as weights expanded beforehand (every e2m1 * e4m3 product is
+    # exact in bf16): bit for bit the bf16 GEMM (same 128-row tiles) on the
+    # expanded weights
     p = H.small(name)
     c = Case(B, W, p)
     idx, w = B.route_topk(c.cfg, c.x, c.w, c.mask)
@@ -493,9 +493,9 @@ def test_shared_expert_added_once_each_k(B, W, k):
 
 
 def test_fp4_uneven_experts(B, W):
-    # the NVFP4 GEMMs size each token tile to its expert: an empty expert, one
-    # expert with most rows (several token tiles) and odd counts elsewhere;
-    # both projections read the packed weights (F % 256 == 0)
+    # the NVFP4 GEMMs with very uneven experts: an empty expert, one expert
+    # with most rows (several 128-row tiles) and odd counts elsewhere; both
+    # projections read the packed weights (F % 256 == 0)
     p = synth.PROBLEMS["sqrt_fp4"].with_(name="fp4_uneven", T=333, D=512, F=512, E=8, k=2, Fs=256)
     a = synth.generate(p)
     bias = np.zeros(p.E, dtype=np.float32)
