@@ -40,7 +40,9 @@ constexpr uint64_t kRWaitNs = 2000000000ull;
 constexpr uint64_t kRDrainNs = 200000000ull;
 
 struct RParams {
-  int T, D, E, E_pad, k, gate, stages, b_rows;
+  int T, D, E;
+  int E_pad;  // expert columns of one CTA (a multiple of 16); CTA (x, y) covers [y * E_pad, (y + 1) * E_pad)
+  int k, gate, stages, b_rows;
   float *logits;  // [T, ld] fp32 out (router logit bias included in softmax mode)
   int ld;         // logit row stride: E_pad rounded up to whole 32-column chunks
   int n_acc;  // independent accumulators over interleaved k-blocks (shorter fp32 sums)
@@ -93,6 +95,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
   RSmem &sm = *reinterpret_cast<RSmem *>(base + (size_t)p.stages * stage_bytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * RBM;
+  const int e0 = blockIdx.y * p.E_pad;              // this CTA's first expert column
+  const int e_cnt = min(p.E_pad, p.E - e0);         // of which real experts
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.stages; ++s) {
@@ -135,7 +139,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
         ptx::mbar_arrive_expect_tx(&sm.full[s], stage_bytes);
         uint8_t *a = base + (size_t)s * stage_bytes;
         ptx::tma_load_2d(a, &tmX, &sm.full[s], kb * RBK, m0);
-        for (int j = 0; j < n_boxes; ++j) ptx::tma_load_2d(a + a_bytes + j * 16384, &tmW, &sm.full[s], kb * RBK, j * 128);
+        for (int j = 0; j < n_boxes; ++j)
+          ptx::tma_load_2d(a + a_bytes + j * 16384, &tmW, &sm.full[s], kb * RBK, e0 + j * 128);
         last = kb;
       }
       // drain the copies still in flight (the last `stages` k-blocks)
@@ -182,7 +187,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
     if (__shfl_sync(0xffffffffu, ok, 0)) {
       ptx::tc_fence_after();
       const bool live = row < p.T;
-      float *dst = p.logits + (long)row * p.ld;  // chunk c writes columns [c, c + 32) < ld
+      float *dst = p.logits + (long)row * p.ld + e0;  // this CTA's columns [e0, e0 + E_pad) of the row
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16);
       for (int c = 0; c < p.E_pad; c += 32) {
         uint32_t v[32];
@@ -200,11 +205,13 @@ __global__ void __launch_bounds__(kRThreads, 1)
         if (live) {
 #pragma unroll
           for (int j = 0; j < 32; j += 4) {
+            if (c + j >= p.E_pad) break;  // the next CTA's columns
+            const float *bb = sm.bias + e0 + c + j;
             float4 o;
-            o.x = c + j < p.E ? lsum[j] + sm.bias[c + j] : -INFINITY;
-            o.y = c + j + 1 < p.E ? lsum[j + 1] + sm.bias[c + j + 1] : -INFINITY;
-            o.z = c + j + 2 < p.E ? lsum[j + 2] + sm.bias[c + j + 2] : -INFINITY;
-            o.w = c + j + 3 < p.E ? lsum[j + 3] + sm.bias[c + j + 3] : -INFINITY;
+            o.x = c + j < e_cnt ? lsum[j] + bb[0] : -INFINITY;
+            o.y = c + j + 1 < e_cnt ? lsum[j + 1] + bb[1] : -INFINITY;
+            o.z = c + j + 2 < e_cnt ? lsum[j + 2] + bb[2] : -INFINITY;
+            o.w = c + j + 3 < e_cnt ? lsum[j + 3] + bb[3] : -INFINITY;
             *reinterpret_cast<float4 *>(dst + c + j) = o;
           }
         }
@@ -268,7 +275,21 @@ moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void 
   p.T = T;
   p.D = c.hidden_dim;
   p.E = c.num_experts;
-  p.E_pad = (c.num_experts + 15) / 16 * 16;
+  // Split the expert columns over 2-4 CTAs per 128 tokens when E allows it
+  // (each part a multiple of 16) and the grid still fits in one wave: at a
+  // few thousand tokens one CTA per 128 tokens would leave most SMs idle.
+  int dev = 0, sms = 148;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const int e_pad_all = (c.num_experts + 15) / 16 * 16;
+  const long m_tiles = (T + RBM - 1) / RBM;
+  int split = 1;
+  for (int sp = 4; sp >= 2; --sp)
+    if (e_pad_all % (16 * sp) == 0 && m_tiles * sp <= sms) {
+      split = sp;
+      break;
+    }
+  p.E_pad = e_pad_all / split;
   p.b_rows = (p.E_pad + 127) / 128 * 128;
   p.k = c.top_k;
   p.gate = c.gate;
@@ -290,13 +311,10 @@ moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void 
   if (!tma_map_bf16(&tx, x, 2, (uint64_t)p.D, (uint64_t)T, 1)) return MOE_ERR_CUDA;
   if (!tma_map_bf16(&tw, w_router, 2, (uint64_t)p.D, (uint64_t)p.E, 1)) return MOE_ERR_CUDA;
   const size_t smem = 1024 + (size_t)p.stages * stage_bytes + sizeof(RSmem);
-  const dim3 grid((T + RBM - 1) / RBM);
+  const dim3 grid((unsigned)m_tiles, (unsigned)split);
   MOE_CUDA_TRY(cudaFuncSetAttribute(tc_route_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   tc_route_topk<<<grid, kRThreads, smem, s>>>(tx, tw, p);
   MOE_LAUNCH_CHECK();
-  int dev = 0, sms = 148;
-  MOE_CUDA_TRY(cudaGetDevice(&dev));
-  MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   long sel_blocks = ((long)T + kSelWarps - 1) / kSelWarps;
   if (sel_blocks > (long)sms * 8) sel_blocks = (long)sms * 8;
   const bool sel = c.gate != MOE_GATE_SOFTMAX_TOPK_RENORM;  // softmax: the logit bias is already in the logits
