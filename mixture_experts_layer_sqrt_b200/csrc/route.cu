@@ -212,11 +212,43 @@ __global__ void __launch_bounds__(32 * kMmaWarps) route_mma_kernel(int T, int D,
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[h][n][q] = 0.0f;
   const __nv_bfloat16 *xr = xs + (size_t)g * ld + 2 * c;
-  int step = 0;
-  for (int k0 = warp * 16; k0 < D; k0 += kMmaWarps * 16, ++step) {
+  // Steps are taken four at a time with every operand load of the four issued
+  // before their MMAs (the W_r fragments come from L1/L2, so their latency has
+  // to overlap); step j of the warp feeds accumulator set j & 1.
+  constexpr int kAhead = 4;
+  const int n_steps = (D / 16 - warp + kMmaWarps - 1) / kMmaWarps;  // this warp's 16-wide steps
+  int j0 = 0;
+  for (; j0 + kAhead <= n_steps; j0 += kAhead) {
+    uint32_t a[kAhead][4], b[kAhead][4][2];
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u) {
+      const int k0 = (warp + (j0 + u) * kMmaWarps) * 16;
+      a[u][0] = *reinterpret_cast<const uint32_t *>(xr + k0);
+      a[u][1] = 0u;  // rows 8..15
+      a[u][2] = *reinterpret_cast<const uint32_t *>(xr + k0 + 8);
+      a[u][3] = 0u;
+#pragma unroll
+      for (int n = 0; n < 4; ++n) {
+        const int e = n * 8 + g;
+        b[u][n][0] = b[u][n][1] = 0u;
+        if (n < n_tiles && e < E) {
+          const __nv_bfloat16 *wrow = wr + (long)e * D + k0 + 2 * c;
+          b[u][n][0] = __ldg(reinterpret_cast<const unsigned int *>(wrow));
+          b[u][n][1] = __ldg(reinterpret_cast<const unsigned int *>(wrow + 8));
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u)
+#pragma unroll
+      for (int n = 0; n < 4; ++n)
+        if (n < n_tiles) mma_bf16_16816(acc[u & 1][n], a[u], b[u][n][0], b[u][n][1]);  // j0 even: set = u & 1
+  }
+  for (int j = j0; j < n_steps; ++j) {  // the remaining steps, one at a time
+    const int k0 = (warp + j * kMmaWarps) * 16;
     uint32_t a[4];
     a[0] = *reinterpret_cast<const uint32_t *>(xr + k0);
-    a[1] = 0u;  // rows 8..15
+    a[1] = 0u;
     a[2] = *reinterpret_cast<const uint32_t *>(xr + k0 + 8);
     a[3] = 0u;
 #pragma unroll
@@ -229,7 +261,7 @@ __global__ void __launch_bounds__(32 * kMmaWarps) route_mma_kernel(int T, int D,
           b0 = __ldg(reinterpret_cast<const unsigned int *>(wrow));
           b1 = __ldg(reinterpret_cast<const unsigned int *>(wrow + 8));
         }
-        if (step & 1) mma_bf16_16816(acc[1][n], a, b0, b1);
+        if (j & 1) mma_bf16_16816(acc[1][n], a, b0, b1);
         else mma_bf16_16816(acc[0][n], a, b0, b1);
       }
     }
