@@ -162,6 +162,7 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+template <int NT>  // expert tiles of 8: ceil(E / 8)
 __global__ void __launch_bounds__(32 * kMmaWarps) route_mma_kernel(int T, int D, int E, int k, int gate,
                                                                    const __nv_bfloat16 *__restrict__ x,
                                                                    const __nv_bfloat16 *__restrict__ wr,
@@ -203,12 +204,11 @@ __global__ void __launch_bounds__(32 * kMmaWarps) route_mma_kernel(int T, int D,
     return;
   }
 
-  const int n_tiles = (E + 7) >> 3;  // <= 4
-  float acc[2][4][4];
+  float acc[2][NT][4];
 #pragma unroll
   for (int h = 0; h < 2; ++h)
 #pragma unroll
-    for (int n = 0; n < 4; ++n)
+    for (int n = 0; n < NT; ++n)
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[h][n][q] = 0.0f;
   const __nv_bfloat16 *xr = xs + (size_t)g * ld + 2 * c;
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(32 * kMmaWarps) route_mma_kernel(int T, int D,
   const int n_steps = (D / 16 - warp + kMmaWarps - 1) / kMmaWarps;  // this warp's 16-wide steps
   int j0 = 0;
   for (; j0 + kAhead <= n_steps; j0 += kAhead) {
-    uint32_t a[kAhead][4], b[kAhead][4][2];
+    uint32_t a[kAhead][4], b[kAhead][NT][2];
 #pragma unroll
     for (int u = 0; u < kAhead; ++u) {
       const int k0 = (warp + (j0 + u) * kMmaWarps) * 16;
@@ -228,10 +228,10 @@ __global__ void __launch_bounds__(32 * kMmaWarps) route_mma_kernel(int T, int D,
       a[u][2] = *reinterpret_cast<const uint32_t *>(xr + k0 + 8);
       a[u][3] = 0u;
 #pragma unroll
-      for (int n = 0; n < 4; ++n) {
+      for (int n = 0; n < NT; ++n) {
         const int e = n * 8 + g;
         b[u][n][0] = b[u][n][1] = 0u;
-        if (n < n_tiles && e < E) {
+        if (e < E) {
           const __nv_bfloat16 *wrow = wr + (long)e * D + k0 + 2 * c;
           b[u][n][0] = __ldg(reinterpret_cast<const unsigned int *>(wrow));
           b[u][n][1] = __ldg(reinterpret_cast<const unsigned int *>(wrow + 8));
@@ -241,8 +241,7 @@ __global__ void __launch_bounds__(32 * kMmaWarps) route_mma_kernel(int T, int D,
 #pragma unroll
     for (int u = 0; u < kAhead; ++u)
 #pragma unroll
-      for (int n = 0; n < 4; ++n)
-        if (n < n_tiles) mma_bf16_16816(acc[u & 1][n], a[u], b[u][n][0], b[u][n][1]);  // j0 even: set = u & 1
+      for (int n = 0; n < NT; ++n) mma_bf16_16816(acc[u & 1][n], a[u], b[u][n][0], b[u][n][1]);  // j0 even: set = u & 1
   }
   for (int j = j0; j < n_steps; ++j) {  // the remaining steps, one at a time
     const int k0 = (warp + j * kMmaWarps) * 16;
@@ -252,25 +251,23 @@ __global__ void __launch_bounds__(32 * kMmaWarps) route_mma_kernel(int T, int D,
     a[2] = *reinterpret_cast<const uint32_t *>(xr + k0 + 8);
     a[3] = 0u;
 #pragma unroll
-    for (int n = 0; n < 4; ++n) {
-      if (n < n_tiles) {
-        const int e = n * 8 + g;
-        uint32_t b0 = 0u, b1 = 0u;
-        if (e < E) {
-          const __nv_bfloat16 *wrow = wr + (long)e * D + k0 + 2 * c;
-          b0 = __ldg(reinterpret_cast<const unsigned int *>(wrow));
-          b1 = __ldg(reinterpret_cast<const unsigned int *>(wrow + 8));
-        }
-        if (j & 1) mma_bf16_16816(acc[1][n], a, b0, b1);
-        else mma_bf16_16816(acc[0][n], a, b0, b1);
+    for (int n = 0; n < NT; ++n) {
+      const int e = n * 8 + g;
+      uint32_t b0 = 0u, b1 = 0u;
+      if (e < E) {
+        const __nv_bfloat16 *wrow = wr + (long)e * D + k0 + 2 * c;
+        b0 = __ldg(reinterpret_cast<const unsigned int *>(wrow));
+        b1 = __ldg(reinterpret_cast<const unsigned int *>(wrow + 8));
       }
+      if (j & 1) mma_bf16_16816(acc[1][n], a, b0, b1);
+      else mma_bf16_16816(acc[0][n], a, b0, b1);
     }
   }
   // C fragment: d0, d1 = token g, experts n*8 + 2c, 2c + 1 (d2, d3: rows 8..15, unused)
 #pragma unroll
   for (int h = 0; h < 2; ++h)
 #pragma unroll
-    for (int n = 0; n < 4; ++n) {
+    for (int n = 0; n < NT; ++n) {
       float *dst = part + ((warp * 2 + h) * kMmaTok + g) * 32 + n * 8 + 2 * c;
       dst[0] = acc[h][n][0];
       dst[1] = acc[h][n][1];
@@ -323,8 +320,15 @@ moe_status launch_route(const MoEConfig &c, int T, const void *x, const void *w_
   if (c.num_experts <= 32 && c.hidden_dim % 16 == 0 && (size_t)kMmaTok * (c.hidden_dim + 8) * 2 <= 160 * 1024) {
     const int E = c.num_experts;
     const size_t smem = (size_t)kMmaTok * (c.hidden_dim + 8) * 2 + (8 * kMmaTok * 32 + (size_t)kMmaTok * E) * 4 + 32;
-    MOE_CUDA_TRY(cudaFuncSetAttribute(route_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    route_mma_kernel<<<(unsigned)((T + kMmaTok - 1) / kMmaTok), 32 * kMmaWarps, smem, s>>>(
+    auto kern = route_mma_kernel<4>;
+    switch ((E + 7) / 8) {
+      case 1: kern = route_mma_kernel<1>; break;
+      case 2: kern = route_mma_kernel<2>; break;
+      case 3: kern = route_mma_kernel<3>; break;
+      default: break;
+    }
+    MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    kern<<<(unsigned)((T + kMmaTok - 1) / kMmaTok), 32 * kMmaWarps, smem, s>>>(
         T, c.hidden_dim, E, c.top_k, c.gate, (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w_router, bias,
         bias_vl, image_mask, topk_idx, topk_w, status);
     MOE_LAUNCH_CHECK();
