@@ -14,25 +14,41 @@
 //                     scaled by row_weight, fp32 out.
 //
 // The expansion runs on the CUDA cores (hardware e2m1 -> f16 conversion, an
-// exponent re-bias to bf16, one bf16 multiply by the scale) and is balanced
-// between the integer-logic and the multiply-add pipes; it still sets the
-// pace (the MMAs wait on converted tiles), so every instruction per weight
-// counts.  N = 256
-// keeps the MMAs' shared-memory operand traffic low; pairs of CTAs are not
-// used because handing a converted half-tile to the peer CTA needs a
-// cluster-scope release per k-block, which costs more than converting the
-// whole tile locally.
+// exponent re-bias to bf16, one bf16 multiply by the scale; or, for f16, the
+// conversion and one f16 multiply) and is balanced between the integer-logic
+// and the multiply-add pipes.  N = 256 keeps the MMAs' shared-memory operand
+// traffic low; pairs of CTAs are not used because handing a converted
+// half-tile to the peer CTA needs a cluster-scope release per k-block, which
+// costs more than converting the whole tile locally.
 //
-// Roles (448 threads per CTA):
-//   warp 0       TMA producer: A rows (128 x 64 bf16), packed codes (256 B
-//                rows x 32 bytes) and scales (256 x 16 bytes: the 4-k-block
-//                group) per k-block into a 4-stage ring.
-//   warp 1       TMEM owner; one thread issues the MMAs (A from the TMA ring,
-//                B from the converted ring) and commits stages back.
+// Three rings, because their data have different latencies and lifetimes:
+//   A rows      (16 KB per k-block, 3 stages)  mostly L2 hits; held until the
+//               MMAs that read them complete.
+//   weights     (32 KB of codes + 4 KB of scales per 4 k-blocks, 2 stages)
+//               from DRAM, in 128-byte rows (a TMA copy costs per row moved:
+//               32-byte code rows and 16-byte scale rows every k-block made
+//               the copies, not the MMAs or the expansion, set the pace);
+//               freed as soon as every converter warp holds the bytes in
+//               registers.
+//   converted B (32 KB per k-block, 3 stages)  written by the converters,
+//               held until the MMAs that read it complete.  Each stage's round
+//               trip (expansion, hand-off, MMA issue to completion, hand-off
+//               back) takes ~2600 cycles against 512 of MMA work, so the
+//               depth of this ring, not the A or weight rings, sets the pace.
+// (One shared A + weights ring, released only after the MMA, left both the
+// MMAs and the converters waiting on copies: each alone ran at ~45% of its
+// own rate.)
+//
+// Roles (480 threads per CTA):
+//   warp 0       TMA producer of A rows (128 x 64 per k-block; or a 4-row
+//                gather per lane through a row map).
+//   warp 1       TMEM owner; one thread issues the MMAs (A from its ring, B
+//                from the converted ring) and commits both stages back.
 //   warps 2-5    epilogue: TMEM -> registers -> SwiGLU or routing weight ->
 //                global stores; two 256-column accumulators overlap tiles.
-//   warps 6-13   converters: codes + scales -> swizzled bf16 B tile (3-stage
-//                ring), one arrival per warp.
+//   warp 6       TMA producer of the packed codes and scales.
+//   warps 7-14   converters: codes + scales -> swizzled 16-bit B tile, one
+//                arrival per warp.
 //
 // F16 (gate/up inside moe_forward): A arrives as f16 rows pre-scaled by a
 // power of two per row (launch_gather_f16), the codes are expanded to f16
@@ -64,23 +80,29 @@ constexpr int TILE_M = 128;                     // rows per tile (TMEM lanes)
 constexpr int FN = 256;                         // MMA N: B rows per k-block
 constexpr int A_BYTES = TILE_M * BK * 2;        // 16 KB
 constexpr int B_BYTES = FN * BK * 2;            // 32 KB
-constexpr int RAW_BYTES = FN * BK / 2;          // 8 KB of e2m1 codes
-constexpr int SCL_BYTES = FN * 16;              // 4 KB of e4m3 scales (4 k-blocks)
-constexpr int STAGES = 4;
-constexpr int B_STAGES = 3;
+constexpr int KW = 4;                           // k-blocks per weight stage
+constexpr int RAW_BYTES = FN * KW * BK / 2;     // 32 KB of e2m1 codes: 128-byte rows
+constexpr int SCL_BYTES = FN * 16;              // 4 KB of e4m3 scales (the same 4 k-blocks)
+constexpr int W_BYTES = RAW_BYTES + SCL_BYTES;  // one weight stage
+constexpr int A_STAGES = 3;                     // A rows (mostly L2 hits)
+constexpr int W_STAGES = 2;                     // codes + scales (DRAM): 8 k-blocks
+constexpr int B_STAGES = 3;                     // converted B tiles
 constexpr int kConv = 8;                        // converter warps
-constexpr int kThreads = 192 + 32 * kConv;
+constexpr int kWProducer = 6;                   // the weight producer's warp
+constexpr int kConv0 = 7;                       // first converter warp
+constexpr int kThreads = 32 * (kConv0 + kConv);
 constexpr uint32_t TMEM_COLS = 512;             // 2 accumulators x FN
-constexpr uint32_t TX_BYTES = A_BYTES + RAW_BYTES + SCL_BYTES;
 constexpr int MAX_E = 1024;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s
 
 struct Smem {
-  uint64_t full[STAGES];      // A, codes and scales of the k-block landed
-  uint64_t empty[STAGES];     // the MMAs reading the stage's A completed
-  uint64_t b_full[B_STAGES];  // converted B tile written
-  uint64_t b_empty[B_STAGES];
+  uint64_t a_full[A_STAGES];   // A rows of the k-block landed
+  uint64_t a_empty[A_STAGES];  // the MMAs reading them completed
+  uint64_t w_full[W_STAGES];   // codes and scales landed
+  uint64_t w_empty[W_STAGES];  // every converter warp holds them in registers
+  uint64_t b_full[B_STAGES];   // converted B tile written
+  uint64_t b_empty[B_STAGES];  // the MMAs reading it completed
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t drain;
@@ -104,16 +126,22 @@ struct Params {
   const float *row_scale;    // F16: 2^-s_r of each A row
 };
 
+// The waits of this kernel spin instead of suspending: its k-block period is
+// a chain of hand-offs (converters -> MMA -> completion -> converters), and a
+// suspended waiter wakes late enough to lengthen every link (measured: 5%).
+// The clock is read every 64 polls.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Smem &sm, int *status) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
-  while (true) {
-    if (ptx::mbar_try_wait_sleep(bar, parity, ptx::kWaitHintNs)) return true;
-    if (*(volatile int *)&sm.abort) return false;
-    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
-      *(volatile int *)&sm.abort = 1;
-      atomicExch(status, kDevTimeout);
-      return false;
+  for (uint32_t n = 1;; ++n) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((n & 63u) == 0) {
+      if (*(volatile int *)&sm.abort) return false;
+      if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+        *(volatile int *)&sm.abort = 1;
+        atomicExch(status, kDevTimeout);
+        return false;
+      }
     }
   }
 }
@@ -206,17 +234,14 @@ __device__ __forceinline__ uint4 expand_e2m1x8(uint32_t q, uint32_t scale2, uint
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// e4m3 scale byte -> f16x2 of the scale, both halves (exact: e4m3 values are
-// normal f16 numbers).
+// e4m3 scale byte -> f16x2 of the scale, both halves: the hardware e4m3 pair
+// conversion of the byte twice (exact: every e4m3 value, subnormals and the
+// NaN code included, is a normal f16 number or NaN).
 __device__ __forceinline__ uint32_t scale_f16x2(uint32_t b) {
-  const uint32_t E = (b >> 3) & 15u, m = b & 7u;
-  float v;
-  if (E == 15u && m == 7u) v = __uint_as_float(0x7fc00000u);          // the NaN code
-  else if (E) v = __uint_as_float(((E + 120u) << 23) | (m << 20));     // 2^(E-7) (1 + m/8)
-  else v = (float)m * __uint_as_float(118u << 23);                     // m 2^-9
-  if (b & 0x80u) v = -v;
-  const uint32_t h = __half_as_ushort(__float2half_rn(v));
-  return h | (h << 16);
+  uint32_t d;
+  const uint16_t two = (uint16_t)(b * 0x0101u);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(two));
+  return d;
 }
 
 // Eight e2m1 codes times one scale (from scale_f16x2) -> eight f16; each
@@ -239,20 +264,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ CUtensorMap tmS1, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t *stage_a = base;                                  // STAGES x 16 KB (1024-aligned)
-  uint8_t *stage_b = stage_a + STAGES * A_BYTES;            // B_STAGES x 32 KB
-  uint8_t *stage_raw = stage_b + B_STAGES * B_BYTES;        // STAGES x 8 KB
-  uint8_t *stage_scl = stage_raw + STAGES * RAW_BYTES;      // STAGES x 4 KB
-  uint32_t *lut = reinterpret_cast<uint32_t *>(stage_scl + STAGES * SCL_BYTES);
-  Smem &sm = *reinterpret_cast<Smem *>(stage_scl + STAGES * SCL_BYTES + 1024);
+  uint8_t *stage_a = base;                                  // A_STAGES x 16 KB (1024-aligned)
+  uint8_t *stage_b = stage_a + A_STAGES * A_BYTES;          // B_STAGES x 32 KB
+  uint8_t *stage_w = stage_b + B_STAGES * B_BYTES;          // W_STAGES x (32 KB codes + 4 KB scales)
+  uint32_t *lut = reinterpret_cast<uint32_t *>(stage_w + W_STAGES * W_BYTES);
+  Smem &sm = *reinterpret_cast<Smem *>(stage_w + W_STAGES * W_BYTES + 1024);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- setup: barriers, TMEM, scale table, tile schedule
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(&sm.full[s], 1);
-      ptx::mbar_init(&sm.empty[s], 1);
+    for (int s = 0; s < A_STAGES; ++s) {
+      ptx::mbar_init(&sm.a_full[s], 1);
+      ptx::mbar_init(&sm.a_empty[s], 1);
+    }
+    for (int s = 0; s < W_STAGES; ++s) {
+      ptx::mbar_init(&sm.w_full[s], 1);
+      ptx::mbar_init(&sm.w_empty[s], kConv);
     }
     for (int b = 0; b < B_STAGES; ++b) {
       ptx::mbar_init(&sm.b_full[b], kConv);
@@ -267,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::fence_mbar_init();
     ptx::fence_proxy_async_smem();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == kWProducer && lane == 0) {
     ptx::prefetch_tmap(&tmA);
     ptx::prefetch_tmap(&tmB0);
     ptx::prefetch_tmap(&tmS0);
@@ -308,9 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (any_bad && blockIdx.x == 0) note_violation();
     }
   }
-  if (warp >= 6) {
-    for (int b = (int)threadIdx.x - 192; b < 256; b += 32 * kConv)
-      lut[b] = F16 ? scale_f16x2((uint32_t)b) : scale_bf16x2((uint32_t)b);
+  if (!F16 && warp >= kConv0) {
+    for (int b = (int)threadIdx.x - 32 * kConv0; b < 256; b += 32 * kConv) lut[b] = scale_bf16x2((uint32_t)b);
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -320,15 +347,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int k_blocks = p.K / BK;
 
   if (warp == 0) {
-    // ================================================= TMA producer
-    // Dense A: lane 0 issues everything.  Gathered A: each lane gathers its 4
-    // rows of the tile (one 4-row TMA gather per k-block).
+    // ================================================= TMA producer: A rows
+    // Dense A: lane 0 issues the 128-row box.  Gathered A: each lane gathers
+    // its 4 rows of the tile (one 4-row TMA gather per k-block).
     const bool gather = p.row_token != nullptr;
     if (gather || lane == 0) {
-      uint32_t last_parity[STAGES];
-      bool used[STAGES];
+      uint32_t last_parity[A_STAGES];
+      bool used[A_STAGES];
 #pragma unroll
-      for (int s = 0; s < STAGES; ++s) {
+      for (int s = 0; s < A_STAGES; ++s) {
         used[s] = false;
         last_parity[s] = 0;
       }
@@ -344,39 +371,72 @@ __global__ void __launch_bounds__(kThreads, 1)
             tok[i] = r < tl.end ? p.row_token[r] : p.src_rows;  // out of range: zero fill
           }
         }
-        const int n0 = GATED ? tl.n_blk * (FN / 2) : tl.n_blk * FN;
-        const int n1 = GATED ? n0 : n0 + FN / 2;
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1u;
+          const int s = it % A_STAGES;
+          const uint32_t ph = (it / A_STAGES) & 1u;
           bool got = true;
-          if (lane == 0) got = wait_bar(&sm.empty[s], ph ^ 1u, sm, p.status);
+          if (lane == 0) got = wait_bar(&sm.a_empty[s], ph ^ 1u, sm, p.status);
           if (gather) got = __shfl_sync(0xffffffffu, got, 0);
           if (!got) {
             ok = false;
             break;
           }
-          const int k0 = kb * BK;
           uint8_t *a = stage_a + s * A_BYTES;
           if (lane == 0) {
-            uint8_t *raw = stage_raw + s * RAW_BYTES;
-            uint8_t *scl = stage_scl + s * SCL_BYTES;
-            ptx::mbar_arrive_expect_tx(&sm.full[s], TX_BYTES);
-            if (!gather) ptx::tma_load_2d(a, &tmA, &sm.full[s], k0, tl.m0);
-            ptx::tma_load_3d(raw, &tmB0, &sm.full[s], kb * (BK / 2), n0, tl.e);
-            ptx::tma_load_3d(raw + RAW_BYTES / 2, GATED ? &tmB1 : &tmB0, &sm.full[s], kb * (BK / 2), n1, tl.e);
-            ptx::tma_load_3d(scl, &tmS0, &sm.full[s], (kb >> 2) * 16, n0, tl.e);
-            ptx::tma_load_3d(scl + SCL_BYTES / 2, GATED ? &tmS1 : &tmS0, &sm.full[s], (kb >> 2) * 16, n1, tl.e);
+            ptx::mbar_arrive_expect_tx(&sm.a_full[s], A_BYTES);
+            if (!gather) ptx::tma_load_2d(a, &tmA, &sm.a_full[s], kb * BK, tl.m0);
           }
-          if (gather) ptx::tma_gather4(a + lane * 512, &tmA, &sm.full[s], k0, tok[0], tok[1], tok[2], tok[3]);
+          if (gather) ptx::tma_gather4(a + lane * 512, &tmA, &sm.a_full[s], kb * BK, tok[0], tok[1], tok[2], tok[3]);
           used[s] = true;
           last_parity[s] = ph;
         }
       }
       if (lane == 0) {
-        for (int s = 0; s < STAGES; ++s)
-          if (used[s]) drain_bar(&sm.full[s], last_parity[s], p.status);
+        for (int s = 0; s < A_STAGES; ++s)
+          if (used[s]) drain_bar(&sm.a_full[s], last_parity[s], p.status);
       }
+    }
+  } else if (warp == kWProducer) {
+    // ================================================= TMA producer: weights
+    // Per stage, four k-blocks: packed codes (256 B rows x 128 bytes, 128-byte
+    // swizzle) and their scales (256 x 16 bytes).  The TMA's cost goes with
+    // the rows it moves, so rows as wide as the swizzle allows, one stage per
+    // four k-blocks; the converters free a stage as soon as they hold its
+    // last k-block's bytes in registers.
+    if (lane == 0) {
+      uint32_t last_parity[W_STAGES];
+      bool used[W_STAGES];
+#pragma unroll
+      for (int s = 0; s < W_STAGES; ++s) {
+        used[s] = false;
+        last_parity[s] = 0;
+      }
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const Tile tl = decode_tile(p, sm, t);
+        const int n0 = GATED ? tl.n_blk * (FN / 2) : tl.n_blk * FN;
+        const int n1 = GATED ? n0 : n0 + FN / 2;
+        for (int kw = 0; kw < k_blocks / KW; ++kw, ++it) {
+          const int s = it % W_STAGES;
+          const uint32_t ph = (it / W_STAGES) & 1u;
+          if (!wait_bar(&sm.w_empty[s], ph ^ 1u, sm, p.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t *raw = stage_w + s * W_BYTES;
+          uint8_t *scl = raw + RAW_BYTES;
+          ptx::mbar_arrive_expect_tx(&sm.w_full[s], W_BYTES);
+          ptx::tma_load_3d(raw, &tmB0, &sm.w_full[s], kw * 128, n0, tl.e);
+          ptx::tma_load_3d(raw + RAW_BYTES / 2, GATED ? &tmB1 : &tmB0, &sm.w_full[s], kw * 128, n1, tl.e);
+          ptx::tma_load_3d(scl, &tmS0, &sm.w_full[s], kw * 16, n0, tl.e);
+          ptx::tma_load_3d(scl + SCL_BYTES / 2, GATED ? &tmS1 : &tmS0, &sm.w_full[s], kw * 16, n1, tl.e);
+          used[s] = true;
+          last_parity[s] = ph;
+        }
+      }
+      for (int s = 0; s < W_STAGES; ++s)
+        if (used[s]) drain_bar(&sm.w_full[s], last_parity[s], p.status);
     }
   } else if (warp == 1) {
     // ================================================= MMA issuer
@@ -390,9 +450,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_bar(&sm.tmem_empty[acc], ((i >> 1) & 1u) ^ 1u, sm, p.status)) break;
         ptx::tc_fence_after();
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
-          const int s = it % STAGES;
+          const int s = it % A_STAGES;
           const int sb = it % B_STAGES;
-          if (!wait_bar(&sm.full[s], (it / STAGES) & 1u, sm, p.status) ||
+          if (!wait_bar(&sm.a_full[s], (it / A_STAGES) & 1u, sm, p.status) ||
               !wait_bar(&sm.b_full[sb], (it / B_STAGES) & 1u, sm, p.status)) {
             ok = false;
             break;
@@ -407,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t bd = ptx::desc_kmajor_sw128(b_addr + k * UMMA_K * 2);
             ptx::mma_bf16(d_tmem, ad, bd, idesc, (kb | k) != 0);
           }
-          ptx::mma_commit(&sm.empty[s]);
+          ptx::mma_commit(&sm.a_empty[s]);
           ptx::mma_commit(&sm.b_empty[sb]);
         }
         if (!ok) break;
@@ -484,50 +544,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&sm.tmem_empty[acc]);
     }
-  } else {
-    // ================================================= converters (warps 6..13)
-    // Per k-block 256 B rows x 8 chunks of 8 elements: thread ct takes chunk
-    // ct % 8 of rows ct / 8 + 32 i.  A warp reads 4 whole rows of codes (128
-    // contiguous bytes) and writes 4 whole 128-byte rows of the swizzled tile
-    // (chunk c of row r at 16 * (c ^ (r % 8))): no bank conflicts.  All loads
-    // of a k-block are issued before its stores so their latencies overlap.
-    constexpr int ROW_STEP = 32 * kConv / 8;
-    constexpr int JOBS = FN / ROW_STEP;
-    const int ct = (int)threadIdx.x - 192;
-    const int c = ct & 7, r0 = ct >> 3;
-    const int raw_off = r0 * (BK / 2) + c * 4;
-    const int scl_off = r0 * 16 + (c >> 1);
-    const int b_off = r0 * (BK * 2) + ((c ^ (r0 & 7)) << 4);
+  } else if (warp >= kConv0) {
+    // ================================================= converters (kConv warps)
+    // Per k-block 256 B rows x 4 groups of 16 codes, one e4m3 scale each:
+    // thread ct takes group ct % 4 of rows ct / 4 + 64 j.  A group is one
+    // 8-byte load of codes, one scale conversion and two 16-byte stores into
+    // the swizzled tile (chunk c of row r at 16 * (c ^ (r % 8))); a warp's
+    // stores cover 8 whole 128-byte rows, four wavefronts each, the minimum.
+    // Codes of k-block kb: bytes 32 (kb % 4) .. +31 of each 128-byte row,
+    // stored swizzled (16-byte chunk c of row r at chunk c ^ (r % 8)), so a
+    // warp's 8 rows read different banks.  The weight stage is released once
+    // its fourth k-block's bytes are in registers.
+    constexpr int ROWS_PER_PASS = 32 * kConv / 4;
+    constexpr int JOBS = FN / ROWS_PER_PASS;
+    const int ct = (int)threadIdx.x - 32 * kConv0;
+    const int g = ct & 3, r0 = ct >> 2;
+    const int scl_off = RAW_BYTES + r0 * 16 + g;
+    const int b_off0 = r0 * (BK * 2) + (((2 * g) ^ (r0 & 7)) << 4);
+    const int b_off1 = r0 * (BK * 2) + (((2 * g + 1) ^ (r0 & 7)) << 4);
     uint32_t it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
       for (int kb = 0; kb < k_blocks; ++kb, ++it) {
-        const int s = it % STAGES;
+        const uint32_t iw = it / KW;  // weight stages so far (every tile starts a stage: k_blocks % KW == 0)
+        const int sw = iw % W_STAGES;
         const int sb = it % B_STAGES;
-        bool got = true;
-        if (lane == 0) {
-          got = wait_bar(&sm.full[s], (it / STAGES) & 1u, sm, p.status) &&
-                wait_bar(&sm.b_empty[sb], ((it / B_STAGES) & 1u) ^ 1u, sm, p.status);
-        }
-        if (!__shfl_sync(0xffffffffu, got, 0)) {
+        const int kq = kb & (KW - 1);
+        if (kq == 0 && !warp_wait(&sm.w_full[sw], (iw / W_STAGES) & 1u, sm, p.status, lane)) {
           ok = false;
           break;
         }
-        const uint8_t *raw = stage_raw + s * RAW_BYTES + raw_off;
-        const uint8_t *scl = stage_scl + s * SCL_BYTES + scl_off + (kb & 3) * 4;
-        uint8_t *dst = stage_b + sb * B_BYTES + b_off;
-        uint32_t qv[JOBS], sc[JOBS];
+        const uint8_t *w = stage_w + sw * W_BYTES;
+        const int raw_off = r0 * 128 + (((2 * kq + (g >> 1)) ^ (r0 & 7)) << 4) + (g & 1) * 8;
+        uint2 qv[JOBS];
+        uint32_t sc[JOBS];
 #pragma unroll
         for (int j = 0; j < JOBS; ++j) {
-          qv[j] = *reinterpret_cast<const uint32_t *>(raw + j * ROW_STEP * (BK / 2));
-          sc[j] = scl[j * ROW_STEP * 16];
+          qv[j] = *reinterpret_cast<const uint2 *>(w + raw_off + j * ROWS_PER_PASS * 128);
+          sc[j] = w[scl_off + kq * 4 + j * ROWS_PER_PASS * 16];
+        }
+        if (kq == KW - 1) {
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&sm.w_empty[sw]);  // release-ordered after the loads above
         }
 #pragma unroll
-        for (int j = 0; j < JOBS; ++j) sc[j] = lut[sc[j]];
+        for (int j = 0; j < JOBS; ++j) sc[j] = F16 ? scale_f16x2(sc[j]) : lut[sc[j]];
+        if (!warp_wait(&sm.b_empty[sb], ((it / B_STAGES) & 1u) ^ 1u, sm, p.status, lane)) {
+          ok = false;
+          break;
+        }
+        uint8_t *dst = stage_b + sb * B_BYTES;
 #pragma unroll
-        for (int j = 0; j < JOBS; ++j)
-          *reinterpret_cast<uint4 *>(dst + j * ROW_STEP * (BK * 2)) =
-              F16 ? expand_e2m1x8_f16(qv[j], sc[j]) : expand_e2m1x8(qv[j], sc[j], p.hi_mul);
+        for (int j = 0; j < JOBS; ++j) {
+          const int rb = j * ROWS_PER_PASS * (BK * 2);  // ROWS_PER_PASS % 8 == 0: the swizzle phase is kept
+          *reinterpret_cast<uint4 *>(dst + b_off0 + rb) =
+              F16 ? expand_e2m1x8_f16(qv[j].x, sc[j]) : expand_e2m1x8(qv[j].x, sc[j], p.hi_mul);
+          *reinterpret_cast<uint4 *>(dst + b_off1 + rb) =
+              F16 ? expand_e2m1x8_f16(qv[j].y, sc[j]) : expand_e2m1x8(qv[j].y, sc[j], p.hi_mul);
+        }
         ptx::fence_proxy_async_smem();  // the MMA reads these stores through the async proxy
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&sm.b_full[sb]);
@@ -545,8 +619,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-constexpr size_t kSmemBytes =
-    1024 + (size_t)STAGES * (A_BYTES + RAW_BYTES + SCL_BYTES) + (size_t)B_STAGES * B_BYTES + 1024 + sizeof(Smem);
+constexpr size_t kSmemBytes = 1024 + (size_t)A_STAGES * A_BYTES + (size_t)B_STAGES * B_BYTES +
+                              (size_t)W_STAGES * W_BYTES + 1024 + sizeof(Smem);
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 // A: [rows, K] bf16 (or the gather source); codes [E, Nw, K/2] bytes and
@@ -558,10 +632,10 @@ moe_status launch_fp4(const Params &p, const void *a, const void *b0, const void
   const uint64_t K = (uint64_t)p.K;
   if (!tma_map_bf16(&ta, a, 2, K, (uint64_t)(p.row_token ? p.src_rows : p.rows), 1, p.row_token ? 1 : TILE_M))
     return MOE_ERR_CUDA;
-  if (!tma_map_u8(&tb0, b0, K / 2, (uint64_t)Nw, (uint64_t)p.E, BK / 2, FN / 2)) return MOE_ERR_CUDA;
+  if (!tma_map_u8(&tb0, b0, K / 2, (uint64_t)Nw, (uint64_t)p.E, 128, FN / 2, true)) return MOE_ERR_CUDA;
   if (!tma_map_u8(&ts0, s0, K / 16, (uint64_t)Nw, (uint64_t)p.E, 16, FN / 2)) return MOE_ERR_CUDA;
   if (GATED) {
-    if (!tma_map_u8(&tb1, b1, K / 2, (uint64_t)Nw, (uint64_t)p.E, BK / 2, FN / 2)) return MOE_ERR_CUDA;
+    if (!tma_map_u8(&tb1, b1, K / 2, (uint64_t)Nw, (uint64_t)p.E, 128, FN / 2, true)) return MOE_ERR_CUDA;
     if (!tma_map_u8(&ts1, s1, K / 16, (uint64_t)Nw, (uint64_t)p.E, 16, FN / 2)) return MOE_ERR_CUDA;
   } else {
     tb1 = tb0;
