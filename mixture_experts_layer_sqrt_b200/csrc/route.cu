@@ -144,15 +144,24 @@ __global__ void __launch_bounds__(512) route_kernel(int T, int D, int E, int k, 
 
 // bf16 activations, E <= 32: the logits on the tensor cores with the
 // warp-level mma.sync (m16n8k16, bf16 in, fp32 accumulate), so the kernel is
-// left with streaming x.  A block owns 8 tokens: one thread bulk-copies their
-// x rows into shared memory (rows padded by 16 bytes so the fragment loads of
-// the 8 rows fall in different banks), and 4 warps each take every fourth
-// 16-wide step of D into two accumulator sets (alternate steps).  The 8
-// partial sums per logit (4 warps x 2 sets) are added in a fixed order,
-// which keeps each fp32 sum short, as the tensor-core router's split-K
-// accumulators do.  Rows 8..15 of every MMA are zero.
-constexpr int kMmaTok = 8;
-constexpr int kMmaWarps = 4;
+// left with streaming x at HBM speed.  A block takes groups of 16 tokens (the
+// MMA's 16 rows); one producer thread streams, per 512-wide slice of D, the
+// group's 16 x rows and the E router rows into a ring of 4 stages (3 for
+// E > 16) with bulk copies, rows padded by 16 bytes so that ldmatrix reads
+// hit 8 different bank groups.  8 consumer warps each take every eighth
+// 16-wide step of a slice into two accumulator sets (alternate steps).  A
+// stage is released as soon as its reads are done, so the copies of the next
+// slices, and of the next group, stay in flight while the tensor cores work.
+// At the end of a group the 16 partial sums per logit (8 warps x 2 sets) are
+// added in a fixed order, which keeps each fp32 sum short (the routing
+// weights are held to 1e-5), and each consumer warp selects for two tokens.
+// Rows of the last group past T repeat row T-1 and are never selected.
+constexpr int kRGTok = 16;    // tokens per group (MMA rows)
+constexpr int kRDC = 512;     // D per stage
+template <int NT>
+constexpr int route_stages() { return NT <= 2 ? 4 : 3; }  // ring depth within 227 KB of shared memory
+constexpr int kRWarps = 8;    // consumer warps; one more warp produces
+constexpr int kRRowBytes = (kRDC + 8) * 2;
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -161,128 +170,173 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void *p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(ptx::smem_addr(p)));
+}
+__device__ __forceinline__ void ldmatrix_x2(uint32_t &r0, uint32_t &r1, const void *p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(ptx::smem_addr(p)));
+}
+
+// Bounded wait; gives up at once when the block is aborting.
+__device__ __forceinline__ bool route_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (*abort_flag) return false;
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((n & 63u) == 0 && ptx::globaltimer_ns() - t0 > kRouteWaitNs) {
+      *abort_flag = 1;
+      if (status) atomicExch(status, kDevTimeout);
+      return false;
+    }
+  }
+}
 
 template <int NT>  // expert tiles of 8: ceil(E / 8)
-__global__ void __launch_bounds__(32 * kMmaWarps) route_mma_kernel(int T, int D, int E, int k, int gate,
-                                                                   const __nv_bfloat16 *__restrict__ x,
-                                                                   const __nv_bfloat16 *__restrict__ wr,
-                                                                   const float *__restrict__ bias,
-                                                                   const float *__restrict__ bias_vl,
-                                                                   const uint8_t *__restrict__ image_mask,
-                                                                   int32_t *__restrict__ topk_idx,
-                                                                   float *__restrict__ topk_w, int *status) {
+constexpr size_t route_ring_smem() {
+  return (size_t)route_stages<NT>() * (kRGTok + NT * 8) * kRRowBytes + (size_t)2 * kRWarps * kRGTok * NT * 8 * 4 +
+         (size_t)kRGTok * NT * 8 * 4 + 2 * route_stages<NT>() * 8 + 16;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(32 * (kRWarps + 1), 1) route_ring_kernel(int T, int D, int E, int k, int gate,
+                                                                     const __nv_bfloat16 *__restrict__ x,
+                                                                     const __nv_bfloat16 *__restrict__ wr,
+                                                                     const float *__restrict__ bias,
+                                                                     const float *__restrict__ bias_vl,
+                                                                     const uint8_t *__restrict__ image_mask,
+                                                                     int32_t *__restrict__ topk_idx,
+                                                                     float *__restrict__ topk_w, int *status) {
+  constexpr int kRStages = route_stages<NT>();
+  constexpr int ROWS = kRGTok + NT * 8;  // x rows, then router rows, per stage
+  constexpr int STAGE = ROWS * kRRowBytes;
+  constexpr int EP = NT * 8;
   extern __shared__ __align__(128) uint8_t smem[];
-  const int ld = D + 8;  // padded row length in bf16 (16 bytes of padding)
-  __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(smem);                      // [kMmaTok][ld]
-  float *part = reinterpret_cast<float *>(smem + (size_t)kMmaTok * ld * 2);         // [8 sums][kMmaTok][32]
-  float *logits = part + 8 * kMmaTok * 32;                                           // [kMmaTok][E]
-  uint64_t *bar = reinterpret_cast<uint64_t *>(((uintptr_t)(logits + kMmaTok * E) + 15) & ~(uintptr_t)15);
+  uint8_t *stages = smem;
+  float *part = reinterpret_cast<float *>(smem + kRStages * STAGE);  // [2 * kRWarps][kRGTok][EP]
+  float *logits = part + 2 * kRWarps * kRGTok * EP;                   // [kRGTok][EP]
+  uint64_t *full = reinterpret_cast<uint64_t *>(logits + kRGTok * EP);
+  uint64_t *empty = full + kRStages;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kRStages);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, c = lane & 3;
-  const long t0 = (long)blockIdx.x * kMmaTok;
-  const int nt = (int)min((long)kMmaTok, (long)T - t0);
-  const uint32_t row_bytes = (uint32_t)D * 2;
+  const int G = (T + kRGTok - 1) / kRGTok;
+  const int nch = (D + kRDC - 1) / kRDC;
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(bar, 1);
+    for (int s = 0; s < kRStages; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], kRWarps);
+    }
+    *abort_flag = 0;
     ptx::fence_mbar_init();
-    ptx::mbar_arrive_expect_tx(bar, row_bytes * nt);
-    for (int i = 0; i < nt; ++i) ptx::bulk_load(xs + (size_t)i * ld, x + (t0 + i) * D, row_bytes, bar);
   }
-  // rows past the last token read as zeros
-  for (int i = nt + warp; i < kMmaTok; i += kMmaWarps)
-    for (int j = lane * 8; j < D; j += 32 * 8) *reinterpret_cast<uint4 *>(xs + (size_t)i * ld + j) = make_uint4(0, 0, 0, 0);
+  // router rows E..EP-1 are never copied: zero them in every stage once
+  for (int i = threadIdx.x; i < kRStages * (EP - E) * (kRRowBytes / 16); i += blockDim.x) {
+    const int per = (EP - E) * (kRRowBytes / 16);
+    const int s = i / per, r = (i % per) / (kRRowBytes / 16), c = i % (kRRowBytes / 16);
+    *reinterpret_cast<uint4 *>(stages + s * STAGE + (kRGTok + E + r) * kRRowBytes + c * 16) = make_uint4(0, 0, 0, 0);
+  }
   __syncthreads();
-  bool ok = ptx::mbar_try_wait(bar, 0);
-  if (!ok) {
-    const uint64_t ts = ptx::globaltimer_ns();
-    while (!(ok = ptx::mbar_try_wait_sleep(bar, 0, ptx::kWaitHintNs)))
-      if (ptx::globaltimer_ns() - ts > kRouteWaitNs) break;
-  }
-  if (!__syncthreads_and(ok)) {
-    if (threadIdx.x == 0 && status) atomicExch(status, kDevTimeout);
-    return;
-  }
 
-  float acc[2][NT][4];
-#pragma unroll
-  for (int h = 0; h < 2; ++h)
-#pragma unroll
-    for (int n = 0; n < NT; ++n)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) acc[h][n][q] = 0.0f;
-  const __nv_bfloat16 *xr = xs + (size_t)g * ld + 2 * c;
-  // Steps are taken four at a time with every operand load of the four issued
-  // before their MMAs (the W_r fragments come from L1/L2, so their latency has
-  // to overlap); step j of the warp feeds accumulator set j & 1.
-  constexpr int kAhead = 4;
-  const int n_steps = (D / 16 - warp + kMmaWarps - 1) / kMmaWarps;  // this warp's 16-wide steps
-  int j0 = 0;
-  for (; j0 + kAhead <= n_steps; j0 += kAhead) {
-    uint32_t a[kAhead][4], b[kAhead][NT][2];
-#pragma unroll
-    for (int u = 0; u < kAhead; ++u) {
-      const int k0 = (warp + (j0 + u) * kMmaWarps) * 16;
-      a[u][0] = *reinterpret_cast<const uint32_t *>(xr + k0);
-      a[u][1] = 0u;  // rows 8..15
-      a[u][2] = *reinterpret_cast<const uint32_t *>(xr + k0 + 8);
-      a[u][3] = 0u;
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        const int e = n * 8 + g;
-        b[u][n][0] = b[u][n][1] = 0u;
-        if (e < E) {
-          const __nv_bfloat16 *wrow = wr + (long)e * D + k0 + 2 * c;
-          b[u][n][0] = __ldg(reinterpret_cast<const unsigned int *>(wrow));
-          b[u][n][1] = __ldg(reinterpret_cast<const unsigned int *>(wrow + 8));
+  if (warp == kRWarps) {
+    // ================================================= producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int g = blockIdx.x; g < G && ok; g += gridDim.x) {
+        for (int c = 0; c < nch; ++c, ++it) {
+          const int s = it % kRStages;
+          if (!route_wait(&empty[s], ((it / kRStages) & 1u) ^ 1u, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          const int d0 = c * kRDC, len = min(kRDC, D - d0);
+          const uint32_t bytes = (uint32_t)len * 2;
+          uint8_t *st = stages + s * STAGE;
+          ptx::mbar_arrive_expect_tx(&full[s], bytes * (uint32_t)(kRGTok + E));
+          for (int r = 0; r < kRGTok; ++r) {
+            const long t = min((long)g * kRGTok + r, (long)T - 1);
+            ptx::bulk_load(st + r * kRRowBytes, x + t * D + d0, bytes, &full[s]);
+          }
+          for (int e = 0; e < E; ++e) ptx::bulk_load(st + (kRGTok + e) * kRRowBytes, wr + (long)e * D + d0, bytes, &full[s]);
         }
       }
-    }
-#pragma unroll
-    for (int u = 0; u < kAhead; ++u)
-#pragma unroll
-      for (int n = 0; n < NT; ++n) mma_bf16_16816(acc[u & 1][n], a[u], b[u][n][0], b[u][n][1]);  // j0 even: set = u & 1
-  }
-  for (int j = j0; j < n_steps; ++j) {  // the remaining steps, one at a time
-    const int k0 = (warp + j * kMmaWarps) * 16;
-    uint32_t a[4];
-    a[0] = *reinterpret_cast<const uint32_t *>(xr + k0);
-    a[1] = 0u;
-    a[2] = *reinterpret_cast<const uint32_t *>(xr + k0 + 8);
-    a[3] = 0u;
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      const int e = n * 8 + g;
-      uint32_t b0 = 0u, b1 = 0u;
-      if (e < E) {
-        const __nv_bfloat16 *wrow = wr + (long)e * D + k0 + 2 * c;
-        b0 = __ldg(reinterpret_cast<const unsigned int *>(wrow));
-        b1 = __ldg(reinterpret_cast<const unsigned int *>(wrow + 8));
+      // every issued copy lands before the block's shared memory is released
+      const uint32_t n_drain = it < (uint32_t)kRStages ? it : (uint32_t)kRStages;
+      for (uint32_t j = it - n_drain; j < it; ++j) {
+        const uint64_t t0 = ptx::globaltimer_ns();
+        while (!ptx::mbar_try_wait(&full[j % kRStages], (j / kRStages) & 1u))
+          if (ptx::globaltimer_ns() - t0 > kRouteWaitNs / 10) break;
       }
-      if (j & 1) mma_bf16_16816(acc[1][n], a, b0, b1);
-      else mma_bf16_16816(acc[0][n], a, b0, b1);
+    }
+  } else {
+    // ================================================= consumers
+    float acc[2][NT][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[h][n][q] = 0.0f;
+    const int a_row = lane & 15, a_col = (lane >> 4) * 8;        // ldmatrix.x4 row addresses
+    const int b_row = lane & 7, b_col = ((lane >> 3) & 1) * 8;   // ldmatrix.x2 (lanes 0-15 used)
+    uint32_t it = 0;
+    for (int g = blockIdx.x; g < G; g += gridDim.x) {
+      for (int c = 0; c < nch; ++c, ++it) {
+        const int s = it % kRStages;
+        bool ok = true;
+        if (lane == 0) ok = route_wait(&full[s], (it / kRStages) & 1u, abort_flag, status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (ok) {
+          const uint8_t *st = stages + s * STAGE;
+          const int nk = min(kRDC, D - c * kRDC) / 16;
+          for (int j = warp; j < nk; j += kRWarps) {
+            uint32_t a[4];
+            ldmatrix_x4(a, st + a_row * kRRowBytes + (j * 16 + a_col) * 2);
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+              uint32_t b0, b1;
+              ldmatrix_x2(b0, b1, st + (kRGTok + n * 8 + b_row) * kRRowBytes + (j * 16 + b_col) * 2);
+              if ((j / kRWarps) & 1) mma_bf16_16816(acc[1][n], a, b0, b1);
+              else mma_bf16_16816(acc[0][n], a, b0, b1);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&empty[s]);  // release-ordered after this warp's reads
+      }
+      // C fragment: d0, d1 = row lane / 4, columns 2 (lane % 4) + 0, 1; d2, d3 = row lane / 4 + 8
+      const int r0 = lane >> 2, c0 = 2 * (lane & 3);
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          float *dst = part + ((warp * 2 + h) * kRGTok) * EP + n * 8 + c0;
+          dst[r0 * EP] = acc[h][n][0];
+          dst[r0 * EP + 1] = acc[h][n][1];
+          dst[(r0 + 8) * EP] = acc[h][n][2];
+          dst[(r0 + 8) * EP + 1] = acc[h][n][3];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[h][n][q] = 0.0f;
+        }
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * kRWarps) : "memory");
+      for (int idx = threadIdx.x; idx < kRGTok * E; idx += 32 * kRWarps) {
+        const int i = idx / E, e = idx - i * E;
+        float sum = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 2 * kRWarps; ++q) sum += part[(q * kRGTok + i) * EP + e];  // fixed order
+        logits[i * EP + e] = sum + ((gate == MOE_GATE_SOFTMAX_TOPK_RENORM && bias) ? bias[e] : 0.0f);
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * kRWarps) : "memory");
+      if (!*abort_flag)
+        for (int i = warp; i < kRGTok; i += kRWarps) {
+          const long t = (long)g * kRGTok + i;
+          if (t < T) select_topk(logits + i * EP, t, E, k, gate, bias, bias_vl, image_mask, topk_idx, topk_w, lane);
+        }
     }
   }
-  // C fragment: d0, d1 = token g, experts n*8 + 2c, 2c + 1 (d2, d3: rows 8..15, unused)
-#pragma unroll
-  for (int h = 0; h < 2; ++h)
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      float *dst = part + ((warp * 2 + h) * kMmaTok + g) * 32 + n * 8 + 2 * c;
-      dst[0] = acc[h][n][0];
-      dst[1] = acc[h][n][1];
-    }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < kMmaTok * E; idx += blockDim.x) {
-    const int i = idx / E, e = idx - i * E;
-    float sum = 0.0f;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) sum += part[(q * kMmaTok + i) * 32 + e];  // fixed order
-    logits[i * E + e] = sum + ((gate == MOE_GATE_SOFTMAX_TOPK_RENORM && bias) ? bias[e] : 0.0f);
-  }
-  __syncthreads();
-  for (int i = warp; i < nt; i += kMmaWarps)
-    select_topk(logits + i * E, t0 + i, E, k, gate, bias, bias_vl, image_mask, topk_idx, topk_w, lane);
 }
 
 }  // namespace
@@ -317,18 +371,25 @@ moe_status launch_route(const MoEConfig &c, int T, const void *x, const void *w_
     return launch_route_tc(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, status, scratch, s);
   if (c.act_dtype == MOE_F32)
     return launch_route_t<float>(c, T, x, w_router, bias, bias_vl, image_mask, topk_idx, topk_w, status, s);
-  if (c.num_experts <= 32 && c.hidden_dim % 16 == 0 && (size_t)kMmaTok * (c.hidden_dim + 8) * 2 <= 160 * 1024) {
-    const int E = c.num_experts;
-    const size_t smem = (size_t)kMmaTok * (c.hidden_dim + 8) * 2 + (8 * kMmaTok * 32 + (size_t)kMmaTok * E) * 4 + 32;
-    auto kern = route_mma_kernel<4>;
-    switch ((E + 7) / 8) {
-      case 1: kern = route_mma_kernel<1>; break;
-      case 2: kern = route_mma_kernel<2>; break;
-      case 3: kern = route_mma_kernel<3>; break;
+  if (c.num_experts <= 32 && c.hidden_dim % 16 == 0) {
+    const int E = c.num_experts, NT = (E + 7) / 8;
+    auto kern = route_ring_kernel<4>;
+    size_t smem = route_ring_smem<4>();
+    switch (NT) {
+      case 1: kern = route_ring_kernel<1>; smem = route_ring_smem<1>(); break;
+      case 2: kern = route_ring_kernel<2>; smem = route_ring_smem<2>(); break;
+      case 3: kern = route_ring_kernel<3>; smem = route_ring_smem<3>(); break;
       default: break;
     }
     MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    kern<<<(unsigned)((T + kMmaTok - 1) / kMmaTok), 32 * kMmaWarps, smem, s>>>(
+    int dev = 0, sms = 148, per_sm = 1;
+    MOE_CUDA_TRY(cudaGetDevice(&dev));
+    MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    MOE_CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32 * (kRWarps + 1), smem));
+    if (per_sm < 1) per_sm = 1;
+    const long groups = (T + kRGTok - 1) / kRGTok;
+    const long cap = (long)sms * per_sm;
+    kern<<<(unsigned)(groups < cap ? groups : cap), 32 * (kRWarps + 1), smem, s>>>(
         T, c.hidden_dim, E, c.top_k, c.gate, (const __nv_bfloat16 *)x, (const __nv_bfloat16 *)w_router, bias,
         bias_vl, image_mask, topk_idx, topk_w, status);
     MOE_LAUNCH_CHECK();

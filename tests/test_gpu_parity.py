@@ -225,7 +225,9 @@ def test_full_size_sampled(B, W, name, n_sample):
                                            (33, 16, "sqrt_softplus", "uniform"), (48, 4, "softmax", "none"),
                                            (64, 2, "softmax", "zipf"), (128, 16, "softmax", "none"),
                                            (300, 6, "sqrt_softplus", "uniform"), (512, 8, "softmax", "none"),
-                                           (8, 2, "sigmoid", "uniform"), (96, 6, "sigmoid", "uniform")])
+                                           (8, 2, "sigmoid", "uniform"), (96, 6, "sigmoid", "uniform"),
+                                           (16, 4, "softmax", "zipf"), (24, 3, "sqrt_softplus", "uniform"),
+                                           (32, 8, "softmax", "none")])
 def test_route_many_experts(B, W, E, k, gate, bias):
     # the router on both paths (CUDA cores up to 32 experts, tensor cores
     # above): ragged 128-token tiles, padded expert columns, one or two MMA
@@ -241,6 +243,23 @@ def test_route_many_experts(B, W, E, k, gate, bias):
     logits, idx_o, w_o, keys = H.oracle_route(p, L, a)
     rc = H.check_route(p, H.to_np(idx), H.to_np(w), logits, idx_o, keys, a.get("bias"))
     print(f"route E={E} k={k} {gate}: {H.route_report(rc)}")
+
+
+@pytest.mark.parametrize("T,D,E,k", [(77, 1040, 8, 2), (45, 2064, 32, 4), (16, 16, 8, 1), (1, 528, 24, 6)])
+def test_route_ring_slices(B, W, T, D, E, k):
+    # the streamed router for up to 32 experts: hidden sizes that end in a
+    # short slice (the ring moves 512 columns at a time), a single 16-wide
+    # step, token counts below and across one 16-token group
+    p = synth.MoEProblem("route", T=T, D=D, F=128, E=E, k=k, gate="softmax", bias="zipf", seed=23)
+    a = synth.generate(p, experts=False)
+    cfg = W.config_of(p)
+    wt = {n: W.to_torch(a.get(n)) for n in ("w_router", "bias", "bias_vl")}
+    idx, w = B.route_topk(cfg, W.to_torch(a["x"]), B.make_weights(wt), W.to_torch(a.get("image_mask")))
+    torch.cuda.synchronize()
+    L = H.oracle_layer(p, a)
+    logits, idx_o, w_o, keys = H.oracle_route(p, L, a)
+    rc = H.check_route(p, H.to_np(idx), H.to_np(w), logits, idx_o, keys, a.get("bias"))
+    print(f"route T={T} D={D} E={E} k={k}: {H.route_report(rc)}")
 
 
 # ---------------------------------------------------------------- edge cases
