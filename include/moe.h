@@ -177,10 +177,11 @@ size_t moe_route_workspace_size(const MoEConfig *cfg, int T);
  *              sqrt(softplus(s)), or raw sigmoid(s))
  *   ws         >= moe_route_workspace_size(cfg, T) bytes (status word)
  * Logits are accumulated in fp32 (ops-transformer walkthrough, 坑三).  With
- * E <= 32 (or fp32 activations) one kernel computes them on the CUDA cores
- * and selects from shared memory.  With bf16 activations and 32 < E <= 512
- * they are computed on the tensor cores and each token's logit row is stored
- * to the route workspace, from which a second kernel selects. */
+ * E <= 32 one kernel computes them (bf16: warp-level tensor-core MMAs on
+ * 16-token groups; fp32 activations: CUDA-core FMA) and selects from shared
+ * memory.  With bf16 activations and 32 < E <= 512 they are computed on the
+ * 5th-generation tensor cores and each token's logit row is stored to the
+ * route workspace, from which a second kernel selects. */
 moe_status moe_route_topk(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
                           const uint8_t *image_mask, int32_t *topk_idx, float *topk_w, void *ws,
                           size_t ws_bytes, moe_stream_t stream);
