@@ -126,22 +126,24 @@ struct Params {
   const float *row_scale;    // F16: 2^-s_r of each A row
 };
 
-// The waits of this kernel spin instead of suspending: its k-block period is
-// a chain of hand-offs (converters -> MMA -> completion -> converters), and a
-// suspended waiter wakes late enough to lengthen every link (measured: 5%).
-// The clock is read every 64 polls.
+// Bounded wait.  The hand-offs on the k-block path (the MMA thread's A and B
+// waits, the converters' weight and B-stage waits) spin: that path is a chain
+// of hand-offs and a suspended waiter wakes late (measured: 5%).  Every other
+// waiter (producers on a full ring, the epilogue for a whole tile) sleeps on
+// the barrier with a suspend-time hint, so that it takes no issue slots from
+// the converter warps.  The clock is read every 64 polls.
+template <bool SPIN>
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Smem &sm, int *status) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t n = 1;; ++n) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    if ((n & 63u) == 0) {
-      if (*(volatile int *)&sm.abort) return false;
-      if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
-        *(volatile int *)&sm.abort = 1;
-        atomicExch(status, kDevTimeout);
-        return false;
-      }
+    if (SPIN ? ptx::mbar_try_wait(bar, parity) : ptx::mbar_try_wait_sleep(bar, parity, ptx::kWaitHintNs)) return true;
+    if (SPIN && (n & 63u) != 0) continue;
+    if (*(volatile int *)&sm.abort) return false;
+    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+      *(volatile int *)&sm.abort = 1;
+      atomicExch(status, kDevTimeout);
+      return false;
     }
   }
 }
@@ -158,9 +160,10 @@ __device__ __forceinline__ void drain_bar(uint64_t *bar, uint32_t parity, int *s
 }
 
 // Warp-uniform wait: lane 0 polls, the outcome is broadcast to the warp.
+template <bool SPIN>
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, Smem &sm, int *status, int lane) {
   bool ok = true;
-  if (lane == 0) ok = wait_bar(bar, parity, sm, status);
+  if (lane == 0) ok = wait_bar<SPIN>(bar, parity, sm, status);
   return __shfl_sync(0xffffffffu, ok, 0);
 }
 
@@ -375,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = it % A_STAGES;
           const uint32_t ph = (it / A_STAGES) & 1u;
           bool got = true;
-          if (lane == 0) got = wait_bar(&sm.a_empty[s], ph ^ 1u, sm, p.status);
+          if (lane == 0) got = wait_bar<false>(&sm.a_empty[s], ph ^ 1u, sm, p.status);
           if (gather) got = __shfl_sync(0xffffffffu, got, 0);
           if (!got) {
             ok = false;
@@ -420,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kw = 0; kw < k_blocks / KW; ++kw, ++it) {
           const int s = it % W_STAGES;
           const uint32_t ph = (it / W_STAGES) & 1u;
-          if (!wait_bar(&sm.w_empty[s], ph ^ 1u, sm, p.status)) {
+          if (!wait_bar<false>(&sm.w_empty[s], ph ^ 1u, sm, p.status)) {
             ok = false;
             break;
           }
@@ -447,13 +450,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++i) {
         const int acc = i & 1;
-        if (!wait_bar(&sm.tmem_empty[acc], ((i >> 1) & 1u) ^ 1u, sm, p.status)) break;
+        if (!wait_bar<false>(&sm.tmem_empty[acc], ((i >> 1) & 1u) ^ 1u, sm, p.status)) break;
         ptx::tc_fence_after();
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
           const int s = it % A_STAGES;
           const int sb = it % B_STAGES;
-          if (!wait_bar(&sm.a_full[s], (it / A_STAGES) & 1u, sm, p.status) ||
-              !wait_bar(&sm.b_full[sb], (it / B_STAGES) & 1u, sm, p.status)) {
+          if (!wait_bar<true>(&sm.a_full[s], (it / A_STAGES) & 1u, sm, p.status) ||
+              !wait_bar<true>(&sm.b_full[sb], (it / B_STAGES) & 1u, sm, p.status)) {
             ok = false;
             break;
           }
@@ -484,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++i) {
       const Tile tl = decode_tile(p, sm, t);
       const int acc = i & 1;
-      if (!warp_wait(&sm.tmem_full[acc], (i >> 1) & 1u, sm, p.status, lane)) break;
+      if (!warp_wait<false>(&sm.tmem_full[acc], (i >> 1) & 1u, sm, p.status, lane)) break;
       ptx::tc_fence_after();
       const int row = tl.m0 + q * 32 + lane;
       const bool live = row < tl.end;
@@ -570,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sw = iw % W_STAGES;
         const int sb = it % B_STAGES;
         const int kq = kb & (KW - 1);
-        if (kq == 0 && !warp_wait(&sm.w_full[sw], (iw / W_STAGES) & 1u, sm, p.status, lane)) {
+        if (kq == 0 && !warp_wait<true>(&sm.w_full[sw], (iw / W_STAGES) & 1u, sm, p.status, lane)) {
           ok = false;
           break;
         }
@@ -589,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int j = 0; j < JOBS; ++j) sc[j] = F16 ? scale_f16x2(sc[j]) : lut[sc[j]];
-        if (!warp_wait(&sm.b_empty[sb], ((it / B_STAGES) & 1u) ^ 1u, sm, p.status, lane)) {
+        if (!warp_wait<true>(&sm.b_empty[sb], ((it / B_STAGES) & 1u) ^ 1u, sm, p.status, lane)) {
           ok = false;
           break;
         }
