@@ -108,12 +108,19 @@ __device__ __forceinline__ void raise_abort(Smem &sm, uint32_t rank) {
 }
 
 // Bounded wait; false if the CTA is aborting (this thread may have started it).
-template <bool PAIR>
+// The stage ring's hand-offs (the producer waiting for a free stage, the MMA
+// thread for a full one) spin: a stage's round trip (copy, MMA, completion,
+// refill) is what bounds the k-block rate, and a suspended waiter woke ~350
+// cycles late in every round trip (clock64 timeline of one CTA).  The
+// epilogue, which waits a whole tile, sleeps on the barrier with a
+// suspend-time hint.  The clock is read every 64 polls when spinning.
+template <bool PAIR, bool SPIN = false>
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Smem &sm, int *status, uint32_t rank) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
-  while (true) {
-    if (ptx::mbar_try_wait_sleep(bar, parity, ptx::kWaitHintNs)) return true;
+  for (uint32_t n = 1;; ++n) {
+    if (SPIN ? ptx::mbar_try_wait(bar, parity) : ptx::mbar_try_wait_sleep(bar, parity, ptx::kWaitHintNs)) return true;
+    if (SPIN && (n & 63u) != 0) continue;
     if (*(volatile int *)&sm.abort) return false;
     if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
       raise_abort<PAIR>(sm, rank);
@@ -284,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1u;
           bool got = true;
-          if (lane == 0) got = wait_bar<PAIR>(&sm.empty[s], ph ^ 1u, sm, p.status, rank);
+          if (lane == 0) got = wait_bar<PAIR, true>(&sm.empty[s], ph ^ 1u, sm, p.status, rank);
           if (gather) {
             got = __shfl_sync(0xffffffffu, got, 0);
             __syncwarp();
@@ -353,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
           const int s = it % C::STAGES;
           const uint32_t ph = (it / C::STAGES) & 1u;
-          if (!wait_bar<PAIR>(&sm.full[s], ph, sm, p.status, rank)) { ok = false; break; }
+          if (!wait_bar<PAIR, true>(&sm.full[s], ph, sm, p.status, rank)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t a_addr = ptx::smem_addr(stage_a + s * A_BYTES);
           const uint32_t b_addr = ptx::smem_addr(stage_b + s * C::B_BYTES);
