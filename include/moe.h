@@ -300,11 +300,17 @@ size_t moe_workspace_size(const MoEConfig *cfg, int T);
  * kept count of expert e is min(expert_counts_out[e], C) (all of it when
  * C = 0) and the layer drops T*k minus their sum.
  * Same kernels and results as the stage entry points called in order, with
- * one difference in operand format: for NVFP4 experts whose gate/up reduction
- * length D is a multiple of 256, the gate/up GEMM multiplies f16 operands
- * (x rows scaled by a power of two each, expanded FP4 weights) instead of
- * bf16 ones.  Both are exact, so the results are identical whenever every
- * element of a token row satisfies |x| >= max|row| * 2^-31 or x = 0. */
+ * two differences in operand format for NVFP4 experts whose gate/up reduction
+ * length D is a multiple of 256:
+ *   - the gate/up GEMM multiplies f16 operands (x rows scaled by a power of
+ *     two each, expanded FP4 weights) instead of bf16 ones.  Both are exact,
+ *     so g and u are identical whenever every element of a token row
+ *     satisfies |x| >= max|row| * 2^-31 or x = 0;
+ *   - when the down reduction length F is a multiple of 256 too and the
+ *     SwiGLU clamp L is in (0, 255] (so |h| <= L^2 < 65504), h is stored in
+ *     f16 rather than bf16 and the down GEMM multiplies in f16.  f16 rounds h
+ *     more finely, so the output differs from the staged bf16-h result by
+ *     less than bf16's rounding of h. */
 moe_status moe_forward(const MoEConfig *cfg, int T, const void *x, const MoEWeights *w,
                        const uint8_t *image_mask, void *out, int32_t *topk_idx_out,
                        int32_t *expert_counts_out, void *ws, size_t ws_bytes, moe_stream_t stream);

@@ -469,17 +469,22 @@ static moe_status forward_impl(const MoEConfig *cfg, int T, const void *x, const
   else st = launch_gather(c, T, f.offsets, f.row_token, x, f.x_perm, s);
   if (st != MOE_OK) return st;
   if ((st = mark(3)) != MOE_OK) return st;
+  // with the SwiGLU clamp bounding |h| below 65504, h is kept in f16 and the
+  // NVFP4 down projection multiplies in f16 too
+  const bool h_f16 = fp4_f16 && down_direct(c) && h_fits_f16(c);
   if (fp4_f16) {
     st = launch_gate_up_fp4(c, rows, f.x_perm, rows, nullptr, f.offsets, w->w_gate, w->w_up, w->s_gate, w->s_up,
-                            f.row_scale, f.h, f.ex.status, s);
+                            f.row_scale, f.h, f.ex.status, s, h_f16);
   } else {
     st = run_gate_up(c, rows, f.x_perm, rows, nullptr, f.offsets, w->w_gate, w->w_up, w->s_gate, w->s_up, f.h,
                      f.ex, s);
   }
   if (st != MOE_OK) return st;
   if ((st = mark(4)) != MOE_OK) return st;
-  if ((st = run_down(c, rows, f.h, f.offsets, w->w_down, w->s_down, f.row_weight, f.y_perm, f.ex, s)) != MOE_OK)
-    return st;
+  if (h_f16) st = launch_down_fp4(c, rows, f.h, f.offsets, w->w_down, w->s_down, f.row_weight, (float *)f.y_perm,
+                                  f.ex.status, s, true);
+  else st = run_down(c, rows, f.h, f.offsets, w->w_down, w->s_down, f.row_weight, f.y_perm, f.ex, s);
+  if (st != MOE_OK) return st;
   if ((st = mark(5)) != MOE_OK) return st;
   if (c.shared_intermediate_dim) {
     const MoEConfig sc = shared_cfg(c);

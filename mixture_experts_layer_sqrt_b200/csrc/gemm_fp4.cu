@@ -50,12 +50,15 @@
 //   warps 7-14   converters: codes + scales -> swizzled 16-bit B tile, one
 //                arrival per warp.
 //
-// F16 (gate/up inside moe_forward): A arrives as f16 rows pre-scaled by a
-// power of two per row (launch_gather_f16), the codes are expanded to f16
+// F16 (inside moe_forward): for gate/up, A arrives as f16 rows pre-scaled by
+// a power of two per row (launch_gather_f16), the codes are expanded to f16
 // (e2m1 -> f16 needs no re-bias, so one conversion and one f16 multiply per
 // pair of weights), the MMAs run f16 x f16 -> fp32, and the epilogue undoes
-// the row scale.  All three steps are exact, so the result equals the bf16
-// path's bit for bit whenever the scaled activations are exact in f16.
+// the row scale.  All three steps are exact, so g and u equal the bf16
+// path's bit for bit whenever the scaled activations are exact in f16.  When
+// the SwiGLU clamp bounds |h| below f16's range the epilogue stores h in f16
+// (10 fraction bits instead of bf16's 7) and the down projection runs in f16
+// as well, without the bf16 re-bias and scale table.
 //
 // Tiles never straddle two experts; the tile list (expert-major, n-block,
 // m-block) comes from expert_offsets on the device.  Every wait is bounded
@@ -123,7 +126,8 @@ struct Params {
   int clamp_mode;
   int *status;
   uint32_t hi_mul;           // 2^29, passed at run time so the multiply-add stays one
-  const float *row_scale;    // F16: 2^-s_r of each A row
+  const float *row_scale;    // F16 gate/up: 2^-s_r of each A row
+  int h_f16;                 // F16 gate/up: store h in f16 (else bf16)
 };
 
 // Bounded wait.  The hand-offs on the k-block path (the MMA thread's A and B
@@ -516,8 +520,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const float h0 = swiglu_h(g0, u0, p.clamp, p.clamp_mode);
                 const float h1 = swiglu_h(g1, u1, p.clamp, p.clamp_mode);
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(h0, h1);
-                pk[j] = *reinterpret_cast<uint32_t *>(&b2);
+                if (F16 && p.h_f16) {
+                  __half2 f2 = __floats2half2_rn(h0, h1);
+                  pk[j] = *reinterpret_cast<uint32_t *>(&f2);
+                } else {
+                  __nv_bfloat162 b2 = __floats2bfloat162_rn(h0, h1);
+                  pk[j] = *reinterpret_cast<uint32_t *>(&b2);
+                }
               }
               uint4 *dst = reinterpret_cast<uint4 *>(hrow + c);
 #pragma unroll
@@ -668,7 +677,8 @@ bool fp4_direct_ok(const MoEConfig &c, int K) {
 
 moe_status launch_gate_up_fp4(const MoEConfig &c, int rows, const void *a, int a_rows, const int32_t *row_token,
                               const int32_t *offsets, const void *w_gate, const void *w_up, const void *s_gate,
-                              const void *s_up, const float *row_scale, void *h, int *status, cudaStream_t s) {
+                              const void *s_up, const float *row_scale, void *h, int *status, cudaStream_t s,
+                              bool h_f16) {
   if (rows == 0) return MOE_OK;
   Params p;
   p.rows = rows;
@@ -686,13 +696,14 @@ moe_status launch_gate_up_fp4(const MoEConfig &c, int rows, const void *a, int a
   p.status = status;
   p.hi_mul = 1u << 29;
   p.row_scale = row_scale;
+  p.h_f16 = row_scale && h_f16 ? 1 : 0;
   if (row_scale) return launch_fp4<true, true>(p, a, w_gate, w_up, s_gate, s_up, c.intermediate_dim, s);
   return launch_fp4<true, false>(p, a, w_gate, w_up, s_gate, s_up, c.intermediate_dim, s);
 }
 
 moe_status launch_down_fp4(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
                            const void *w_down, const void *s_down, const float *row_weight, float *y,
-                           int *status, cudaStream_t s) {
+                           int *status, cudaStream_t s, bool h_f16) {
   if (rows == 0) return MOE_OK;
   Params p;
   p.rows = rows;
@@ -710,6 +721,8 @@ moe_status launch_down_fp4(const MoEConfig &c, int rows, const void *h, const in
   p.status = status;
   p.hi_mul = 1u << 29;
   p.row_scale = nullptr;
+  p.h_f16 = 0;
+  if (h_f16) return launch_fp4<false, true>(p, h, w_down, nullptr, s_down, nullptr, c.hidden_dim, s);
   return launch_fp4<false, false>(p, h, w_down, nullptr, s_down, nullptr, c.hidden_dim, s);
 }
 

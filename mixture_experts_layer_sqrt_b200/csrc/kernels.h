@@ -76,12 +76,19 @@ moe_status launch_down_tc(const MoEConfig &c, int rows, const void *h, const int
 bool fp4_direct_ok(const MoEConfig &c, int K);
 // row_scale non-null: `a` holds f16 rows scaled by 2^s_r (launch_gather_f16)
 // and the MMAs run in f16; the epilogue multiplies g and u by row_scale[r].
+// h_f16 (only with row_scale): h is stored in f16 instead of bf16.
 moe_status launch_gate_up_fp4(const MoEConfig &c, int rows, const void *a, int a_rows, const int32_t *row_token,
                               const int32_t *offsets, const void *w_gate, const void *w_up, const void *s_gate,
-                              const void *s_up, const float *row_scale, void *h, int *status, cudaStream_t s);
+                              const void *s_up, const float *row_scale, void *h, int *status, cudaStream_t s,
+                              bool h_f16 = false);
+// h_f16: h is f16 (from launch_gate_up_fp4 with h_f16) and the MMAs run in f16.
 moe_status launch_down_fp4(const MoEConfig &c, int rows, const void *h, const int32_t *offsets,
                            const void *w_down, const void *s_down, const float *row_weight, float *y,
-                           int *status, cudaStream_t s);
+                           int *status, cudaStream_t s, bool h_f16 = false);
+// The SwiGLU clamp bounds |h| within f16's range: |SiLU(g) u| <= L^2 with
+// both pre-activations clipped, |h| <= L with h clipped; L <= 255 keeps
+// either below 65504.
+inline bool h_fits_f16(const MoEConfig &c) { return c.swiglu_clamp > 0.0f && c.swiglu_clamp <= 255.0f; }
 
 // One block whose bounded wait never completes: records the timeout status.
 moe_status launch_wait_selftest(int *status, cudaStream_t s);

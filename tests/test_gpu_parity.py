@@ -435,6 +435,37 @@ def test_fp4_forward_f16_rows_exact(B, W):
     assert torch.equal(out_f, g["out"])
 
 
+@pytest.mark.parametrize("clamp,x_scale", [(10.0, 1.0), (10.0, 20.0), (300.0, 1.0)])
+def test_fp4_forward_h_f16(B, W, clamp, x_scale):
+    # inside moe_forward an NVFP4 layer whose SwiGLU clamp bounds |h| below
+    # f16's range (L <= 255) keeps h in f16 and runs the down projection in
+    # f16: the layer meets the oracle, and differs from the staged bf16-h path
+    # by no more than bf16's rounding of h; with L > 255 h stays bf16 and the
+    # layer equals the staged path bit for bit
+    p = synth.PROBLEMS["sqrt_fp4"].with_(name="fp4_hf16", T=333, D=512, F=512, E=8, k=2, Fs=128, clamp=clamp)
+    a = synth.generate(p)
+    if x_scale != 1.0:
+        a["x"] = synth.f32_to_bf16_bits((O.decode_act(a["x"], p.act) * x_scale).astype(np.float32))
+    c = Case(B, W, p, a)
+    g = _stages(B, c)
+    ws = B.workspace(B.workspace_size(c.cfg, p.T))
+    out_f = B.forward(c.cfg, c.x, c.w, ws, c.mask)
+    torch.cuda.synchronize()
+    B.check_device_status(ws)
+    idx_g = H.to_np(g["idx"]).astype(np.int64)
+    logits, idx_o, w_o, keys = H.oracle_route(p, c.L, a)
+    w_sel = O.route_weights(logits, idx_g, p.gate)
+    o = O.moe_forward(c.L.x(), logits, idx_g, w_sel, c.L.expert, p.E, 0, p.clamp, "preact", c.L.shared())
+    rel = H.assert_close_layer(p, H.to_np(out_f), o["out"], "forward")
+    if clamp > 255.0:
+        assert torch.equal(out_f, g["out"])
+    else:
+        rms = float(np.sqrt(np.mean(o["out"] ** 2)))
+        diff = float((out_f - g["out"]).abs().max())
+        assert diff <= 2.0 ** -6 * rms, (diff, rms)
+        print(f"clamp {clamp}, x*{x_scale}: forward vs oracle {rel:.3g} rms, vs staged bf16-h path {diff / rms:.3g} rms")
+
+
 def test_bounded_wait_times_out_and_context_survives(B, W):
     # a wait that nothing satisfies gives up after its limit, records the
     # timeout in the status word and returns; the GPU keeps working
