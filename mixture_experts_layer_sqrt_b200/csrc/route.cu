@@ -145,9 +145,9 @@ __global__ void __launch_bounds__(512) route_kernel(int T, int D, int E, int k, 
 // bf16 activations, E <= 32: the logits on the tensor cores with the
 // warp-level mma.sync (m16n8k16, bf16 in, fp32 accumulate), so the kernel is
 // left with streaming x at HBM speed.  A block takes groups of 16 tokens (the
-// MMA's 16 rows); one producer thread streams, per 512-wide slice of D, the
+// MMA's 16 rows); a producer warp streams, per 512-wide slice of D, the
 // group's 16 x rows and the E router rows into a ring of 4 stages (3 for
-// E > 16) with bulk copies, rows padded by 16 bytes so that ldmatrix reads
+// E > 16) with one bulk copy per row issued by its own lane, rows padded by 16 bytes so that ldmatrix reads
 // hit 8 different bank groups.  8 consumer warps each take every eighth
 // 16-wide step of a slice into two accumulator sets (alternate steps).  A
 // stage is released as soon as its reads are done, so the copies of the next
@@ -245,28 +245,35 @@ __global__ void __launch_bounds__(32 * (kRWarps + 1), 1) route_ring_kernel(int T
 
   if (warp == kRWarps) {
     // ================================================= producer
-    if (lane == 0) {
-      uint32_t it = 0;
-      bool ok = true;
-      for (int g = blockIdx.x; g < G && ok; g += gridDim.x) {
-        for (int c = 0; c < nch; ++c, ++it) {
-          const int s = it % kRStages;
-          if (!route_wait(&empty[s], ((it / kRStages) & 1u) ^ 1u, abort_flag, status)) {
-            ok = false;
-            break;
-          }
-          const int d0 = c * kRDC, len = min(kRDC, D - d0);
-          const uint32_t bytes = (uint32_t)len * 2;
-          uint8_t *st = stages + s * STAGE;
-          ptx::mbar_arrive_expect_tx(&full[s], bytes * (uint32_t)(kRGTok + E));
-          for (int r = 0; r < kRGTok; ++r) {
-            const long t = min((long)g * kRGTok + r, (long)T - 1);
-            ptx::bulk_load(st + r * kRRowBytes, x + t * D + d0, bytes, &full[s]);
-          }
-          for (int e = 0; e < E; ++e) ptx::bulk_load(st + (kRGTok + e) * kRRowBytes, wr + (long)e * D + d0, bytes, &full[s]);
+    // lane 0 waits for a free stage and expects its bytes; the warp's lanes
+    // then issue the row copies side by side (lane i: x row i, lanes 16..:
+    // router rows), so no single thread serialises 16 + E copy issues.
+    uint32_t it = 0;
+    bool ok = true;
+    for (int g = blockIdx.x; g < G && ok; g += gridDim.x) {
+      for (int c = 0; c < nch; ++c, ++it) {
+        const int s = it % kRStages;
+        bool got = true;
+        if (lane == 0) got = route_wait(&empty[s], ((it / kRStages) & 1u) ^ 1u, abort_flag, status);
+        if (!__shfl_sync(0xffffffffu, got, 0)) {
+          ok = false;
+          break;
+        }
+        const int d0 = c * kRDC, len = min(kRDC, D - d0);
+        const uint32_t bytes = (uint32_t)len * 2;
+        uint8_t *st = stages + s * STAGE;
+        if (lane == 0) ptx::mbar_arrive_expect_tx(&full[s], bytes * (uint32_t)(kRGTok + E));
+        __syncwarp();
+        for (int r = lane; r < kRGTok + E; r += 32) {
+          const __nv_bfloat16 *src;
+          if (r < kRGTok) src = x + min((long)g * kRGTok + r, (long)T - 1) * D + d0;
+          else src = wr + (long)(r - kRGTok) * D + d0;
+          ptx::bulk_load(st + r * kRRowBytes, src, bytes, &full[s]);
         }
       }
-      // every issued copy lands before the block's shared memory is released
+    }
+    // every issued copy lands before the block's shared memory is released
+    if (lane == 0) {
       const uint32_t n_drain = it < (uint32_t)kRStages ? it : (uint32_t)kRStages;
       for (uint32_t j = it - n_drain; j < it; ++j) {
         const uint64_t t0 = ptx::globaltimer_ns();
