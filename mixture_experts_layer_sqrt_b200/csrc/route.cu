@@ -182,7 +182,7 @@ __device__ __forceinline__ void ldmatrix_x2(uint32_t &r0, uint32_t &r1, const vo
 // Bounded wait; gives up at once when the block is aborting.  Waiters sleep
 // on the barrier (a suspend-time hint) instead of spinning: measured the same
 // (23-25 us for the Mixtral-shaped router either way) with fewer issue slots
-// taken from the producer thread.
+// taken from the producer.
 __device__ __forceinline__ bool route_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
