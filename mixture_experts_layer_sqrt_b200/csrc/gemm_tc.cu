@@ -28,7 +28,9 @@
 //               back to the producers; two 256-column fp32 accumulators let
 //               the epilogue of tile i overlap the MMAs of tile i+1.
 //   warps 2-5   epilogue: tcgen05.ld (one TMEM lane = one output row per
-//               thread), fused SwiGLU or routing weight, global store.
+//               thread), fused SwiGLU or routing weight, global store (the
+//               fp32 y through a 4 KB shared-memory stage per warp, so that
+//               the stores are whole 128-byte row segments).
 //
 // Tiles never straddle two experts: expert e owns ceil(rows_e / tile_rows)
 // m-blocks; the tile list (expert-major, then n-block, then m-block, so the
@@ -63,6 +65,7 @@ constexpr int MAX_E = 1024;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s
 constexpr int kThreads = 192;
+constexpr int kStagingOffset = 5120;  // past Smem, 1024-aligned; 4 warps x 4 KB
 
 template <bool PAIR>
 struct Cfg {
@@ -84,6 +87,8 @@ struct Smem {
   int abort;
   int tile_start[MAX_E + 1];
 };
+
+static_assert(sizeof(Smem) <= kStagingOffset, "the epilogue staging follows the barriers and tile list");
 
 struct Params {
   int rows;                  // rows of the output (and of A unless gathered)
@@ -188,6 +193,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *stage_a = base;
   uint8_t *stage_b = base + C::STAGES * A_BYTES;
   Smem &sm = *reinterpret_cast<Smem *>(base + C::STAGES * C::STAGE_BYTES);
+  // fp32 epilogue staging: 32 rows x 32 columns per epilogue warp
+  float *staging = reinterpret_cast<float *>(base + C::STAGES * C::STAGE_BYTES + kStagingOffset);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
@@ -426,21 +433,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
+        // Each 32 x 32 fp32 chunk goes through this warp's 4 KB of shared
+        // memory: lane r writes its row (16-byte piece j at j ^ (r % 8), four
+        // wavefronts per 512 bytes), then every store instruction writes four
+        // whole 128-byte row segments instead of 32 rows' 16-byte pieces.
         const int ncol0 = tl.n_blk * BN;
         const float rw = (live && p.row_weight) ? p.row_weight[row] : 1.0f;
-        float *yrow = (float *)p.out + (long)row * p.N + ncol0;
+        float *stg = staging + q * 32 * 32;
+        const int row0 = tl.m0 + (int)rank * BM + q * 32;  // this warp's first row
+        const int rr = lane >> 3, ff = lane & 7;            // read-back: row 4 i + rr, piece ff
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t v[32];
           ptx::tmem_ld32(tbase + c, v);
           ptx::tmem_ld_wait();
-          if (live) {
-            float4 *dst = reinterpret_cast<float4 *>(yrow + c);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              dst[j] = make_float4(__uint_as_float(v[4 * j]) * rw, __uint_as_float(v[4 * j + 1]) * rw,
-                                   __uint_as_float(v[4 * j + 2]) * rw, __uint_as_float(v[4 * j + 3]) * rw);
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4 *>(stg + lane * 32 + ((j ^ (lane & 7)) << 2)) =
+                make_float4(__uint_as_float(v[4 * j]) * rw, __uint_as_float(v[4 * j + 1]) * rw,
+                            __uint_as_float(v[4 * j + 2]) * rw, __uint_as_float(v[4 * j + 3]) * rw);
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + rr;
+            const float4 val = *reinterpret_cast<const float4 *>(stg + r * 32 + ((ff ^ (r & 7)) << 2));
+            if (row0 + r < tl.end)
+              *reinterpret_cast<float4 *>((float *)p.out + (long)(row0 + r) * p.N + ncol0 + c + ff * 4) = val;
           }
+          __syncwarp();
         }
       }
       ptx::tc_fence_before();
@@ -469,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------ host
 template <bool GATED, bool PAIR>
 size_t smem_bytes() {
-  return 1024 + (size_t)Cfg<PAIR>::STAGES * Cfg<PAIR>::STAGE_BYTES + sizeof(Smem);
+  return 1024 + (size_t)Cfg<PAIR>::STAGES * Cfg<PAIR>::STAGE_BYTES + kStagingOffset + 4 * 32 * 32 * sizeof(float);
 }
 
 template <bool GATED, bool PAIR>
