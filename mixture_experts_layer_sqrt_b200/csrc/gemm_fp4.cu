@@ -83,15 +83,25 @@ constexpr int TILE_M = 128;                     // rows per tile (TMEM lanes)
 constexpr int FN = 256;                         // MMA N: B rows per k-block
 constexpr int A_BYTES = TILE_M * BK * 2;        // 16 KB
 constexpr int B_BYTES = FN * BK * 2;            // 32 KB
-constexpr int KW = 4;                           // k-blocks per weight stage
-constexpr int RAW_BYTES = FN * KW * BK / 2;     // 32 KB of e2m1 codes: 128-byte rows
-constexpr int SCL_BYTES = FN * 16;              // 4 KB of e4m3 scales (the same 4 k-blocks)
-constexpr int W_BYTES = RAW_BYTES + SCL_BYTES;  // one weight stage
+constexpr int SCL_BYTES = FN * 16;              // 4 KB of e4m3 scales (4 k-blocks)
+
+// Per projection: gate/up keeps 4 k-blocks of codes per weight stage
+// (128-byte rows); down takes 2 (64-byte rows) and spends the 32 KB saved on
+// staging its fp32 epilogue through shared memory (whole-row stores).
+template <bool GATED>
+struct WCfg {
+  static constexpr int KW = GATED ? 4 : 2;                 // k-blocks per weight stage
+  static constexpr int W_ROW = KW * BK / 2;                // bytes of codes per B row per stage
+  static constexpr int RAW_BYTES = FN * W_ROW;             // codes of a stage (swizzled rows)
+  static constexpr int W_BYTES = RAW_BYTES + SCL_BYTES;
+  static constexpr int STAGING = GATED ? 0 : 4 * 32 * 32 * 4;  // 4 epilogue warps x 32 x 32 fp32
+};
 constexpr int A_STAGES = 3;                     // A rows (mostly L2 hits)
 constexpr int W_STAGES = 2;                     // codes + scales (DRAM): 8 k-blocks
 constexpr int B_STAGES = 3;                     // converted B tiles
 constexpr int kConv = 8;                        // converter warps
 constexpr int kWProducer = 6;                   // the weight producer's warp
+constexpr int kStagingOffset = 5120;            // epilogue staging, past Smem
 constexpr int kConv0 = 7;                       // first converter warp
 constexpr int kThreads = 32 * (kConv0 + kConv);
 constexpr uint32_t TMEM_COLS = 512;             // 2 accumulators x FN
@@ -274,8 +284,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *stage_a = base;                                  // A_STAGES x 16 KB (1024-aligned)
   uint8_t *stage_b = stage_a + A_STAGES * A_BYTES;          // B_STAGES x 32 KB
   uint8_t *stage_w = stage_b + B_STAGES * B_BYTES;          // W_STAGES x (32 KB codes + 4 KB scales)
+  using WC = WCfg<GATED>;
+  constexpr int KW = WC::KW, W_ROW = WC::W_ROW, RAW_BYTES = WC::RAW_BYTES, W_BYTES = WC::W_BYTES;
   uint32_t *lut = reinterpret_cast<uint32_t *>(stage_w + W_STAGES * W_BYTES);
   Smem &sm = *reinterpret_cast<Smem *>(stage_w + W_STAGES * W_BYTES + 1024);
+  float *staging = reinterpret_cast<float *>(stage_w + W_STAGES * W_BYTES + 1024 + kStagingOffset);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -434,10 +447,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t *raw = stage_w + s * W_BYTES;
           uint8_t *scl = raw + RAW_BYTES;
           ptx::mbar_arrive_expect_tx(&sm.w_full[s], W_BYTES);
-          ptx::tma_load_3d(raw, &tmB0, &sm.w_full[s], kw * 128, n0, tl.e);
-          ptx::tma_load_3d(raw + RAW_BYTES / 2, GATED ? &tmB1 : &tmB0, &sm.w_full[s], kw * 128, n1, tl.e);
-          ptx::tma_load_3d(scl, &tmS0, &sm.w_full[s], kw * 16, n0, tl.e);
-          ptx::tma_load_3d(scl + SCL_BYTES / 2, GATED ? &tmS1 : &tmS0, &sm.w_full[s], kw * 16, n1, tl.e);
+          const int sx = (kw * KW >> 2) * 16;  // the scale box covers 4 k-blocks
+          ptx::tma_load_3d(raw, &tmB0, &sm.w_full[s], kw * W_ROW, n0, tl.e);
+          ptx::tma_load_3d(raw + RAW_BYTES / 2, GATED ? &tmB1 : &tmB0, &sm.w_full[s], kw * W_ROW, n1, tl.e);
+          ptx::tma_load_3d(scl, &tmS0, &sm.w_full[s], sx, n0, tl.e);
+          ptx::tma_load_3d(scl + SCL_BYTES / 2, GATED ? &tmS1 : &tmS0, &sm.w_full[s], sx, n1, tl.e);
           used[s] = true;
           last_parity[s] = ph;
         }
@@ -535,20 +549,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         } else {
+          // each 32 x 32 fp32 chunk through this warp's 4 KB of shared memory
+          // (row r's 16-byte piece j at j ^ (r % 8)), so that every global
+          // store writes four whole 128-byte row segments
           const float rw = (live && p.row_weight) ? p.row_weight[row] : 1.0f;
-          float *yrow = (float *)p.out + (long)row * p.N + tl.n_blk * FN;
+          float *stg = staging + q * 32 * 32;
+          const int row0 = tl.m0 + q * 32;
+          const int rr = lane >> 3, ff = lane & 7;
+          const int ncol0 = tl.n_blk * FN;
 #pragma unroll 1
           for (int c = 0; c < FN; c += 32) {
             uint32_t v[32];
             ptx::tmem_ld32(tbase + c, v);
             ptx::tmem_ld_wait();
-            if (live) {
-              float4 *dst = reinterpret_cast<float4 *>(yrow + c);
 #pragma unroll
-              for (int j = 0; j < 8; ++j)
-                dst[j] = make_float4(__uint_as_float(v[4 * j]) * rw, __uint_as_float(v[4 * j + 1]) * rw,
-                                     __uint_as_float(v[4 * j + 2]) * rw, __uint_as_float(v[4 * j + 3]) * rw);
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<float4 *>(stg + lane * 32 + ((j ^ (lane & 7)) << 2)) =
+                  make_float4(__uint_as_float(v[4 * j]) * rw, __uint_as_float(v[4 * j + 1]) * rw,
+                              __uint_as_float(v[4 * j + 2]) * rw, __uint_as_float(v[4 * j + 3]) * rw);
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int r = 4 * i + rr;
+              const float4 val = *reinterpret_cast<const float4 *>(stg + r * 32 + ((ff ^ (r & 7)) << 2));
+              if (row0 + r < tl.end)
+                *reinterpret_cast<float4 *>((float *)p.out + (long)(row0 + r) * p.N + ncol0 + c + ff * 4) = val;
             }
+            __syncwarp();
           }
         }
       }
@@ -587,13 +614,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         const uint8_t *w = stage_w + sw * W_BYTES;
-        const int raw_off = r0 * 128 + (((2 * kq + (g >> 1)) ^ (r0 & 7)) << 4) + (g & 1) * 8;
+        // the group's 16-byte chunk, swizzled as the TMA stored it
+        const int chunk = 2 * kq + (g >> 1);
+        const int raw_off = r0 * W_ROW + ((KW == 4 ? chunk ^ (r0 & 7) : chunk ^ ((r0 >> 1) & 3)) << 4) + (g & 1) * 8;
         uint2 qv[JOBS];
         uint32_t sc[JOBS];
 #pragma unroll
         for (int j = 0; j < JOBS; ++j) {
-          qv[j] = *reinterpret_cast<const uint2 *>(w + raw_off + j * ROWS_PER_PASS * 128);
-          sc[j] = w[scl_off + kq * 4 + j * ROWS_PER_PASS * 16];
+          qv[j] = *reinterpret_cast<const uint2 *>(w + raw_off + j * ROWS_PER_PASS * W_ROW);
+          sc[j] = w[scl_off + (kb & 3) * 4 + j * ROWS_PER_PASS * 16];
         }
         if (kq == KW - 1) {
           __syncwarp();
@@ -631,9 +660,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-constexpr size_t kSmemBytes = 1024 + (size_t)A_STAGES * A_BYTES + (size_t)B_STAGES * B_BYTES +
-                              (size_t)W_STAGES * W_BYTES + 1024 + sizeof(Smem);
-static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+template <bool GATED>
+constexpr size_t fp4_smem_bytes() {
+  return 1024 + (size_t)A_STAGES * A_BYTES + (size_t)B_STAGES * B_BYTES + (size_t)W_STAGES * WCfg<GATED>::W_BYTES +
+         1024 + kStagingOffset + WCfg<GATED>::STAGING;
+}
+static_assert(sizeof(Smem) <= kStagingOffset, "the epilogue staging follows the barriers and tile list");
+static_assert(fp4_smem_bytes<true>() <= 232448 && fp4_smem_bytes<false>() <= 232448, "shared memory per CTA");
 
 // A: [rows, K] bf16 (or the gather source); codes [E, Nw, K/2] bytes and
 // scales [E, Nw, K/16] bytes for b0/s0 (and b1/s1 when gated).
@@ -644,10 +677,11 @@ moe_status launch_fp4(const Params &p, const void *a, const void *b0, const void
   const uint64_t K = (uint64_t)p.K;
   if (!tma_map_bf16(&ta, a, 2, K, (uint64_t)(p.row_token ? p.src_rows : p.rows), 1, p.row_token ? 1 : TILE_M))
     return MOE_ERR_CUDA;
-  if (!tma_map_u8(&tb0, b0, K / 2, (uint64_t)Nw, (uint64_t)p.E, 128, FN / 2, true)) return MOE_ERR_CUDA;
+  constexpr int W_ROW = WCfg<GATED>::W_ROW;
+  if (!tma_map_u8(&tb0, b0, K / 2, (uint64_t)Nw, (uint64_t)p.E, W_ROW, FN / 2, W_ROW)) return MOE_ERR_CUDA;
   if (!tma_map_u8(&ts0, s0, K / 16, (uint64_t)Nw, (uint64_t)p.E, 16, FN / 2)) return MOE_ERR_CUDA;
   if (GATED) {
-    if (!tma_map_u8(&tb1, b1, K / 2, (uint64_t)Nw, (uint64_t)p.E, 128, FN / 2, true)) return MOE_ERR_CUDA;
+    if (!tma_map_u8(&tb1, b1, K / 2, (uint64_t)Nw, (uint64_t)p.E, W_ROW, FN / 2, W_ROW)) return MOE_ERR_CUDA;
     if (!tma_map_u8(&ts1, s1, K / 16, (uint64_t)Nw, (uint64_t)p.E, 16, FN / 2)) return MOE_ERR_CUDA;
   } else {
     tb1 = tb0;
@@ -657,6 +691,7 @@ moe_status launch_fp4(const Params &p, const void *a, const void *b0, const void
   MOE_CUDA_TRY(cudaGetDevice(&dev));
   MOE_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   auto kern = tc_fp4_gemm<GATED, F16>;
+  constexpr size_t kSmemBytes = fp4_smem_bytes<GATED>();
   MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes));
   const long ub = ((long)(p.rows + TILE_M - 1) / TILE_M + (p.offsets ? p.E : 0)) * p.n_tiles;  // tile bound
   if (ub <= 0) return MOE_OK;

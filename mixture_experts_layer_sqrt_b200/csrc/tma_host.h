@@ -40,10 +40,11 @@ inline bool tma_map_bf16(CUtensorMap *m, const void *ptr, int rank, uint64_t d0,
 }
 
 // uint8 tensor [d2][d1][d0] (d0 contiguous, in bytes); box {box0, box_rows, 1};
-// rows land box0 bytes apart, or with swizzle128 (box0 = 128) 16-byte chunk c
-// of row r lands at chunk c ^ (r % 8) of the row; zero fill outside the tensor.
+// rows land box0 bytes apart; with swizzle_bytes = 128 (box0 = 128) 16-byte
+// chunk c of row r lands at chunk c ^ (r % 8) of the row, with 64 (box0 = 64)
+// at chunk c ^ ((r / 2) % 4); zero fill outside the tensor.
 inline bool tma_map_u8(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
-                       uint32_t box_rows, bool swizzle128 = false) {
+                       uint32_t box_rows, int swizzle_bytes = 0) {
   auto fn = tma_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {d0, d1, d2};
@@ -51,7 +52,10 @@ inline bool tma_map_u8(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1
   cuuint32_t box[3] = {box0, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                  : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                        : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
