@@ -24,20 +24,18 @@
 // Three rings, because their data have different latencies and lifetimes:
 //   A rows      (16 KB per k-block, 3 stages)  mostly L2 hits; held until the
 //               MMAs that read them complete.
-//   weights     (32 KB of codes + 4 KB of scales per 4 k-blocks, 2 stages)
-//               from DRAM, in 128-byte rows (a TMA copy costs per row moved:
-//               32-byte code rows and 16-byte scale rows every k-block made
-//               the copies, not the MMAs or the expansion, set the pace);
-//               freed as soon as every converter warp holds the bytes in
-//               registers.
+//   weights     (2 stages, from DRAM)  gate/up: 32 KB of codes in 128-byte
+//               swizzled rows + 4 KB of scales per 4 k-blocks; down: 16 KB of
+//               codes in 64-byte swizzled rows per 2 k-blocks, the 32 KB saved
+//               holding the fp32 epilogue's staging.  Freed as soon as every
+//               converter warp holds the bytes in registers.
 //   converted B (32 KB per k-block, 3 stages)  written by the converters,
-//               held until the MMAs that read it complete.  Each stage's round
-//               trip (expansion, hand-off, MMA issue to completion, hand-off
-//               back) takes ~2600 cycles against 512 of MMA work, so the
-//               depth of this ring, not the A or weight rings, sets the pace.
-// (One shared A + weights ring, released only after the MMA, left both the
-// MMAs and the converters waiting on copies: each alone ran at ~45% of its
-// own rate.)
+//               held until the MMAs that read it complete.
+// With one shared A + weights ring released only after the MMA, gate/up took
+// 1.55 ms on the sqrt-softplus layer; now 1.36-1.39.  The k-block period
+// (~1200 cycles) is the MMA thread issuing its four MMAs (~740) plus waiting
+// for A and for the slowest converter warp; deeper A or converted-B rings
+// measured no faster.
 //
 // Roles (480 threads per CTA):
 //   warp 0       TMA producer of A rows (128 x 64 per k-block; or a 4-row
@@ -45,7 +43,9 @@
 //   warp 1       TMEM owner; one thread issues the MMAs (A from its ring, B
 //                from the converted ring) and commits both stages back.
 //   warps 2-5    epilogue: TMEM -> registers -> SwiGLU or routing weight ->
-//                global stores; two 256-column accumulators overlap tiles.
+//                global stores (fp32 y through 4 KB of shared memory per
+//                warp, so that every store writes whole 128-byte row
+//                segments); two 256-column accumulators overlap tiles.
 //   warp 6       TMA producer of the packed codes and scales.
 //   warps 7-14   converters: codes + scales -> swizzled 16-bit B tile, one
 //                arrival per warp.
@@ -97,7 +97,7 @@ struct WCfg {
   static constexpr int STAGING = GATED ? 0 : 4 * 32 * 32 * 4;  // 4 epilogue warps x 32 x 32 fp32
 };
 constexpr int A_STAGES = 3;                     // A rows (mostly L2 hits)
-constexpr int W_STAGES = 2;                     // codes + scales (DRAM): 8 k-blocks
+constexpr int W_STAGES = 2;                     // codes + scales (DRAM)
 constexpr int B_STAGES = 3;                     // converted B tiles
 constexpr int kConv = 8;                        // converter warps
 constexpr int kWProducer = 6;                   // the weight producer's warp
