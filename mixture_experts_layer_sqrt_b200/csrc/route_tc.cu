@@ -229,8 +229,10 @@ __global__ void __launch_bounds__(kRThreads, 1)
   }
 }
 
-// One warp per token: copy its logit row to shared memory, then select.
+// One warp per token: copy its logit row to shared memory, then select with
+// each lane's keys cached in registers (NJ = keys per lane, E <= 32 NJ).
 constexpr int kSelWarps = 8;
+template <int NJ>
 __global__ void __launch_bounds__(32 * kSelWarps) route_select_kernel(int T, int E, int ld, int k, int gate,
                                                                      const float *__restrict__ logits,
                                                                      const float *__restrict__ bias,
@@ -245,7 +247,7 @@ __global__ void __launch_bounds__(32 * kSelWarps) route_select_kernel(int T, int
     const float *src = logits + t * ld;
     for (int e = lane; e < E; e += 32) lg[e] = src[e];
     __syncwarp();
-    select_topk(lg, t, E, k, gate, bias, bias_vl, image_mask, topk_idx, topk_w, lane);
+    select_topk_cached<NJ>(lg, t, E, k, gate, bias, bias_vl, image_mask, topk_idx, topk_w, lane);
     __syncwarp();
   }
 }
@@ -318,7 +320,11 @@ moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void 
   long sel_blocks = ((long)T + kSelWarps - 1) / kSelWarps;
   if (sel_blocks > (long)sms * 8) sel_blocks = (long)sms * 8;
   const bool sel = c.gate != MOE_GATE_SOFTMAX_TOPK_RENORM;  // softmax: the logit bias is already in the logits
-  route_select_kernel<<<(unsigned)sel_blocks, 32 * kSelWarps, (size_t)kSelWarps * p.ld * sizeof(float), s>>>(
+  auto sel_kern = route_select_kernel<16>;  // up to 512 experts
+  if (p.E <= 64) sel_kern = route_select_kernel<2>;
+  else if (p.E <= 128) sel_kern = route_select_kernel<4>;
+  else if (p.E <= 256) sel_kern = route_select_kernel<8>;
+  sel_kern<<<(unsigned)sel_blocks, 32 * kSelWarps, (size_t)kSelWarps * p.ld * sizeof(float), s>>>(
       T, p.E, p.ld, p.k, p.gate, scratch, sel ? bias : nullptr, sel ? bias_vl : nullptr, image_mask, topk_idx,
       topk_w);
   MOE_LAUNCH_CHECK();
