@@ -119,17 +119,11 @@ class ClockSampler:
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
             self.stop_evt = threading.Event()
 
-            def power_w():
-                try:
-                    return pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
-                except Exception:
-                    return None
-
             def loop():
                 while not self.stop_evt.is_set():
                     try:
                         self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
-                                             pynvml.nvmlDeviceGetCurrentClocksEventReasons(h), power_w()))
+                                             pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)))
                     except Exception:
                         pass
                     self.stop_evt.wait(period_s)
@@ -151,17 +145,10 @@ class ClockSampler:
             self.thread.join(timeout=5)
             if not self.samples:
                 return None
-            sm = [float(c) for c, _, _ in self.samples]
-            reasons = sorted({n for _, r, _ in self.samples for n, bit in self.REASONS if r & bit})
-            watts = [w for _, _, w in self.samples if w is not None]
-            # NVML's SM clock can read the maximum while the power limit slows
-            # the tensor-core kernels further (clock64 against %globaltimer
-            # inside the gate/up GEMM: ~1.46 GHz at a reading of 1965 MHz), so
-            # the board power is reported beside it
+            sm = [float(c) for c, _ in self.samples]
+            reasons = sorted({n for _, r in self.samples for n, bit in self.REASONS if r & bit})
             return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(self.max_mhz), "reasons": reasons,
-                    "samples": len(self.samples),
-                    "power_w_median": statistics.median(watts) if watts else None,
-                    "power_w_max": max(watts) if watts else None, "source": "nvml, 5 ms"}
+                    "samples": len(self.samples), "source": "nvml, 5 ms"}
         if self.proc is None:
             return None
         self.proc.terminate()
