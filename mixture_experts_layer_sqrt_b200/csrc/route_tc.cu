@@ -10,8 +10,9 @@
 // logits.  Sqrt mode: selection on s + bias / bias_vl, weights
 // sqrt(softplus(s)) of the raw score ("5A · MoE fine-grained" sec. 1, 3).
 //
-// One CTA per 128 tokens, 192 threads: warp 0 loads x (128 x 64) and W_r
-// (E_pad x 64, in 128-row boxes) per k-block with TMA; warp 1 issues
+// One CTA per 128 tokens and E_pad experts, 192 threads: warp 0 loads x
+// (128 x 64) and the CTA's own W_r rows (E_pad x 64, in equal boxes of up
+// to 128 rows) per k-block with TMA; warp 1 issues
 // tcgen05.mma (M=128, N <= 256 per instruction, two instructions when
 // E_pad > 256) into fp32 TMEM accumulators of E_pad columns -- up to four,
 // fed by interleaved k-blocks and summed in a fixed order afterwards, which
@@ -42,7 +43,7 @@ constexpr uint64_t kRDrainNs = 200000000ull;
 struct RParams {
   int T, D, E;
   int E_pad;  // expert columns of one CTA (a multiple of 16); CTA (x, y) covers [y * E_pad, (y + 1) * E_pad)
-  int k, gate, stages, b_rows;
+  int k, gate, stages, b_rows, w_box;  // W_r rows per stage, and per TMA box
   float *logits;  // [T, ld] fp32 out (router logit bias included in softmax mode)
   int ld;         // logit row stride: E_pad rounded up to whole 32-column chunks
   int n_acc;  // independent accumulators over interleaved k-blocks (shorter fp32 sums)
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem_base = sm.tmem_base;
   const int k_blocks = p.D / RBK;
-  const int n_boxes = p.b_rows / 128;
+  const int n_boxes = p.b_rows / p.w_box;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -140,7 +141,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
         uint8_t *a = base + (size_t)s * stage_bytes;
         ptx::tma_load_2d(a, &tmX, &sm.full[s], kb * RBK, m0);
         for (int j = 0; j < n_boxes; ++j)
-          ptx::tma_load_2d(a + a_bytes + j * 16384, &tmW, &sm.full[s], kb * RBK, e0 + j * 128);
+          ptx::tma_load_2d(a + a_bytes + j * p.w_box * 128, &tmW, &sm.full[s], kb * RBK, e0 + j * p.w_box);
         last = kb;
       }
       // drain the copies still in flight (the last `stages` k-blocks)
@@ -244,8 +245,14 @@ __global__ void __launch_bounds__(32 * kSelWarps) route_select_kernel(int T, int
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float *lg = rows + warp * ld;
   for (long t = (long)blockIdx.x * kSelWarps + warp; t < T; t += (long)gridDim.x * kSelWarps) {
+    // all of the row's loads in flight at once (one L2 round trip, not NJ)
     const float *src = logits + t * ld;
-    for (int e = lane; e < E; e += 32) lg[e] = src[e];
+    float v[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) v[j] = lane + 32 * j < E ? src[lane + 32 * j] : 0.0f;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j)
+      if (lane + 32 * j < E) lg[lane + 32 * j] = v[j];
     __syncwarp();
     select_topk_cached<NJ>(lg, t, E, k, gate, bias, bias_vl, image_mask, topk_idx, topk_w, lane);
     __syncwarp();
@@ -292,7 +299,14 @@ moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void 
       break;
     }
   p.E_pad = e_pad_all / split;
-  p.b_rows = (p.E_pad + 127) / 128 * 128;
+  // W_r rows per stage: exactly this CTA's E_pad columns, in at most 8 equal
+  // boxes of 128, 64, 32 or 16 rows (else 128-row boxes past E_pad, zero
+  // filled beyond E), so that no CTA also loads its neighbour's rows.
+  p.w_box = 0;
+  for (int b = 128; b >= 16 && !p.w_box; b >>= 1)
+    if (p.E_pad % b == 0 && p.E_pad / b <= 8) p.w_box = b;
+  if (!p.w_box) p.w_box = 128;
+  p.b_rows = (p.E_pad + p.w_box - 1) / p.w_box * p.w_box;
   p.k = c.top_k;
   p.gate = c.gate;
   p.n_acc = p.E_pad <= 128 ? 4 : (p.E_pad <= 256 ? 2 : 1);
@@ -311,7 +325,7 @@ moe_status launch_route_tc(const MoEConfig &c, int T, const void *x, const void 
   p.stages = stages > kMaxStages ? kMaxStages : stages;
   CUtensorMap tx, tw;
   if (!tma_map_bf16(&tx, x, 2, (uint64_t)p.D, (uint64_t)T, 1)) return MOE_ERR_CUDA;
-  if (!tma_map_bf16(&tw, w_router, 2, (uint64_t)p.D, (uint64_t)p.E, 1)) return MOE_ERR_CUDA;
+  if (!tma_map_bf16(&tw, w_router, 2, (uint64_t)p.D, (uint64_t)p.E, 1, (uint32_t)p.w_box)) return MOE_ERR_CUDA;
   const size_t smem = 1024 + (size_t)p.stages * stage_bytes + sizeof(RSmem);
   const dim3 grid((unsigned)m_tiles, (unsigned)split);
   MOE_CUDA_TRY(cudaFuncSetAttribute(tc_route_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
